@@ -1,0 +1,351 @@
+"""Pins for the oracle: checks against what the page and the mathematics fix.
+
+Each pin compares the oracle with something other than itself: a published
+test vector, a closed form, an invariant, a textbook or library routine, or
+brute force on tiny inputs. The "planted" tests at the end put a plausible
+mistake into the oracle (on the CPU, via monkeypatch) and check that the pin
+meant to catch it fails.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import sws_oracle as so
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------- pins ----
+
+def pin_splitmix64():
+    with open(os.path.join(GOLDEN, "splitmix64_seed0.txt")) as f:
+        want = [int(x, 16) for x in f.read().split() if x.startswith("0x")]
+    state, got = 0, []
+    for _ in want:
+        state, z = so.splitmix64(state)
+        got.append(z)
+    assert got == want
+
+
+def pin_hadamard():
+    for d in (1, 2, 4, 8, 16, 64, 128):
+        H = so.sylvester_hadamard(d)
+        formula = np.array([[(-1) ** bin(r & c).count("1") for c in range(d)] for r in range(d)], dtype=float)
+        assert np.array_equal(H, formula)
+        assert np.array_equal(H @ H.T, d * np.eye(d))
+
+
+def pin_srht_draws():
+    for d, k, seed in ((64, 16, 0), (128, 32, 1), (128, 128, 7), (8, 3, 99)):
+        signs, cols = so.srht_draws(d, k, seed)
+        assert set(signs) <= {1, -1} and len(signs) == d
+        assert len(cols) == k and len(set(cols)) == k and all(0 <= c < d for c in cols)
+        assert so.srht_draws(d, k, seed) == (signs, cols)
+    _, perm = so.srht_draws(32, 32, 5)
+    assert sorted(perm) == list(range(32))
+
+
+def pin_srht_orthogonal_when_k_equals_d():
+    """k = d: H_d is orthogonal, so the sketch keeps every inner product (Parseval)."""
+    for d, seed in ((64, 3), (128, 11)):
+        Hd = so.srht_matrix(d, d, seed)
+        assert np.allclose(Hd @ Hd.T, np.eye(d), atol=1e-12)
+        u, v = rng.standard_normal(d), rng.standard_normal(d)
+        assert abs((u @ Hd) @ (v @ Hd) - u @ v) <= 1e-11 * np.linalg.norm(u) * np.linalg.norm(v)
+
+
+def pin_srht_unbiased():
+    """§6.2: the sketch preserves inner products in expectation. Averaging
+    (u H_d)(v H_d)^T over every choice of the k columns gives u.v exactly."""
+    for d, k in ((16, 1), (8, 3), (8, 8)):
+        signs = [1 if x > 0 else -1 for x in rng.standard_normal(d)]
+        u, v = rng.standard_normal(d), rng.standard_normal(d)
+        vals = [(u @ so.srht_from_draws(signs, c)) @ (v @ so.srht_from_draws(signs, c))
+                for c in itertools.combinations(range(d), k)]
+        assert abs(np.mean(vals) - u @ v) < 1e-12 * max(1.0, abs(u @ v)) + 1e-12
+
+
+def pin_srht_concentration():
+    """§6.2 bound |(u^T H)(H^T v) - u^T v| <= eps |u||v|: over many seeds the
+    error shrinks like 1/sqrt(k) and its mean is ~0 (statistical, loose)."""
+    d = 128
+    u, v = rng.standard_normal(d), rng.standard_normal(d)
+    scale = np.linalg.norm(u) * np.linalg.norm(v)
+    rms = {}
+    for k in (8, 32, 128):
+        errs = np.array([((u @ (H := so.srht_matrix(d, k, s))) @ (v @ H) - u @ v) / scale for s in range(300)])
+        assert abs(errs.mean()) < 4 * errs.std() / math.sqrt(len(errs)) + 1e-12
+        rms[k] = math.sqrt((errs ** 2).mean())
+    assert rms[128] < 1e-12
+    assert rms[8] > rms[32] and 1.3 < rms[8] / rms[32] < 3.0  # ~ sqrt(32/8) = 2
+
+
+def pin_block_means_identity():
+    """§2 vs §3.1: the literal double sum of A_true equals q_bar . k_bar / sqrt(d)."""
+    n, B, d = 12, 3, 5
+    Q, K = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    lit = so.a_true_literal(Q, K, B)
+    via = so.a_true(so.block_means(Q, B), so.block_means(K, B))
+    assert np.allclose(lit, via, rtol=1e-12, atol=1e-13)
+
+
+def pin_block_means_partial():
+    """A partial last block averages only the rows it holds (reading R1)."""
+    X = rng.standard_normal((7, 4))
+    m = so.block_means(X, 3)
+    assert m.shape == (3, 4)
+    assert np.allclose(m[2], X[6])
+    assert np.allclose(m[1], (X[3] + X[4] + X[5]) / 3)
+
+
+def pin_sws_special_case():
+    """B = 1 and k = d: the sketched scores are exactly Q K^T / sqrt(d) (causal part)."""
+    n, d = 20, 16
+    Q, K = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    Hd = so.srht_matrix(d, d, 4)
+    S = so.sketch_scores(so.sketch_project(so.block_means(Q, 1), Hd), so.sketch_project(so.block_means(K, 1), Hd))
+    ref = np.asarray(torch.from_numpy(Q) @ torch.from_numpy(K).T / math.sqrt(d))
+    low = np.tril_indices(n)
+    assert np.allclose(S[low], ref[low], rtol=1e-11, atol=1e-11)
+    assert np.all(np.isneginf(S[np.triu_indices(n, 1)]))
+
+
+def pin_block_attention():
+    S = so.sketch_scores(rng.standard_normal((9, 4)), rng.standard_normal((9, 4)))
+    A = so.block_attention(S)
+    assert np.allclose(A.sum(axis=1), 1.0, atol=1e-14)
+    assert np.all(A[np.triu_indices(9, 1)] == 0.0)
+    assert A[0, 0] == 1.0
+    ref = torch.softmax(torch.from_numpy(np.where(np.isneginf(S), -np.inf, S)), dim=1).numpy()
+    assert np.allclose(A, ref, atol=1e-14)
+
+
+def pin_walk_power():
+    """(A)^s as a matrix power: numpy's matrix_power and repeated squaring agree."""
+    A = so.block_attention(so.sketch_scores(rng.standard_normal((10, 4)), rng.standard_normal((10, 4))))
+    for s in (1, 2, 3, 8):
+        assert np.allclose(so.walk_matrix(A, s), np.linalg.matrix_power(A, s), rtol=1e-12, atol=1e-15)
+    sq = A @ A
+    sq = sq @ sq
+    sq = sq @ sq
+    assert np.allclose(so.walk_matrix(A, 8), sq, rtol=1e-12, atol=1e-15)
+
+
+def pin_walk_path_sum():
+    """§4: R^l[i, j] sums, over every walk i -> ... -> j, the product of the
+    per-step block attention weights: s steps with layer 0's matrix, then s
+    steps with layer 1's. Enumerated path by path on a tiny case."""
+    b, s = 3, 2
+    A0 = so.block_attention(so.sketch_scores(rng.standard_normal((b, 3)), rng.standard_normal((b, 3))))
+    A1 = so.block_attention(so.sketch_scores(rng.standard_normal((b, 3)), rng.standard_normal((b, 3))))
+    R = so.walk_update(so.walk_update(None, so.walk_matrix(A0, s)), so.walk_matrix(A1, s))
+    mats = [A0] * s + [A1] * s
+    for i in range(b):
+        for j in range(b):
+            tot = 0.0
+            for mid in itertools.product(range(b), repeat=len(mats) - 1):
+                path = (i,) + mid + (j,)
+                p = 1.0
+                for t, M in enumerate(mats):
+                    p *= M[path[t], path[t + 1]]
+                tot += p
+            assert abs(R[i, j] - tot) < 1e-14
+
+
+def pin_walk_invariants():
+    """R^l stays row-stochastic and lower-triangular across layers (real inputs)."""
+    import sws_inputs as W
+    w = W.TINY
+    Hd = so.srht_matrix(w.d, w.k, w.seed)
+    st = so.PrefillState()
+    for layer in range(w.layers):
+        Q, K, V = W.prefill_layer_inputs(w, layer)
+        R = so.prefill_layer(Q.numpy(), K.numpy(), V.numpy(), Hd, w.B, w.s, w.density, st, attention_blocks=None)[0]["R"]
+        assert np.allclose(R.sum(axis=1), 1.0, atol=1e-12)
+        assert np.all(R[np.triu_indices(w.b, 1)] == 0.0)
+        assert np.all(R[np.tril_indices(w.b)] > 0.0)
+
+
+def pin_top_tau_bruteforce():
+    """Brute force: the chosen set maximises the sum of the row over all sets
+    of size tau; among maximisers it takes the lowest indices (tie rule R6)."""
+    r = np.random.default_rng(7)
+    for trial in range(300):
+        m = int(r.integers(1, 10))
+        row = r.integers(0, 4, size=m).astype(float)  # small range: many ties
+        tau = int(r.integers(1, m + 1))
+        got = tuple(int(x) for x in so.top_tau_row(row, tau))
+        best = max(sum(row[list(c)]) for c in itertools.combinations(range(m), tau))
+        cands = [c for c in itertools.combinations(range(m), tau) if sum(row[list(c)]) == best]
+        assert got == min(cands), (row, tau, got)
+
+
+def pin_tau():
+    table = {0: 1, 3: 1, 4: 1, 5: 2, 9: 2, 10: 3, 255: 52, 1023: 205}
+    for i, t in table.items():
+        assert so.tau_of_row(i, 1, 5) == t
+    assert so.tau_of_row(9, 1, 10) == 1 and so.tau_of_row(10, 1, 10) == 2
+    assert all(so.tau_of_row(i, 1, 1) == i + 1 for i in range(50))
+    assert so.csr_nnz(16, 1, 5) == 34 and so.csr_nnz(1024, 1, 5) == 105370
+
+
+def _dense_causal_sdpa(Q, K, V):
+    q, k, v = (torch.from_numpy(np.asarray(x, dtype=np.float64))[None, None] for x in (Q, K, V))
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)[0, 0].numpy()
+
+
+def pin_attention_dense_limit():
+    """Density 100%: every causal block is kept, so the sparse attention equals
+    dense causal softmax attention (torch's SDPA in fp64)."""
+    n, d, B = 40, 8, 8
+    Q, K, V = (rng.standard_normal((n, d)) for _ in range(3))
+    b = n // B
+    row_ptr, col_idx = so.select_top_tau(np.tril(np.ones((b, b))), 1, 1)
+    O = so.sparse_attention(Q, K, V, row_ptr, col_idx, B)
+    assert np.allclose(O, _dense_causal_sdpa(Q, K, V), rtol=1e-12, atol=1e-12)
+    # ragged n (partial last block)
+    n2 = 37
+    b2 = -(-n2 // B)
+    rp, ci = so.select_top_tau(np.tril(np.ones((b2, b2))), 1, 1)
+    O2 = so.sparse_attention(Q[:n2], K[:n2], V[:n2], rp, ci, B)
+    assert np.allclose(O2, _dense_causal_sdpa(Q[:n2], K[:n2], V[:n2]), rtol=1e-12, atol=1e-12)
+
+
+def pin_attention_special_cases():
+    n, d, B = 24, 4, 4
+    Q, K = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    Vc = np.tile(rng.standard_normal(d), (n, 1))
+    b = n // B
+    rp, ci = so.select_top_tau(rng.random((b, b)), 1, 3)
+    assert np.allclose(so.sparse_attention(Q, K, Vc, rp, ci, B), Vc, atol=1e-13)  # constant V
+    V = rng.standard_normal((n, d))
+    O = so.sparse_attention(Q, K, V, rp, ci, B)
+    assert np.allclose(O[0], V[0])  # the first token only sees itself
+    # a query block whose only key block is block 0, strictly below it: plain softmax over block 0
+    rp1 = np.array([0, 1, 2])
+    ci1 = np.array([0, 0])
+    O1 = so.sparse_attention(Q[:8], K[:8], V[:8], rp1, ci1, B)
+    w = np.exp(Q[4:8] @ K[:4].T / math.sqrt(d))
+    assert np.allclose(O1[4:8], (w / w.sum(axis=1, keepdims=True)) @ V[:4])
+
+
+def pin_one_hop_when_s1():
+    """s = 1 and one layer: the selection is the top-tau of the sketched scores
+    themselves (the row softmax is monotone)."""
+    S = so.sketch_scores(rng.standard_normal((30, 4)), rng.standard_normal((30, 4)))
+    R = so.walk_update(None, so.walk_matrix(so.block_attention(S), 1))
+    rp, ci = so.select_top_tau(R, 1, 5)
+    for i in range(30):
+        raw = S[i, :i + 1]
+        want = np.sort(np.argsort(-raw, kind="stable")[:so.tau_of_row(i, 1, 5)])
+        assert np.array_equal(ci[rp[i]:rp[i + 1]], want)
+
+
+def pin_gqa_mapping():
+    """Query head h reads KV head h // (hq / hkv)."""
+    n, d, B = 32, 8, 8
+    Q = rng.standard_normal((4, n, d))
+    K, V = rng.standard_normal((2, n, d)), rng.standard_normal((2, n, d))
+    Hd = so.srht_matrix(d, 4, 1)
+    full = so.prefill_layer(Q, K, V, Hd, B, 2, (1, 2), so.PrefillState())
+    for h in range(4):
+        one = so.prefill_layer(Q[h:h + 1], K[h // 2:h // 2 + 1], V[h // 2:h // 2 + 1], Hd, B, 2, (1, 2),
+                               so.PrefillState())[0]
+        assert np.array_equal(one["col_idx"], full[h]["col_idx"])
+        assert np.allclose(one["O"], full[h]["O"])
+
+
+def pin_decode():
+    """Decode (readings R7, R8): block means by count; rho^0 / s is the log of a
+    softmax; with s = 1 and one layer the choice is the top-tau of the row
+    logits; s does not change the ranking; all blocks kept = dense attention."""
+    hq, hkv, d, B, L = 2, 1, 8, 4, 19
+    Kc, Vc = rng.standard_normal((hkv, 24, d)), rng.standard_normal((hkv, 24, d))
+    q = rng.standard_normal((hq, d))
+    Hd = so.srht_matrix(d, 4, 2)
+    means = so.decode_block_means(Kc[0], L, B)
+    assert means.shape == (5, d) and np.allclose(means[4], Kc[0, 16:19].mean(axis=0))
+    assert np.allclose(means[1], Kc[0, 4:8].sum(axis=0) / 4)
+    rho1, z, sel1 = so.decode_layer_select(q, Kc, L, Hd, B, 1, (2, 5), None)
+    assert np.allclose(np.exp(rho1).sum(axis=1), 1.0, atol=1e-13)
+    tau = so.tau_of_row(4, 2, 5)
+    for h in range(hq):
+        assert np.array_equal(sel1[h], np.sort(np.argsort(-z[h], kind="stable")[:tau]))
+    rho8, _, sel8 = so.decode_layer_select(q, Kc, L, Hd, B, 8, (2, 5), None)
+    assert np.allclose(rho8, 8 * rho1)
+    assert all(np.array_equal(a, b) for a, b in zip(sel1, sel8))
+    o = so.decode_attention(q[0], Kc[0], Vc[0], L, range(5), B)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[0])[None, None, None], torch.from_numpy(Kc[0, :L])[None, None],
+        torch.from_numpy(Vc[0, :L])[None, None])[0, 0, 0].numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin()
+
+
+# ------------------------------------------------------- planted mistakes ----
+
+PLANTED = {
+    "hadamard_scale_dropped": ("srht_from_draws",
+                               lambda orig: (lambda signs, cols: orig(signs, cols) / math.sqrt(len(signs) / len(cols))),
+                               pin_srht_unbiased),
+    "splitmix_constant": ("splitmix64", lambda orig: (lambda s: (orig(s)[0], orig(s)[1] ^ 1)), pin_splitmix64),
+    "partial_block_divides_by_B": ("block_means", lambda orig: (
+        lambda X, B: np.stack([np.asarray(X, float)[i * B:(i + 1) * B].sum(0) / B for i in range(-(-len(X) // B))])),
+        pin_block_means_partial),
+    "no_causal_block_mask": ("block_attention", lambda orig: (
+        lambda S: (lambda e: e / e.sum(1, keepdims=True))(np.exp(np.where(np.isneginf(S), 0.0, S)))),
+        pin_block_attention),
+    "walk_power_off_by_one": ("walk_matrix", lambda orig: (lambda A, s, mode="matrix_power": orig(A, s + 1, mode)),
+                              pin_walk_power),
+    "walk_operands_swapped": ("walk_update", lambda orig: (lambda R, M: M.copy() if R is None else M @ R),
+                              pin_walk_path_sum),
+    "ties_to_higher_index": ("top_tau_row", lambda orig: (
+        lambda row, tau: np.sort(np.lexsort((-np.arange(len(row)), -row))[:tau])), pin_top_tau_bruteforce),
+    "tau_floor": ("tau_of_row", lambda orig: (lambda i, num, den: max(1, (i + 1) * num // den)), pin_tau),
+    "no_causal_mask_in_diagonal_block": ("sparse_attention_block", lambda orig: (
+        lambda Q, K, V, i, blocks, B: orig(Q, K, V, i, blocks, B) if i == 0 else
+        (lambda u: (lambda s: (np.exp(s - s.max(1, keepdims=True)) @ V[u]) /
+                    np.exp(s - s.max(1, keepdims=True)).sum(1, keepdims=True))(
+            Q[i * B:(i + 1) * B] @ K[u].T / math.sqrt(Q.shape[1])))(
+            np.concatenate([np.arange(j * B, min(len(Q), (j + 1) * B)) for j in blocks]))),
+        pin_attention_dense_limit),
+    "attention_scale_1_over_d": ("sparse_attention_block", lambda orig: (
+        lambda Q, K, V, i, blocks, B: orig(np.asarray(Q) / math.sqrt(Q.shape[1]), K, V, i, blocks, B)),
+        pin_attention_dense_limit),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLANTED))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, make, pin = PLANTED[name]
+    orig = getattr(so, attr)
+    monkeypatch.setattr(so, attr, make(orig))
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_planted_decode_lse_dropped(monkeypatch):
+    """Dropping logsumexp leaves the decode ranking unchanged; the softmax
+    normalisation check inside pin_decode still catches it."""
+    orig = so.decode_layer_select
+
+    def wrong(q_tok, Kc, length, Hd, B, s, density, rho_prev):
+        rho, z, sel = orig(q_tok, Kc, length, Hd, B, s, density, rho_prev)
+        return s * z + (0.0 if rho_prev is None else rho_prev), z, sel
+
+    monkeypatch.setattr(so, "decode_layer_select", wrong)
+    with pytest.raises(AssertionError):
+        pin_decode()
