@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Benchmark of the Sketch&Walk hot path on B200 (one process per GPU).
+
+Default run (N=1): the prefill workload of 4 layers, 32 query / 8 KV heads,
+d=128, n=16384, B=64, k=32, s=8, 20% density (bf16), one step = one pass of
+sws_sketch -> sws_walk_select -> sws_sparse_attn_prefill over all 4 layers.
+The decode workload (16 sequences x 131072 cached tokens, 8 layers, 64 steps)
+is timed in the same run and reported under "decode". Every input is seeded
+synthetic data resident in HBM before the timed region; "e2e" repeats the
+prefill step with the inputs copied from pinned host memory and the outputs
+copied back inside the timed region.
+
+With --gpus N under torchrun each rank runs an independent replica (the path
+has no data exchange); times are the max over ranks.
+--impl reference times the oracle (fp64, host cores) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s + % tensor peak at 20% density; decode step µs + HBM GB/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi sampling of the SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id.lower()
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        mhz, mx, reasons, watts = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            bus = parts[0].lower()
+            if self.bus_id and not (bus.endswith(self.bus_id) or self.bus_id.endswith(bus)):
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                watts.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(watts) if watts else None, "samples": len(mhz), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- distributed --
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ cpu baseline --
+
+def oracle_prefill_sample(w, budget_s: float, max_heads=None):
+    """Times the oracle on whole heads (all layers, every query block) until the
+    budget is spent; returns (seconds, heads done)."""
+    import numpy as np
+    import oracle
+    import sws_inputs as W
+    from oracle import sws_oracle as so
+    Hd = oracle.srht_matrix(w.d, w.k, w.seed)
+    t0 = time.perf_counter()
+    heads = 0
+    limit = w.hq if max_heads is None else max_heads
+    gen_time = 0.0
+    while heads < limit:
+        st = so.PrefillState()
+        h = heads
+        for layer in range(w.layers):
+            g0 = time.perf_counter()
+            q, k, v = W.prefill_head_inputs(w, layer, h)
+            q64, k64, v64 = (x.double().numpy()[None] for x in (q, k, v))
+            gen_time += time.perf_counter() - g0
+            so.prefill_layer(q64, k64, v64, Hd, w.B, w.s, w.density, st, heads=[0], attention_blocks="all")
+        heads += 1
+        if time.perf_counter() - t0 - gen_time >= budget_s:
+            break
+    return time.perf_counter() - t0 - gen_time, heads
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, budget_s=12.0):
+    secs, heads = oracle_prefill_sample(w, budget_s)
+    full = secs * w.hq / heads
+    return {"value": w.n / full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"oracle (fp64 numpy) on {heads} of {w.hq} query heads x {w.layers} layers, every query block; "
+                      f"{secs:.1f} s measured, scaled by heads to the whole {w.hq}-head pass",
+            "host_cpus": os.cpu_count()}
+
+
+# --------------------------------------------------------------- reference --
+
+def run_reference(args, world, rank):
+    import sws_inputs as W
+    if rank != 0:
+        return 0
+    w = W.PREFILL_16K
+    for _ in range(args.warmup):
+        oracle_prefill_sample(w, 0.0, max_heads=1)
+    times = []
+    for _ in range(args.steps):
+        secs, heads = oracle_prefill_sample(w, 0.0, max_heads=1)
+        times.append(secs * w.hq / heads)
+    step = statistics.mean(times)
+    value = w.n / step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
+                   "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
+                         "sample": f"each step: the oracle on 1 of {w.hq} query heads x {w.layers} layers, "
+                                   f"scaled by heads to the whole pass"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- ours ---
+
+def bench_prefill(args, world, S, W, torch):
+    w = W.PREFILL_16K
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    path = S.PrefillPath(h, w.n, w.hq, w.hkv, torch.bfloat16)
+    inputs = [W.prefill_layer_inputs(w, layer, "cuda") for layer in range(w.layers)]
+    stream = torch.cuda.current_stream()
+    in_bytes = sum(x.numel() * x.element_size() for t in inputs for x in t)
+
+    def step(ev=None):
+        for layer, (Q, K, V) in enumerate(inputs):
+            if ev is not None:
+                ev[layer][0].record(stream)
+            path.sketch(Q, K)
+            if ev is not None:
+                ev[layer][1].record(stream)
+            path.walk_select(layer == 0)
+            if ev is not None:
+                ev[layer][2].record(stream)
+            path.attention(Q, K, V)
+            if ev is not None:
+                ev[layer][3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(w.layers)]
+           for _ in range(args.steps)]
+    dev_props = torch.cuda.get_device_properties(0)
+    bus = f"{getattr(dev_props, 'pci_domain_id', 0):08x}:{getattr(dev_props, 'pci_bus_id', 0):02x}:" \
+          f"{getattr(dev_props, 'pci_device_id', 0):02x}.0"
+    clocks = ClockSampler(bus)
+    clocks.start()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = S.sws_launch_count()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    launches = S.sws_launch_count() - launches0
+    barrier(world)
+    clk = clocks.stop()
+    assert S.sws_sync_check(h) == 0
+    ms = t_start.elapsed_time(t_end)
+    ms_max = max_over_ranks(ms, world)
+    stage = {"sketch": 0.0, "walk_select": 0.0, "attention": 0.0}
+    attn_ms = []
+    for i in range(args.steps):
+        for layer in range(w.layers):
+            e = evs[i][layer]
+            stage["sketch"] += e[0].elapsed_time(e[1])
+            stage["walk_select"] += e[1].elapsed_time(e[2])
+            a = e[2].elapsed_time(e[3])
+            stage["attention"] += a
+            attn_ms.append(a)
+    stage = {k: v / args.steps for k, v in stage.items()}
+    flops = w.hq * path.nnz * 4 * w.B * w.B * w.d  # executed block pairs x 4 B^2 d
+    sketch_bytes = (w.hq + w.hkv) * w.n * w.d * 2 + 8 * (w.hq + w.hkv) * path.b * w.k + 8 * w.hq * path.b * (path.b + 1) // 2
+    res = dict(w=w, h=h, path=path, inputs=inputs, ms=ms_max, launches=launches, clocks=clk, stage=stage,
+               attn_ms=statistics.mean(attn_ms), flops=flops, sketch_bytes=sketch_bytes, in_bytes=in_bytes)
+    return res
+
+
+def bench_prefill_e2e(args, world, S, torch, pf):
+    w, path, inputs = pf["w"], pf["path"], pf["inputs"]
+    host_in = [tuple(x.cpu().pin_memory() for x in t) for t in inputs]
+    host_out = [torch.empty_like(path.o, device="cpu").pin_memory() for _ in range(w.layers)]
+    outs = [torch.empty_like(path.o) for _ in range(w.layers)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for layer in range(w.layers):
+            dq, dk, dv = inputs[layer]
+            hq_, hk_, hv_ = host_in[layer]
+            dq.copy_(hq_, non_blocking=True)
+            dk.copy_(hk_, non_blocking=True)
+            dv.copy_(hv_, non_blocking=True)
+            path.layer(dq, dk, dv, layer == 0, out=outs[layer])
+            host_out[layer].copy_(outs[layer], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    steps = max(3, args.steps // 2)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    h2d = sum(x.numel() * x.element_size() for t in host_in for x in t)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    return {"value": world * w.n / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def bench_decode(args, world, S, W, torch, peaks):
+    wd = W.DECODE_128K
+    cfg = S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed)
+    h = S.Handle(cfg)
+    path = S.DecodePath(h, wd.batch, wd.hq, wd.hkv, wd.max_len, wd.layers)
+    toks_k = torch.empty(wd.steps, wd.layers, wd.batch, wd.hkv, wd.d, dtype=torch.bfloat16, device="cuda")
+    toks_v = torch.empty_like(toks_k)
+    toks_q = torch.empty(wd.steps, wd.layers, wd.batch, wd.hq, wd.d, dtype=torch.bfloat16, device="cuda")
+    for layer in range(wd.layers):
+        for s_ in range(wd.batch):
+            K, V = W.decode_cache_inputs(wd, s_, layer, "cuda")
+            path.k_cache[layer][s_].copy_(K)
+            path.v_cache[layer][s_].copy_(V)
+            toks_k[:, layer, s_] = K[:, wd.n0:].transpose(0, 1)
+            toks_v[:, layer, s_] = V[:, wd.n0:].transpose(0, 1)
+            del K, V
+            toks_q[:, layer, s_] = W.decode_queries(wd, s_, layer, "cuda").transpose(0, 1)
+    path.init_cache(torch.full((wd.batch,), wd.n0, dtype=torch.int32, device="cuda"))
+    union_log = torch.zeros(wd.steps, wd.layers, wd.batch, wd.hkv, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    warm = min(args.warmup, wd.steps - 1)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * wd.layers + 1)] for _ in range(wd.steps)]
+
+    def step(t, rec):
+        path.begin_step()
+        if rec:
+            ev[t][0].record(stream)
+        for layer in range(wd.layers):
+            L = S
+            L.sws_decode_step(h, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer], path.seq_lens,
+                              path.k_cache[layer], path.v_cache[layer], path.k_psum[layer], path.k_sketch[layer],
+                              layer == 0, path.walk_state, path.head_sel, path.head_cnt, path.sel, path.sel_mask,
+                              path.sel_cnt)
+            if rec:
+                ev[t][1 + 2 * layer].record(stream)
+            L.sws_sparse_attn_decode(h, toks_q[t, layer], path.k_cache[layer], path.v_cache[layer], path.seq_lens,
+                                     path.sel, path.sel_mask, path.sel_cnt, path.o, path.ws)
+            if rec:
+                ev[t][2 + 2 * layer].record(stream)
+            union_log[t, layer].copy_(path.sel_cnt, non_blocking=True)
+
+    for t in range(warm):
+        step(t, False)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for t in range(warm, wd.steps):
+        step(t, True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    timed = wd.steps - warm
+    step_ms = max_over_ranks(a.elapsed_time(b), world) / timed
+    attn_ms, sel_ms = [], []
+    for t in range(warm, wd.steps):
+        for layer in range(wd.layers):
+            sel_ms.append(ev[t][2 * layer].elapsed_time(ev[t][1 + 2 * layer]))
+            attn_ms.append(ev[t][1 + 2 * layer].elapsed_time(ev[t][2 + 2 * layer]))
+    u = union_log[warm:].double()
+    kv_bytes = float(u.sum().item()) * wd.B * wd.d * 2 * 2 / timed  # union blocks x (K + V) per step
+    nb = -(-(wd.n0 + wd.steps) // wd.B)
+    units = wd.batch * wd.hkv * wd.layers
+    sk_bytes = units * nb * wd.k * 8 + wd.batch * wd.hq * wd.layers * nb * 8 * 2  # k~ reads, rho read+write
+    tok_bytes = wd.layers * wd.batch * (2 * wd.hq + 2 * wd.hkv) * wd.d * 2
+    step_bytes = kv_bytes + sk_bytes + tok_bytes
+    attn_launch_ms = statistics.mean(attn_ms)
+    attn_bytes = kv_bytes / wd.layers
+    hbm = peaks["hbm_gbs"]
+    dense_bytes = units * (wd.n0 + wd.steps) * wd.d * 4
+    out = {
+        "workload": wd.name, "step_us": step_ms * 1e3, "steps_timed": timed,
+        "hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
+        "bytes_per_step": step_bytes, "kv_bytes_per_step": kv_bytes, "dense_kv_bytes_per_step": dense_bytes,
+        "union_blocks_per_unit": float(u.mean().item()),
+        "stages_us_per_layer": {"decode_step": statistics.mean(sel_ms) * 1e3, "attention": attn_launch_ms * 1e3},
+        "roofline": {"kernel": "sws_sparse_attn_decode (split + combine)", "bound": "hbm",
+                     "achieved": attn_bytes / (attn_launch_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": attn_bytes / (attn_launch_ms * 1e-3) / 1e9 / hbm, "traffic": None},
+    }
+    h.close()
+    return out
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+    import torch
+    import block_sparse_attention_sws_b200 as S
+    import sws_inputs as W
+    S.load()
+    peaks, peak_kind = load_peaks()
+    pf = bench_prefill(args, world, S, W, torch)
+    w = pf["w"]
+    ms_step = pf["ms"] / args.steps
+    value = world * w.n / (ms_step * 1e-3)
+    attn_tflops = pf["flops"] / (pf["attn_ms"] * 1e-3) / 1e12
+    peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded AR(1) + sink + hub generator (sws_inputs); no datasets or weights",
+        "config": {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
+                   "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 ({pf['in_bytes'] / 1e6:.0f} MB per step)"},
+        "stages_ms_per_step": pf["stage"],
+        "roofline": {"kernel": "sws_sparse_attn_prefill", "bound": "tensor", "achieved": attn_tflops, "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_t, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 sustained", "flops_per_launch": pf["flops"],
+                     "ms_per_launch": pf["attn_ms"]},
+        "sketch_roofline": {"bound": "hbm", "achieved": pf["sketch_bytes"] / (pf["stage"]["sketch"] / w.layers * 1e-3) / 1e9,
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+        "clocks": pf["clocks"], "gpu_launches": pf["launches"],
+    }
+    line["sketch_roofline"]["frac"] = line["sketch_roofline"]["achieved"] / peaks["hbm_gbs"]
+    if not args.no_e2e:
+        line["e2e"] = bench_prefill_e2e(args, world, S, torch, pf)
+    pf["h"].close()
+    del pf
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        line["decode"] = bench_decode(args, world, S, W, torch, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(W.PREFILL_16K)
+    if rank == 0:
+        s = json.dumps(line)
+        print(s, flush=True)
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(s + "\n")
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,254 @@
+"""ctypes binding of libsws (include/sws.h): argument marshalling only.
+
+Every entry point here forwards to the C function of the same name with raw
+pointers taken from torch tensors; no step of the computation happens in
+Python. If the shared library is missing, loading fails loudly: there is no
+fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsws.so")
+
+SWS_OK, SWS_ERR_INVALID_ARG, SWS_ERR_UNSUPPORTED, SWS_ERR_WORKSPACE, SWS_ERR_CUDA, SWS_ERR_DEVICE_CHECK = range(6)
+SWS_BF16, SWS_FP32 = 0, 1
+SWS_WALK_MATRIX_POWER, SWS_WALK_ELEMENTWISE = 0, 1
+SWS_OP_SKETCH, SWS_OP_WALK_SELECT, SWS_OP_PREFILL_ATTN, SWS_OP_DECODE_ATTN = range(4)
+
+# Every exported symbol of include/sws.h (the CPU test checks the header and this list agree).
+EXPORTS = [
+    "sws_status_string", "sws_config_check", "sws_num_blocks", "sws_csr_nnz", "sws_build_projection_host",
+    "sws_workspace_size", "sws_create", "sws_destroy", "sws_projection_device", "sws_launch_count",
+    "sws_sync_check", "sws_sketch",
+    "sws_walk_select", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
+    "sws_sparse_attn_decode",
+]
+
+
+class SwsConfig(ctypes.Structure):
+    _fields_ = [
+        ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("sketch_dim", ctypes.c_int32),
+        ("walk_power", ctypes.c_int32), ("walk_mode", ctypes.c_int32), ("density_num", ctypes.c_int32),
+        ("density_den", ctypes.c_int32), ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64),
+    ]
+
+
+class SwsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libsws.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    CFG = ctypes.POINTER(SwsConfig)
+    sig = {
+        "sws_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "sws_config_check": (ctypes.c_int, [CFG]),
+        "sws_num_blocks": (I64, [CFG, I64]),
+        "sws_csr_nnz": (I64, [CFG, I64]),
+        "sws_build_projection_host": (ctypes.c_int, [CFG, P]),
+        "sws_workspace_size": (ctypes.c_int, [CFG, ctypes.c_int, I64, I32, I32, I32, ctypes.POINTER(SZ)]),
+        "sws_create": (ctypes.c_int, [CFG, ctypes.POINTER(P)]),
+        "sws_destroy": (ctypes.c_int, [P]),
+        "sws_projection_device": (P, [P]),
+        "sws_launch_count": (U64, []),
+        "sws_sync_check": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
+        "sws_sketch": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P]),
+        "sws_walk_select": (ctypes.c_int, [P, P, I64, I32, ctypes.c_int, P, P, P, P, SZ, P]),
+        "sws_sparse_attn_prefill": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, SZ, P]),
+        "sws_decode_init_cache": (ctypes.c_int, [P, P, I32, I32, I64, P, P, P, P]),
+        "sws_decode_advance": (ctypes.c_int, [P, P, I32, P]),
+        "sws_decode_step": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, ctypes.c_int, P, P, P, P,
+                                           P, P, P]),
+        "sws_sparse_attn_decode": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load().sws_status_string(int(s)).decode()
+
+
+def _check(s: int, where: str) -> None:
+    if s != SWS_OK:
+        raise SwsError(s, where)
+
+
+def make_config(head_dim=128, block_size=64, sketch_dim=32, walk_power=8, walk_mode=SWS_WALK_MATRIX_POWER,
+                density=(1, 5), seed=0) -> SwsConfig:
+    return SwsConfig(head_dim, block_size, sketch_dim, walk_power, walk_mode, density[0], density[1], 0, seed)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SWS_BF16
+    if t.dtype == torch.float32:
+        return SWS_FP32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ host ----
+
+def sws_config_check(cfg: SwsConfig) -> int:
+    return load().sws_config_check(ctypes.byref(cfg))
+
+
+def sws_num_blocks(cfg: SwsConfig, n: int) -> int:
+    return load().sws_num_blocks(ctypes.byref(cfg), n)
+
+
+def sws_csr_nnz(cfg: SwsConfig, n: int) -> int:
+    return load().sws_csr_nnz(ctypes.byref(cfg), n)
+
+
+def sws_build_projection_host(cfg: SwsConfig) -> torch.Tensor:
+    out = torch.empty(cfg.head_dim, cfg.sketch_dim, dtype=torch.float64)
+    _check(load().sws_build_projection_host(ctypes.byref(cfg), out.data_ptr()), "sws_build_projection_host")
+    return out
+
+
+def sws_workspace_size(cfg: SwsConfig, op: int, n: int, hq: int, hkv: int, batch: int = 1) -> int:
+    v = ctypes.c_size_t(0)
+    _check(load().sws_workspace_size(ctypes.byref(cfg), op, n, hq, hkv, batch, ctypes.byref(v)), "sws_workspace_size")
+    return v.value
+
+
+# ---------------------------------------------------------------- handle ----
+
+class Handle:
+    """Owns an sws_handle (H_d on the current CUDA device)."""
+
+    def __init__(self, cfg: SwsConfig):
+        self.cfg = cfg
+        self._lib = load()
+        p = ctypes.c_void_p()
+        _check(self._lib.sws_create(ctypes.byref(cfg), ctypes.byref(p)), "sws_create")
+        self.ptr = p
+
+    def close(self):
+        if getattr(self, "ptr", None):
+            self._lib.sws_destroy(self.ptr)
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def as_parameter(self):
+        return self.ptr
+
+
+def sws_create(cfg: SwsConfig) -> Handle:
+    return Handle(cfg)
+
+
+def sws_destroy(h: Handle) -> None:
+    h.close()
+
+
+def sws_launch_count() -> int:
+    return int(load().sws_launch_count())
+
+
+def sws_sync_check(h: Handle, stream=None) -> int:
+    code = ctypes.c_int32(0)
+    s = load().sws_sync_check(h.ptr, _stream(stream), ctypes.byref(code))
+    if s not in (SWS_OK, SWS_ERR_DEVICE_CHECK):
+        _check(s, "sws_sync_check")
+    return code.value
+
+
+# --------------------------------------------------------------- prefill ----
+
+def sws_sketch(h: Handle, q, k, q_sk, k_sk, scores, stream=None) -> None:
+    hq, n, _ = q.shape
+    hkv = k.shape[0]
+    _check(load().sws_sketch(h.ptr, _ptr(q), _ptr(k), _dtype_code(q), n, hq, hkv, _ptr(q_sk), _ptr(k_sk),
+                             _ptr(scores), _stream(stream)), "sws_sketch")
+
+
+def sws_walk_select(h: Handle, scores, n: int, first_layer: bool, walk_state, row_ptr, col_idx, ws,
+                    stream=None) -> None:
+    hq = scores.shape[0]
+    _check(load().sws_walk_select(h.ptr, _ptr(scores), n, hq, int(bool(first_layer)), _ptr(walk_state),
+                                  _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "sws_walk_select")
+
+
+def sws_sparse_attn_prefill(h: Handle, q, k, v, row_ptr, col_idx, o, ws=None, stream=None) -> None:
+    hq, n, _ = q.shape
+    hkv = k.shape[0]
+    wsp = _ptr(ws) if ws is not None else None
+    wsb = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(load().sws_sparse_attn_prefill(h.ptr, _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), n, hq, hkv, _ptr(row_ptr),
+                                          _ptr(col_idx), _ptr(o), wsp, wsb, _stream(stream)),
+           "sws_sparse_attn_prefill")
+
+
+# ---------------------------------------------------------------- decode ----
+
+def sws_decode_init_cache(h: Handle, k_cache, seq_lens, k_psum, k_sketch, stream=None) -> None:
+    batch, hkv, max_len, _ = k_cache.shape
+    _check(load().sws_decode_init_cache(h.ptr, _ptr(k_cache), batch, hkv, max_len, _ptr(seq_lens), _ptr(k_psum),
+                                        _ptr(k_sketch), _stream(stream)), "sws_decode_init_cache")
+
+
+def sws_decode_advance(h: Handle, seq_lens, stream=None) -> None:
+    _check(load().sws_decode_advance(h.ptr, _ptr(seq_lens), seq_lens.numel(), _stream(stream)), "sws_decode_advance")
+
+
+def sws_decode_step(h: Handle, q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer: bool,
+                    walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    hkv, max_len = k_cache.shape[1], k_cache.shape[2]
+    _check(load().sws_decode_step(h.ptr, _ptr(q_tok), _ptr(k_tok), _ptr(v_tok), batch, hq, hkv, max_len,
+                                  _ptr(seq_lens), _ptr(k_cache), _ptr(v_cache), _ptr(k_psum), _ptr(k_sketch),
+                                  int(bool(first_layer)), _ptr(walk_state), _ptr(head_sel), _ptr(head_cnt), _ptr(sel),
+                                  _ptr(sel_mask), _ptr(sel_cnt), _stream(stream)), "sws_decode_step")
+
+
+def sws_sparse_attn_decode(h: Handle, q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o, ws,
+                           stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    hkv, max_len = k_cache.shape[1], k_cache.shape[2]
+    _check(load().sws_sparse_attn_decode(h.ptr, _ptr(q_tok), _ptr(k_cache), _ptr(v_cache), batch, hq, hkv, max_len,
+                                         _ptr(seq_lens), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt), _ptr(o), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)), "sws_sparse_attn_decode")

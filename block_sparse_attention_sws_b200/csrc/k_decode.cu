@@ -1,0 +1,564 @@
+// Decode-side kernels.
+//
+// "Scout Before You Attend" §5: every decode step chooses the KV-cache blocks
+// for its one new query token with the same sketch-and-walk score, then runs
+// exact attention over them (memory-bound: the cost is reading K and V).
+//
+// Per layer and step:
+//   decode_select_kernel (one CTA per (sequence, KV head)):
+//     1. appends the token's K/V to the cache, adds K to the running sum of the
+//        last block and refreshes that block's sketch k~ = mean * H_d;
+//     2. for each query head of the GQA group (one warp each): q~ = q H_d,
+//        z_j = q~ . k~_j / sqrt(k) over the cached blocks, the log-domain walk
+//        rho_j += s * (z_j - logsumexp(z)), and the top-tau blocks of rho;
+//     3. the union of the group's choices, ascending, with a per-block head mask.
+//   decode_attn_kernel (split over the union): each CTA streams a slice of the
+//     union's K/V blocks (cp.async, 3 stages), scores all heads of the group
+//     with mma.sync tiles (heads are the M rows), keeps a running max / sum per
+//     head, and writes a partial (o, max, sum) per head.
+//   decode_combine_kernel: merges the partials of each (sequence, head).
+#include <algorithm>
+
+#include "select.cuh"
+#include "sws_common.cuh"
+
+namespace sws {
+namespace {
+
+// ---------------------------------------------------------------- init ------
+// k_sketch for every cached block and k_psum (sum of the last block's keys).
+template <int D>
+__global__ void __launch_bounds__(D) init_cache_kernel(const __nv_bfloat16* __restrict__ kc, int32_t hkv,
+                                                       int64_t max_len, int32_t B, int64_t max_blocks,
+                                                       const int32_t* __restrict__ seq_lens,
+                                                       const double* __restrict__ hdt, int32_t k,
+                                                       double* __restrict__ k_psum, double* __restrict__ k_sketch,
+                                                       int32_t* err) {
+  __shared__ double mean[D];
+  const int64_t unit = blockIdx.y;  // sequence * hkv + kv head
+  const int bi = static_cast<int>(unit / hkv);
+  const int32_t len = seq_lens[bi];
+  if (len < 1 || len > max_len) {
+    if (threadIdx.x == 0) record_error(err, GUARD_BAD_LEN);
+    return;
+  }
+  const int64_t nb = ceil_div64(len, B);
+  const int64_t j = blockIdx.x;
+  if (j >= nb) return;
+  const int64_t r0 = j * B, r1 = std::min<int64_t>(len, r0 + B);
+  const __nv_bfloat16* base = kc + unit * max_len * D;
+  double s = 0.0;
+  for (int64_t r = r0; r < r1; ++r) s += static_cast<double>(__bfloat162float(base[r * D + threadIdx.x]));
+  if (j == nb - 1) k_psum[unit * D + threadIdx.x] = s;
+  mean[threadIdx.x] = s / static_cast<double>(r1 - r0);
+  __syncthreads();
+  for (int c = threadIdx.x; c < k; c += D) {
+    double acc = 0.0;
+    for (int t = 0; t < D; ++t) acc += mean[t] * hdt[(size_t)c * D + t];
+    k_sketch[(unit * max_blocks + j) * k + c] = acc;
+  }
+}
+
+__global__ void advance_kernel(int32_t* seq_lens, int32_t batch) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < batch) seq_lens[i] += 1;
+}
+
+// -------------------------------------------------------------- select ------
+constexpr int kSelThreads = 256;
+constexpr int kChunk = 64;  // k~ rows staged per pass
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
+    const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_tok,
+    const __nv_bfloat16* __restrict__ v_tok, int32_t hq, int32_t hkv, int64_t max_len, int64_t max_blocks,
+    const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache,
+    double* __restrict__ k_psum, double* __restrict__ k_sketch, int first_layer, double* __restrict__ walk_state,
+    int32_t* __restrict__ head_sel, int32_t* __restrict__ head_cnt, int32_t* __restrict__ sel,
+    uint8_t* __restrict__ sel_mask, int32_t* __restrict__ sel_cnt, const double* __restrict__ hdt, int32_t k,
+    int32_t B, int32_t s_pow, int32_t num, int32_t den, int32_t* err) {
+  const int group = hq / hkv;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                 // [group][max_blocks] (z, then keys)
+  uint32_t* mark = reinterpret_cast<uint32_t*>(keys + group * max_blocks);  // [max_blocks]
+  double* qt = reinterpret_cast<double*>(mark + ((max_blocks + 1) & ~int64_t(1)));  // [group][k]
+  double* ks = qt + group * k;                                        // [kChunk][k + 1]
+  double* mean = ks + kChunk * (k + 1);                               // [D]
+  int* wsum = reinterpret_cast<int*>(mean + D);                       // [kSelThreads / 32 + 1]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t unit = blockIdx.x;
+  const int bi = static_cast<int>(unit / hkv), g = static_cast<int>(unit % hkv);
+  const int32_t len = seq_lens[bi];
+  if (len < 1 || len > max_len) {
+    if (tid == 0) record_error(err, GUARD_BAD_LEN);
+    return;
+  }
+  const int64_t pos = len - 1;
+  const int64_t blk = pos / B;
+  const int cnt = static_cast<int>(pos % B) + 1;
+  const int64_t nb = blk + 1;
+  for (int64_t j = tid; j < nb; j += kSelThreads) mark[j] = 0u;
+
+  // 1. append the token and refresh the last block's sketch
+  if (tid < D) {
+    const __nv_bfloat16 kt = k_tok[unit * D + tid];
+    k_cache[(unit * max_len + pos) * D + tid] = kt;
+    v_cache[(unit * max_len + pos) * D + tid] = v_tok[unit * D + tid];
+    double ps = (cnt == 1) ? 0.0 : k_psum[unit * D + tid];
+    ps += static_cast<double>(__bfloat162float(kt));
+    k_psum[unit * D + tid] = ps;
+    mean[tid] = ps / cnt;
+  }
+  __syncthreads();
+  double* ksk = k_sketch + unit * max_blocks * k;
+  for (int c = tid; c < k; c += kSelThreads) {
+    double acc = 0.0;
+    for (int t = 0; t < D; ++t) acc += mean[t] * hdt[(size_t)c * D + t];
+    ksk[blk * k + c] = acc;
+  }
+  // q~ = q H_d for every head of the group
+  for (int x = tid; x < group * k; x += kSelThreads) {
+    const int r = x / k, c = x % k;
+    const __nv_bfloat16* qr = q_tok + ((int64_t)bi * hq + g * group + r) * D;
+    double acc = 0.0;
+    for (int t = 0; t < D; ++t) acc += static_cast<double>(__bfloat162float(qr[t])) * hdt[(size_t)c * D + t];
+    qt[r * k + c] = acc;
+  }
+  __syncthreads();
+
+  // 2a. z_j for every head, k~ staged through shared memory
+  double* z = reinterpret_cast<double*>(keys);
+  const double inv_sqrt_k = 1.0 / sqrt((double)k);
+  for (int64_t j0 = 0; j0 < nb; j0 += kChunk) {
+    const int rows = static_cast<int>(std::min<int64_t>(kChunk, nb - j0));
+    for (int x = tid; x < rows * k; x += kSelThreads) ks[(x / k) * (k + 1) + x % k] = ksk[j0 * k + x];
+    __syncthreads();
+    for (int x = tid; x < group * rows; x += kSelThreads) {
+      const int r = x / rows, jj = x % rows;
+      double acc = 0.0;
+      for (int c = 0; c < k; ++c) acc += qt[r * k + c] * ks[jj * (k + 1) + c];
+      z[r * max_blocks + j0 + jj] = acc * inv_sqrt_k;
+    }
+    __syncthreads();
+  }
+
+  // 2b. log-domain walk and top-tau, one warp per head
+  const int tau = tau_of_row(nb - 1, num, den);
+  for (int r = warp; r < group; r += kSelThreads / 32) {
+    const int h = g * group + r;
+    double* zr = z + r * max_blocks;
+    double mx = -INFINITY;
+    for (int64_t j = lane; j < nb; j += 32) mx = fmax(mx, zr[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    double se = 0.0;
+    for (int64_t j = lane; j < nb; j += 32) se += exp(zr[j] - mx);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
+    const double lse = mx + log(se);
+    double* rho = walk_state + ((int64_t)bi * hq + h) * max_blocks;
+    uint64_t* kr = keys + r * max_blocks;
+    for (int64_t j = lane; j < nb; j += 32) {
+      const double val = (first_layer ? 0.0 : rho[j]) + s_pow * (zr[j] - lse);
+      rho[j] = val;
+      kr[j] = order_key(val);
+    }
+    __syncwarp();
+    warp_top_tau(kr, static_cast<int>(nb), tau, head_sel + ((int64_t)bi * hq + h) * max_blocks, err, mark, 1u << r);
+    if (lane == 0) head_cnt[(int64_t)bi * hq + h] = tau;
+  }
+  __syncthreads();
+
+  // 3. ordered compaction of the union
+  int base = 0;
+  for (int64_t j0 = 0; j0 < nb; j0 += kSelThreads) {
+    const int64_t j = j0 + tid;
+    const uint32_t mk = (j < nb) ? mark[j] : 0u;
+    const unsigned bal = __ballot_sync(0xffffffffu, mk != 0u);
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    int off = base;
+    for (int w = 0; w < warp; ++w) off += wsum[w];
+    int tot = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) tot += wsum[w];
+    if (mk != 0u) {
+      const int p = off + __popc(bal & lanemask_lt());
+      sel[unit * max_blocks + p] = static_cast<int32_t>(j);
+      sel_mask[unit * max_blocks + p] = static_cast<uint8_t>(mk);
+    }
+    base += tot;
+    __syncthreads();
+  }
+  if (tid == 0) sel_cnt[unit] = base;
+}
+
+// ----------------------------------------------------------- attention ------
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kAttnThreads = 128;
+constexpr int kStages = 3;
+
+// Row u of a staged [B][D] bf16 tile keeps its 16-byte chunks XOR-swizzled by
+// u mod (D/8), so that the column accesses of the mma fragments and of
+// ldmatrix hit distinct banks.
+template <int D>
+__device__ __forceinline__ int swz(int u, int d) {
+  constexpr int CPR = D / 8;
+  return u * D + (((d >> 3) ^ (u & (CPR - 1))) << 3) + (d & 7);
+}
+
+template <int D, int BS, int G>
+__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
+    const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_cache,
+    const __nv_bfloat16* __restrict__ v_cache, int32_t hkv, int64_t max_len, int64_t max_blocks,
+    const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ sel, const uint8_t* __restrict__ sel_mask,
+    const int32_t* __restrict__ sel_cnt, float* __restrict__ partial, int32_t splits, int32_t* err) {
+  static_assert(G >= 1 && G <= 8, "GQA group of 1..8 query heads");
+  constexpr int NT_QK = BS / 8 / 4;  // score n-tiles (8 tokens) per warp
+  constexpr int NT_PV = D / 8 / 4;   // output n-tiles (8 dims) per warp
+  constexpr int TILE = BS * D;
+  extern __shared__ __align__(16) uint8_t smem[];
+  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);  // [kStages][2][BS][D]
+  float* sc = reinterpret_cast<float*>(stage + kStages * 2 * TILE);  // [8][BS]
+  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(sc + 8 * BS);  // [8][BS + 8]
+  float* corr_s = reinterpret_cast<float*>(ps + 8 * (BS + 8));       // [8]
+  float* ml_s = corr_s + 8;                                          // [8][2]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int64_t unit = blockIdx.y;
+  const int bi = static_cast<int>(unit / hkv);
+  const int split = blockIdx.x;
+  int32_t len = seq_lens[bi];
+  int64_t U = sel_cnt[unit];
+  if (len < 1 || len > max_len || U < 0 || U > ceil_div64(len, BS)) {  // stale or corrupt state: no work
+    if (tid == 0) record_error(err, GUARD_BAD_LEN);
+    len = 0;
+    U = 0;
+  }
+  const int64_t lo = U * split / splits, hi = U * (split + 1) / splits;
+  const int32_t* blist = sel + unit * max_blocks;
+  const uint8_t* mlist = sel_mask + unit * max_blocks;
+  const __nv_bfloat16* kbase = k_cache + unit * max_len * D;
+  const __nv_bfloat16* vbase = v_cache + unit * max_len * D;
+
+  // Q fragments (rows = heads of the group, pre-scaled later in fp32)
+  uint32_t qa[D / 16][2];
+  {
+    const int h = (gq < G) ? gq : 0;
+    const __nv_bfloat16* qr = q_tok + ((int64_t)bi * hkv * G + (unit % hkv) * G + h) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tq);
+      const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tq);
+      qa[ks][0] = (gq < G) ? x0 : 0u;
+      qa[ks][1] = (gq < G) ? x1 : 0u;
+    }
+  }
+  for (int x = tid; x < 8 * (BS + 8); x += kAttnThreads) ps[x] = __float2bfloat16_rn(0.f);
+  if (tid < 8) {  // running max (log2 units) and sum per head
+    ml_s[2 * tid] = -INFINITY;
+    ml_s[2 * tid + 1] = 0.f;
+  }
+  float oacc[NT_PV][4];
+#pragma unroll
+  for (int nt = 0; nt < NT_PV; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+
+  auto block_ok = [&](int64_t j) { return j >= 0 && j * BS < len; };
+  auto issue = [&](int64_t idx, int st) {
+    const int64_t j = block_ok(blist[idx]) ? blist[idx] : -1;
+    const int64_t t0 = j < 0 ? (int64_t)len : j * BS;  // an invalid block stages zeros
+    __nv_bfloat16* ksm = stage + (st * 2) * TILE;
+    __nv_bfloat16* vsm = ksm + TILE;
+    for (int x = tid; x < TILE / 8; x += kAttnThreads) {
+      const int u = x / (D / 8), c = x % (D / 8);
+      const bool valid = t0 + u < len;
+      const int64_t row = valid ? (t0 + u) : 0;
+      cp_async16(ksm + swz<D>(u, c * 8), kbase + row * D + c * 8, valid);
+      cp_async16(vsm + swz<D>(u, c * 8), vbase + row * D + c * 8, valid);
+    }
+  };
+
+  const float qscale = 1.4426950408889634f / sqrtf((float)D);
+#pragma unroll
+  for (int p = 0; p < kStages - 1; ++p) {
+    if (lo + p < hi) issue(lo + p, p);
+    cp_async_commit();
+  }
+  for (int64_t it = lo; it < hi; ++it) {
+    const int st = static_cast<int>((it - lo) % kStages);
+    if (it + kStages - 1 < hi) issue(it + kStages - 1, static_cast<int>((it - lo + kStages - 1) % kStages));
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();
+    __syncthreads();
+    const __nv_bfloat16* ksm = stage + (st * 2) * TILE;
+    const __nv_bfloat16* vsm = ksm + TILE;
+    const int64_t jraw = blist[it];
+    const bool jok = block_ok(jraw);
+    if (!jok && tid == 0) record_error(err, GUARD_BAD_CSR);
+    const uint32_t hm = jok ? mlist[it] : 0u;
+    const int64_t t0 = jok ? jraw * BS : 0;
+
+    // scores: warp handles n-tiles [warp*NT_QK, (warp+1)*NT_QK)
+#pragma unroll
+    for (int nt = 0; nt < NT_QK; ++nt) {
+      const int n0 = (warp * NT_QK + nt) * 8;
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int u = n0 + gq;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(ksm + swz<D>(u, ks * 16 + 2 * tq));
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(ksm + swz<D>(u, ks * 16 + 8 + 2 * tq));
+        const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+        mma_bf16_16816(c, a, b0, b1);
+      }
+      if (gq < G) {
+        const bool hv = (hm >> gq) & 1u;
+        const int u0 = n0 + 2 * tq;
+        sc[gq * BS + u0] = (hv && t0 + u0 < len) ? c[0] * qscale : -INFINITY;
+        sc[gq * BS + u0 + 1] = (hv && t0 + u0 + 1 < len) ? c[1] * qscale : -INFINITY;
+      }
+    }
+    __syncthreads();
+    // online softmax: warp w owns heads w, w + 4
+    for (int r = warp; r < G; r += 4) {
+      float mx = -INFINITY;
+      for (int u = lane; u < BS; u += 32) mx = fmaxf(mx, sc[r * BS + u]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mr = ml_s[2 * r];
+      const float mn = fmaxf(mr, mx);
+      float corr = 1.f, sum = 0.f;
+      if (mn != -INFINITY) {
+        corr = exp2f(mr - mn);
+        for (int u = lane; u < BS; u += 32) {
+          const float p = exp2f(sc[r * BS + u] - mn);
+          sum += p;
+          ps[r * (BS + 8) + u] = __float2bfloat16_rn(p);
+        }
+      } else {
+        for (int u = lane; u < BS; u += 32) ps[r * (BS + 8) + u] = __float2bfloat16_rn(0.f);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      __syncwarp();
+      if (lane == 0) {
+        corr_s[r] = corr;
+        ml_s[2 * r] = mn;
+        ml_s[2 * r + 1] = ml_s[2 * r + 1] * corr + sum;
+      }
+    }
+    __syncthreads();
+    // P V: warp handles output dims [warp*NT_PV*8, (warp+1)*NT_PV*8)
+    {
+      const float cr = (gq < G) ? corr_s[gq] : 1.f;
+#pragma unroll
+      for (int nt = 0; nt < NT_PV; ++nt) {
+        oacc[nt][0] *= cr;
+        oacc[nt][1] *= cr;
+      }
+#pragma unroll
+      for (int kk = 0; kk < BS / 16; ++kk) {
+        uint32_t a[4];
+        a[0] = *reinterpret_cast<const uint32_t*>(ps + gq * (BS + 8) + kk * 16 + 2 * tq);
+        a[1] = 0u;
+        a[2] = *reinterpret_cast<const uint32_t*>(ps + gq * (BS + 8) + kk * 16 + 8 + 2 * tq);
+        a[3] = 0u;
+#pragma unroll
+        for (int np = 0; np < NT_PV / 2; ++np) {
+          const int n0 = (warp * NT_PV + 2 * np) * 8;
+          const int mi = lane >> 3, ri = lane & 7;
+          const int u = kk * 16 + ri + 8 * (mi & 1);
+          const int dcol = n0 + 8 * (mi >> 1);
+          uint32_t bfr[4];
+          ldsm_x4_trans(bfr, vsm + swz<D>(u, dcol));
+          mma_bf16_16816(oacc[2 * np], a, bfr[0], bfr[1]);
+          mma_bf16_16816(oacc[2 * np + 1], a, bfr[2], bfr[3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+
+  // partial results: [unit][head][split][D + 2]
+  if (gq < G) {
+    float* pr = partial + (((unit * G + gq) * splits) + split) * (D + 2);
+#pragma unroll
+    for (int nt = 0; nt < NT_PV; ++nt) {
+      const int d0 = (warp * NT_PV + nt) * 8 + 2 * tq;
+      pr[d0] = oacc[nt][0];
+      pr[d0 + 1] = oacc[nt][1];
+    }
+  }
+  if (tid < G) {
+    float* pr = partial + (((unit * G + tid) * splits) + split) * (D + 2);
+    const bool any = hi > lo;
+    pr[D] = any ? ml_s[2 * tid] : -INFINITY;
+    pr[D + 1] = any ? ml_s[2 * tid + 1] : 0.f;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ partial, int32_t hq, int32_t hkv,
+                                                           int32_t splits, __nv_bfloat16* __restrict__ o) {
+  const int64_t bh = blockIdx.x;  // sequence * hq + head
+  const int group = hq / hkv;
+  const int64_t bi = bh / hq;
+  const int h = static_cast<int>(bh % hq);
+  const int64_t unit = bi * hkv + h / group;
+  const float* pr = partial + ((unit * group + h % group) * splits) * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, pr[s * (D + 2) + D]);
+  float L = 0.f, acc = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float ms = pr[s * (D + 2) + D];
+    if (ms == -INFINITY) continue;
+    const float w = exp2f(ms - M);
+    L += w * pr[s * (D + 2) + D + 1];
+    acc += w * pr[s * (D + 2) + threadIdx.x];
+  }
+  o[bh * D + threadIdx.x] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+}
+
+template <int D, int BS, int G>
+cudaError_t launch_attn3(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, int32_t batch,
+                         int32_t hkv, int64_t max_len, int64_t max_blocks, const int32_t* lens, const int32_t* sel,
+                         const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits, int32_t* err,
+                         cudaStream_t st) {
+  const size_t smem = (size_t)kStages * 2 * BS * D * 2 + 8 * BS * 4 + 8 * (BS + 8) * 2 + 8 * 4 + 16 * 4;
+  auto kern = decode_attn_kernel<D, BS, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(splits, static_cast<unsigned>((int64_t)batch * hkv));
+  kern<<<grid, kAttnThreads, smem, st>>>(q, kc, vc, hkv, max_len, max_blocks, lens, sel, mask, cnt, partial, splits,
+                                         err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_attn2(int32_t group, const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc,
+                         int32_t batch, int32_t hkv, int64_t max_len, int64_t max_blocks, const int32_t* lens,
+                         const int32_t* sel, const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits,
+                         int32_t* err, cudaStream_t st) {
+#define SWS_G(GG)                                                                                                  \
+  case GG:                                                                                                         \
+    return launch_attn3<D, BS, GG>(q, kc, vc, batch, hkv, max_len, max_blocks, lens, sel, mask, cnt, partial, \
+                                   splits, err, st);
+  switch (group) {
+    SWS_G(1) SWS_G(2) SWS_G(4) SWS_G(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef SWS_G
+}
+
+}  // namespace
+
+size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group) {
+  const int64_t k = cfg.sketch_dim, D = cfg.head_dim;
+  return (size_t)group * max_blocks * 8 + (size_t)((max_blocks + 1) & ~int64_t(1)) * 4 + (size_t)group * k * 8 +
+         (size_t)kChunk * (k + 1) * 8 + (size_t)D * 8 + (kSelThreads / 32 + 1) * 4;
+}
+
+int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group) {
+  const int64_t mb = ceil_div64(max_len, cfg.block_size);
+  const int64_t umax = std::min<int64_t>(mb, (int64_t)group * tau_of_row(mb - 1, cfg.density_num, cfg.density_den));
+  return static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(256, ceil_div64(umax, 16))));
+}
+
+cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, int32_t batch, int32_t hkv,
+                                     int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+                                     cudaStream_t st) {
+  const int32_t B = h->cfg.block_size;
+  const int64_t mb = ceil_div64(max_len, B);
+  dim3 grid(static_cast<unsigned>(mb), static_cast<unsigned>((int64_t)batch * hkv));
+  if (h->cfg.head_dim == 128)
+    init_cache_kernel<128><<<grid, 128, 0, st>>>(k_cache, hkv, max_len, B, mb, seq_lens, h->hdt, h->cfg.sketch_dim,
+                                                 k_psum, k_sketch, h->err);
+  else
+    init_cache_kernel<64><<<grid, 64, 0, st>>>(k_cache, hkv, max_len, B, mb, seq_lens, h->hdt, h->cfg.sketch_dim,
+                                               k_psum, k_sketch, h->err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_advance(int32_t* seq_lens, int32_t batch, cudaStream_t st) {
+  advance_kernel<<<static_cast<unsigned>(ceil_div64(batch, 128)), 128, 0, st>>>(seq_lens, batch);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
+                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                 const int32_t* seq_lens, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
+                                 double* k_psum, double* k_sketch, int first_layer, double* walk_state,
+                                 int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
+                                 int32_t* sel_cnt, cudaStream_t st) {
+  const sws_config& c = h->cfg;
+  const int64_t mb = ceil_div64(max_len, c.block_size);
+  const size_t smem = decode_select_smem_bytes(c, mb, hq / hkv);
+  auto kern = c.head_dim == 128 ? decode_select_kernel<128> : decode_select_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<static_cast<unsigned>((int64_t)batch * hkv), kSelThreads, smem, st>>>(
+      q_tok, k_tok, v_tok, hq, hkv, max_len, mb, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
+      walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, h->hdt, c.sketch_dim, c.block_size, c.walk_power,
+      c.density_num, c.density_den, h->err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,
+                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                               const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
+                               const int32_t* sel_cnt, __nv_bfloat16* o, float* partial, int32_t splits,
+                               cudaStream_t st) {
+  const sws_config& c = h->cfg;
+  const int64_t mb = ceil_div64(max_len, c.block_size);
+  const int32_t group = hq / hkv;
+  cudaError_t e;
+  if (c.head_dim == 128)
+    e = c.block_size == 64 ? launch_attn2<128, 64>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
+                                                    sel, sel_mask, sel_cnt, partial, splits, h->err, st)
+                           : launch_attn2<128, 128>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb,
+                                                     seq_lens, sel, sel_mask, sel_cnt, partial, splits, h->err, st);
+  else
+    e = c.block_size == 64 ? launch_attn2<64, 64>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
+                                                   sel, sel_mask, sel_cnt, partial, splits, h->err, st)
+                           : launch_attn2<64, 128>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
+                                                    sel, sel_mask, sel_cnt, partial, splits, h->err, st);
+  if (e != cudaSuccess) return e;
+  if (c.head_dim == 128)
+    decode_combine_kernel<128><<<static_cast<unsigned>((int64_t)batch * hq), 128, 0, st>>>(partial, hq, hkv, splits,
+                                                                                          o);
+  else
+    decode_combine_kernel<64><<<static_cast<unsigned>((int64_t)batch * hq), 64, 0, st>>>(partial, hq, hkv, splits, o);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sws

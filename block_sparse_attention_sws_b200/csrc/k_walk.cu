@@ -1,0 +1,208 @@
+// sw_walk_select kernels.
+//
+// "Scout Before You Attend" §4 (sketch-determined walk):
+//   A^l  = row softmax of the sketched scores over the causal blocks j <= i,
+//   R^0  = (A^0)^s,  R^l = R^{l-1} (A^l)^s,
+// then the top-tau key blocks of every row of R^l.
+//
+// Everything here is fp64: after a few layers the entries of R that decide the
+// selection are 1e-20 .. 1e-40 of the row maximum, below what fp32 holds.
+// The b x b matrices are lower-triangular, so the GEMM only visits tiles on or
+// below the diagonal and, inside a tile pair, only k in [tile(j), tile(i)].
+#include <algorithm>
+
+#include "select.cuh"
+#include "sws_common.cuh"
+
+namespace sws {
+namespace {
+
+// One warp per row. temp = 1 for the softmax of §4; temp = s gives the
+// entrywise power with renormalised rows (softmax(S)^s / sum = softmax(s S)).
+__global__ void __launch_bounds__(256) block_softmax_kernel(const double* __restrict__ S, int64_t b, int64_t rows,
+                                                            double temp, double* __restrict__ A) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t i = row % b;
+  const double* s = S + row * b;
+  double* a = A + row * b;
+  double mx = -INFINITY;
+  for (int64_t j = lane; j <= i; j += 32) mx = fmax(mx, temp * s[j]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  double sum = 0.0;
+  for (int64_t j = lane; j <= i; j += 32) sum += exp(temp * s[j] - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) / sum : 0.0;
+}
+
+// C = A * Bm for lower-triangular b x b matrices, one 64 x 64 output tile per
+// CTA, 64 threads with 8 x 8 accumulators each, k staged 8 at a time.
+constexpr int kTT = 64, kTK = 8;
+
+__device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int64_t& tj) {
+  // heaviest tiles (largest ti - tj) first
+  for (int64_t dl = nt - 1; dl >= 0; --dl) {
+    const int64_t cnt = nt - dl;
+    if (t < cnt) { tj = t; ti = t + dl; return; }
+    t -= cnt;
+  }
+  ti = tj = 0;
+}
+
+__global__ void __launch_bounds__(64) tri_gemm_kernel(const double* __restrict__ A, const double* __restrict__ Bm,
+                                                      double* __restrict__ C, int64_t b) {
+  __shared__ __align__(16) double As[2][kTK][kTT];  // k-major
+  __shared__ __align__(16) double Bs[2][kTK][kTT];
+  const int64_t nt = ceil_div64(b, kTT);
+  int64_t ti, tj;
+  tile_of(blockIdx.x, nt, ti, tj);
+  const size_t hoff = (size_t)blockIdx.y * b * b;
+  const double* Ah = A + hoff;
+  const double* Bh = Bm + hoff;
+  double* Ch = C + hoff;
+  const int tid = threadIdx.x;
+  const int tr = tid / 8, tc = tid % 8;
+  const int64_t i0 = ti * kTT, j0 = tj * kTT;
+  const int64_t kbeg = j0, kend = std::min<int64_t>(b, i0 + kTT);
+
+  double ra[kTK], rb[kTK];
+  auto load = [&](int64_t k0) {
+    // A: thread owns row i0 + tid, 8 consecutive k
+    const int64_t ar = i0 + tid;
+#pragma unroll
+    for (int q = 0; q < kTK; ++q) {
+      const int64_t kk = k0 + q;
+      ra[q] = (ar < b && kk < kend && kk <= ar) ? Ah[ar * b + kk] : 0.0;  // lower triangle only
+    }
+    // B: row k0 + tid/8, 8 consecutive columns starting at (tid%8)*8
+    const int64_t br = k0 + tid / 8;
+    const int64_t bc = j0 + (tid % 8) * 8;
+#pragma unroll
+    for (int q = 0; q < kTK; ++q) rb[q] = (br < kend && bc + q < b && bc + q <= br) ? Bh[br * b + bc + q] : 0.0;
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < kTK; ++q) As[buf][q][tid] = ra[q];
+#pragma unroll
+    for (int q = 0; q < kTK; ++q) Bs[buf][tid / 8][(tid % 8) * 8 + q] = rb[q];
+  };
+
+  double acc[8][8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+
+  int buf = 0;
+  load(kbeg);
+  store(0);
+  __syncthreads();
+  for (int64_t k0 = kbeg; k0 < kend; k0 += kTK) {
+    const bool more = k0 + kTK < kend;
+    if (more) load(k0 + kTK);
+#pragma unroll
+    for (int q = 0; q < kTK; ++q) {
+      double a[8], bv[8];
+      const double2* ap = reinterpret_cast<const double2*>(&As[buf][q][tr * 8]);
+      const double2* bp = reinterpret_cast<const double2*>(&Bs[buf][q][tc * 8]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double2 x = ap[u], y = bp[u];
+        a[2 * u] = x.x;
+        a[2 * u + 1] = x.y;
+        bv[2 * u] = y.x;
+        bv[2 * u + 1] = y.y;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[u][v] = fma(a[u], bv[v], acc[u][v]);
+    }
+    if (more) {
+      store(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int64_t i = i0 + tr * 8 + u;
+    if (i >= b) continue;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int64_t j = j0 + tc * 8 + v;
+      if (j < b) Ch[i * b + j] = acc[u][v];
+    }
+  }
+}
+
+// One warp per row: copies R's row to the walk state (zeros above the
+// diagonal), writes row_ptr, and emits the row's top-tau blocks ascending.
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ R, int64_t b, int64_t rows,
+                                                     int32_t num, int32_t den, int64_t nnz,
+                                                     double* __restrict__ walk_state, int32_t* __restrict__ row_ptr,
+                                                     int32_t* __restrict__ col_idx, int32_t* err) {
+  extern __shared__ __align__(16) uint64_t keys_all[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  uint64_t* keys = keys_all + (size_t)warp * b;
+  const int64_t h = row / b, i = row % b;
+  const double* r = R + row * b;
+  double* ws = walk_state + row * b;
+  for (int64_t j = lane; j < b; j += 32) {
+    const double x = (j <= i) ? r[j] : 0.0;
+    ws[j] = x;
+    if (j <= i) keys[j] = order_key(x);
+  }
+  int64_t rp = 0;
+  for (int64_t q = lane; q < i; q += 32) rp += tau_of_row(q, num, den);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) rp += __shfl_xor_sync(0xffffffffu, rp, off);
+  const int tau = tau_of_row(i, num, den);
+  if (lane == 0) {
+    row_ptr[h * (b + 1) + i] = static_cast<int32_t>(rp);
+    if (i == b - 1) row_ptr[h * (b + 1) + b] = static_cast<int32_t>(rp + tau);
+  }
+  __syncwarp();
+  warp_top_tau(keys, static_cast<int>(i + 1), tau, col_idx + h * nnz + rp, err);
+}
+
+}  // namespace
+
+cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int64_t b, int32_t hq, double* A,
+                                 cudaStream_t st) {
+  const int64_t rows = (int64_t)hq * b;
+  const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
+  block_softmax_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st) {
+  const int64_t nt = ceil_div64(b, kTT);
+  dim3 grid(static_cast<unsigned>(nt * (nt + 1) / 2), hq);
+  tri_gemm_kernel<<<grid, 64, 0, st>>>(A, Bm, C, b);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32_t hq, double* walk_state,
+                          int32_t* row_ptr, int32_t* col_idx, cudaStream_t st) {
+  const int64_t rows = (int64_t)hq * b;
+  int warps = static_cast<int>(std::min<int64_t>(8, std::max<int64_t>(1, (160 << 10) / (b * 8))));
+  const size_t smem = (size_t)warps * b * sizeof(uint64_t);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int64_t nnz = 0;
+  for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
+  select_kernel<<<static_cast<unsigned>(ceil_div64(rows, warps)), warps * 32, smem, st>>>(
+      R, b, rows, h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sws

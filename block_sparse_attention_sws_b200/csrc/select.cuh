@@ -1,0 +1,83 @@
+// Warp-level exact top-tau selection (radix select on 64-bit keys).
+//
+// "Scout Before You Attend" §4: for each query block, the tau key blocks with the
+// largest walk score. Ties go to the lower block index and the chosen indices are
+// written in ascending order.
+#pragma once
+
+#include "sws_common.cuh"
+
+namespace sws {
+
+// Order-preserving map from a double to an unsigned 64-bit key.
+__device__ __forceinline__ uint64_t order_key(double x) {
+  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// keys[0, m): shared memory, written before the call and visible to the warp.
+// Writes the tau chosen indices, ascending, to out[0, tau). If `mark` is not
+// null, also ORs `bit` into mark[j] for every chosen j (shared memory).
+// 1 <= tau <= m <= 65535 * 2 (counts are held in 16-bit fields).
+__device__ __forceinline__ void warp_top_tau(const uint64_t* keys, int m, int tau, int32_t* out, int32_t* err,
+                                             uint32_t* mark = nullptr, uint32_t bit = 0) {
+  const int lane = threadIdx.x & 31;
+  uint64_t prefix = 0, pmask = 0;
+  int need = tau;
+  bool all_cands = false;
+  for (int shift = 62; shift >= 0; shift -= 2) {
+    uint32_t lo = 0, hi = 0;  // 16-bit counters: digits {0,1} in lo, {2,3} in hi
+    for (int j = lane; j < m; j += 32) {
+      const uint64_t key = keys[j];
+      if ((key & pmask) == prefix) {
+        const uint32_t dg = static_cast<uint32_t>(key >> shift) & 3u;
+        const uint32_t inc = 1u << ((dg & 1u) * 16);
+        if (dg < 2) lo += inc; else hi += inc;
+      }
+    }
+    lo = __reduce_add_sync(0xffffffffu, lo);
+    hi = __reduce_add_sync(0xffffffffu, hi);
+    const int cnt[4] = {static_cast<int>(lo & 0xffffu), static_cast<int>(lo >> 16), static_cast<int>(hi & 0xffffu),
+                        static_cast<int>(hi >> 16)};
+    int dsel = 0;
+    for (int dd = 3; dd >= 0; --dd) {
+      if (need <= cnt[dd]) { dsel = dd; break; }
+      need -= cnt[dd];
+    }
+    prefix |= static_cast<uint64_t>(dsel) << shift;
+    pmask |= 3ull << shift;
+    if (cnt[dsel] == need) { all_cands = true; break; }
+  }
+  const unsigned lt = lanemask_lt();
+  int base = 0, ties = 0;
+  for (int j0 = 0; j0 < m; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < m;
+    const uint64_t km = valid ? (keys[j] & pmask) : 0;
+    const bool above = valid && km > prefix;
+    const bool cand = valid && km == prefix;
+    const unsigned cb = __ballot_sync(0xffffffffu, cand);
+    bool take = cand;
+    if (!all_cands) {
+      take = cand && (ties + __popc(cb & lt)) < need;
+      ties += __popc(cb);
+    }
+    const bool sel = above || take;
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = base + __popc(sb & lt);
+      if (pos < tau) out[pos] = j;
+      if (mark) atomicOr(&mark[j], bit);
+    }
+    base += __popc(sb);
+  }
+  if (lane == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
+}
+
+}  // namespace sws

@@ -1,0 +1,376 @@
+// libsws C ABI: argument validation, the projection builder, handle lifetime
+// and the launch sequence of every entry point. No allocation happens here
+// except in sws_create.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "sws_common.cuh"
+
+using namespace sws;
+
+namespace sws {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int count) { g_launches.fetch_add(static_cast<uint64_t>(count), std::memory_order_relaxed); }
+}  // namespace sws
+
+namespace {
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool log_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("SWS_LOG");
+    on = (e && e[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
+sws_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SWS_OK;
+  if (log_enabled()) std::fprintf(stderr, "[sws] %s: %s\n", what, cudaGetErrorString(e));
+  return SWS_ERR_CUDA;
+}
+
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// splitmix64 (Steele, Lea and Flood, OOPSLA 2014): state advance + output mix.
+uint64_t splitmix_next(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+constexpr uint64_t kProjectionTag = 0x5357535F48414431ull;
+
+int popcount32(uint32_t x) {
+  int c = 0;
+  while (x) {
+    x &= x - 1;
+    ++c;
+  }
+  return c;
+}
+
+sws_status check_heads(int32_t hq, int32_t hkv) {
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hq > 4096) return SWS_ERR_INVALID_ARG;
+  return SWS_OK;
+}
+
+constexpr int64_t kMaxPrefillBlocks = 8192;  // top-tau counters and row staging limit
+
+}  // namespace
+
+extern "C" {
+
+const char* sws_status_string(sws_status s) {
+  switch (s) {
+    case SWS_OK: return "ok";
+    case SWS_ERR_INVALID_ARG: return "invalid argument";
+    case SWS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SWS_ERR_WORKSPACE: return "workspace too small";
+    case SWS_ERR_CUDA: return "CUDA error";
+    case SWS_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+sws_status sws_config_check(const sws_config* c) {
+  if (!c) return SWS_ERR_INVALID_ARG;
+  if (c->reserved != 0) return SWS_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return SWS_ERR_UNSUPPORTED;
+  if (c->block_size != 64 && c->block_size != 128) return SWS_ERR_UNSUPPORTED;
+  if (c->sketch_dim < 1 || c->sketch_dim > c->head_dim) return SWS_ERR_INVALID_ARG;
+  if (c->walk_power < 1 || c->walk_power > 64) return SWS_ERR_INVALID_ARG;
+  if (c->walk_mode != SWS_WALK_MATRIX_POWER && c->walk_mode != SWS_WALK_ELEMENTWISE) return SWS_ERR_INVALID_ARG;
+  if (c->density_num < 1 || c->density_den < 1 || c->density_num > c->density_den) return SWS_ERR_INVALID_ARG;
+  if (!pow2(c->head_dim)) return SWS_ERR_UNSUPPORTED;
+  return SWS_OK;
+}
+
+int64_t sws_num_blocks(const sws_config* c, int64_t n) {
+  if (sws_config_check(c) != SWS_OK || n < 1) return -1;
+  return ceil_div64(n, c->block_size);
+}
+
+int64_t sws_csr_nnz(const sws_config* c, int64_t n) {
+  const int64_t b = sws_num_blocks(c, n);
+  if (b < 0) return -1;
+  int64_t nnz = 0;
+  for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, c->density_num, c->density_den);
+  return nnz;
+}
+
+sws_status sws_build_projection_host(const sws_config* c, double* hd) {
+  sws_status s = sws_config_check(c);
+  if (s != SWS_OK) return s;
+  if (!hd) return SWS_ERR_INVALID_ARG;
+  const int d = c->head_dim, k = c->sketch_dim;
+  uint64_t state = c->seed ^ kProjectionTag;
+  std::vector<uint64_t> draws(2 * d - 1);
+  for (auto& x : draws) x = splitmix_next(state);
+  std::vector<int> sign(d), perm(d);
+  for (int r = 0; r < d; ++r) sign[r] = (draws[r] >> 63) ? -1 : 1;
+  for (int r = 0; r < d; ++r) perm[r] = r;
+  int next = d;
+  for (int r = d - 1; r >= 1; --r) {
+    const int j = static_cast<int>(draws[next++] % static_cast<uint64_t>(r + 1));
+    std::swap(perm[r], perm[j]);
+  }
+  // H_d[r][c] = sqrt(d/k) * sign[r] * (-1)^popcount(r & perm[c]) / sqrt(d) = sign * (+-1) / sqrt(k)
+  const double scale = std::sqrt(static_cast<double>(d) / k) / std::sqrt(static_cast<double>(d));
+  for (int r = 0; r < d; ++r)
+    for (int cc = 0; cc < k; ++cc) {
+      const int par = popcount32(static_cast<uint32_t>(r & perm[cc])) & 1;
+      hd[r * k + cc] = scale * sign[r] * (par ? -1.0 : 1.0);
+    }
+  return SWS_OK;
+}
+
+sws_status sws_workspace_size(const sws_config* c, sws_op op, int64_t n, int32_t hq, int32_t hkv, int32_t batch,
+                              size_t* bytes) {
+  sws_status s = sws_config_check(c);
+  if (s != SWS_OK) return s;
+  if (!bytes || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  const int64_t b = ceil_div64(n, c->block_size);
+  switch (op) {
+    case SWS_OP_SKETCH:
+    case SWS_OP_PREFILL_ATTN:
+      *bytes = 0;
+      return SWS_OK;
+    case SWS_OP_WALK_SELECT:
+      // up to four b x b fp64 matrices per head live at once (power by squaring)
+      *bytes = 4 * static_cast<size_t>(hq) * b * b * sizeof(double);
+      return SWS_OK;
+    case SWS_OP_DECODE_ATTN: {
+      if (batch < 1) return SWS_ERR_INVALID_ARG;
+      const int32_t splits = decode_num_splits(*c, n, hq / hkv);
+      *bytes = static_cast<size_t>(batch) * hq * splits * (c->head_dim + 2) * sizeof(float);
+      return SWS_OK;
+    }
+  }
+  return SWS_ERR_INVALID_ARG;
+}
+
+sws_status sws_create(const sws_config* c, sws_handle** out) {
+  if (!out) return SWS_ERR_INVALID_ARG;
+  *out = nullptr;
+  sws_status s = sws_config_check(c);
+  if (s != SWS_OK) return s;
+  const int d = c->head_dim, k = c->sketch_dim;
+  std::vector<double> hd(static_cast<size_t>(d) * k), hdt(static_cast<size_t>(d) * k);
+  sws_build_projection_host(c, hd.data());
+  for (int r = 0; r < d; ++r)
+    for (int cc = 0; cc < k; ++cc) hdt[(size_t)cc * d + r] = hd[(size_t)r * k + cc];
+  auto* h = new sws_handle();
+  h->cfg = *c;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  void* mem = nullptr;
+  const size_t hd_bytes = hd.size() * sizeof(double);
+  if (e == cudaSuccess) e = cudaMalloc(&mem, 2 * hd_bytes + 256);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_status(e, "sws_create");
+  }
+  h->hd = static_cast<double*>(mem);
+  h->hdt = h->hd + hd.size();
+  h->err = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mem) + 2 * hd_bytes);
+  e = cudaMemcpy(h->hd, hd.data(), hd_bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->hdt, hdt.data(), hd_bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int32_t));
+  if (e != cudaSuccess) {
+    cudaFree(mem);
+    delete h;
+    return cuda_status(e, "sws_create upload");
+  }
+  *out = h;
+  return SWS_OK;
+}
+
+sws_status sws_destroy(sws_handle* h) {
+  if (!h) return SWS_ERR_INVALID_ARG;
+  cudaError_t e = cudaFree(h->hd);
+  delete h;
+  return cuda_status(e, "sws_destroy");
+}
+
+const double* sws_projection_device(const sws_handle* h) { return h ? h->hd : nullptr; }
+
+uint64_t sws_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code) {
+  if (!h) return SWS_ERR_INVALID_ARG;
+  auto st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->err, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v != 0) e = cudaMemset(h->err, 0, sizeof(int32_t));
+  if (code) *code = v;
+  if (e != cudaSuccess) return cuda_status(e, "sws_sync_check");
+  return v ? SWS_ERR_DEVICE_CHECK : SWS_OK;
+}
+
+sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n, int32_t hq,
+                      int32_t hkv, double* q_sk, double* k_sk, double* scores, void* stream) {
+  if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (dtype != SWS_BF16 && dtype != SWS_FP32) return SWS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sk) || !aligned16(k_sk) || !aligned16(scores))
+    return SWS_ERR_INVALID_ARG;
+  const int64_t b = ceil_div64(n, h->cfg.block_size);
+  if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
+  auto st = static_cast<cudaStream_t>(stream);
+  sws_status s = cuda_status(launch_sketch_pool_project(h, q, dtype, n, hq, q_sk, st), "sketch q");
+  if (s != SWS_OK) return s;
+  s = cuda_status(launch_sketch_pool_project(h, k, dtype, n, hkv, k_sk, st), "sketch k");
+  if (s != SWS_OK) return s;
+  return cuda_status(launch_sketch_scores(h, q_sk, k_sk, b, hq, hkv, scores, st), "sketch scores");
+}
+
+sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n, int32_t hq, int first_layer,
+                           double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (!h || n < 1 || hq < 1) return SWS_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(walk_state) || !aligned16(row_ptr) || !aligned16(col_idx) || !aligned16(ws))
+    return SWS_ERR_INVALID_ARG;
+  const int64_t b = ceil_div64(n, h->cfg.block_size);
+  if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
+  size_t need = 0;
+  sws_workspace_size(&h->cfg, SWS_OP_WALK_SELECT, n, hq, 1, 1, &need);
+  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
+  auto st = static_cast<cudaStream_t>(stream);
+  const size_t mat = static_cast<size_t>(hq) * b * b;
+  double* buf[4] = {static_cast<double*>(ws), static_cast<double*>(ws) + mat, static_cast<double*>(ws) + 2 * mat,
+                    static_cast<double*>(ws) + 3 * mat};
+  bool busy[4] = {false, false, false, false};
+  auto take = [&]() -> int {
+    for (int q = 0; q < 4; ++q)
+      if (!busy[q]) {
+        busy[q] = true;
+        return q;
+      }
+    return -1;
+  };
+  const int a = take();
+  sws_status s = cuda_status(launch_block_softmax(h, scores, b, hq, buf[a], st), "block softmax");
+  if (s != SWS_OK) return s;
+  int m_idx = a;  // holds M = A^s when done
+  if (h->cfg.walk_mode == SWS_WALK_MATRIX_POWER && h->cfg.walk_power > 1) {
+    // binary powering: result = prod of base^(2^t) over the set bits of s
+    int base = a, result = -1;
+    int e = h->cfg.walk_power;
+    while (true) {
+      if (e & 1) {
+        if (result < 0) {
+          result = base;
+        } else {
+          const int dst = take();
+          s = cuda_status(launch_tri_gemm(buf[result], buf[base], buf[dst], b, hq, st), "walk power");
+          if (s != SWS_OK) return s;
+          if (result != base) busy[result] = false;
+          result = dst;
+        }
+      }
+      e >>= 1;
+      if (!e) break;
+      const int dst = take();
+      s = cuda_status(launch_tri_gemm(buf[base], buf[base], buf[dst], b, hq, st), "walk square");
+      if (s != SWS_OK) return s;
+      if (base != result) busy[base] = false;
+      base = dst;
+    }
+    if (base != result) busy[base] = false;
+    m_idx = result;
+  }
+  const double* Rnew = buf[m_idx];
+  if (!first_layer) {
+    const int dst = take();
+    s = cuda_status(launch_tri_gemm(walk_state, buf[m_idx], buf[dst], b, hq, st), "walk update");
+    if (s != SWS_OK) return s;
+    Rnew = buf[dst];
+  }
+  return cuda_status(launch_select(h, Rnew, b, hq, walk_state, row_ptr, col_idx, st), "top-tau select");
+}
+
+sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const void* k, const void* v,
+                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
+                                   const int32_t* col_idx, void* o, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (dtype != SWS_BF16 && dtype != SWS_FP32) return SWS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(row_ptr) || !aligned16(col_idx))
+    return SWS_ERR_INVALID_ARG;
+  if (ceil_div64(n, h->cfg.block_size) > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
+  auto st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_attn_prefill_simt(h, q, k, v, dtype, n, hq, hkv, row_ptr, col_idx, o, st),
+                     "prefill attention");
+}
+
+sws_status sws_decode_init_cache(const sws_handle* h, const void* k_cache, int32_t batch, int32_t hkv,
+                                 int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+                                 void* stream) {
+  if (!h || batch < 1 || hkv < 1 || max_len < 1) return SWS_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(seq_lens) || !aligned16(k_psum) || !aligned16(k_sketch))
+    return SWS_ERR_INVALID_ARG;
+  return cuda_status(launch_decode_init_cache(h, static_cast<const __nv_bfloat16*>(k_cache), batch, hkv, max_len,
+                                              seq_lens, k_psum, k_sketch, static_cast<cudaStream_t>(stream)),
+                     "decode init cache");
+}
+
+sws_status sws_decode_advance(const sws_handle* h, int32_t* seq_lens, int32_t batch, void* stream) {
+  if (!h || batch < 1 || !aligned16(seq_lens)) return SWS_ERR_INVALID_ARG;
+  return cuda_status(launch_decode_advance(seq_lens, batch, static_cast<cudaStream_t>(stream)), "decode advance");
+}
+
+sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                           int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
+                           void* k_cache, void* v_cache, double* k_psum, double* k_sketch, int first_layer,
+                           double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
+                           uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
+  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (hq / hkv > 8) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch,
+                        walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  const int64_t mb = ceil_div64(max_len, h->cfg.block_size);
+  if (decode_select_smem_bytes(h->cfg, mb, hq / hkv) > (200u << 10)) return SWS_ERR_UNSUPPORTED;
+  return cuda_status(
+      launch_decode_select(h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_tok),
+                           static_cast<const __nv_bfloat16*>(v_tok), batch, hq, hkv, max_len, seq_lens,
+                           static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), k_psum,
+                           k_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                           static_cast<cudaStream_t>(stream)),
+      "decode step");
+}
+
+sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const void* k_cache, const void* v_cache,
+                                  int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
+                                  const int32_t* sel, const uint8_t* sel_mask, const int32_t* sel_cnt, void* o,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  const int32_t group = hq / hkv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o, ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  size_t need = 0;
+  sws_workspace_size(&h->cfg, SWS_OP_DECODE_ATTN, max_len, hq, hkv, batch, &need);
+  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
+  const int32_t splits = decode_num_splits(h->cfg, max_len, group);
+  return cuda_status(launch_decode_attn(h, static_cast<const __nv_bfloat16*>(q_tok),
+                                        static_cast<const __nv_bfloat16*>(k_cache),
+                                        static_cast<const __nv_bfloat16*>(v_cache), batch, hq, hkv, max_len,
+                                        seq_lens, sel, sel_mask, sel_cnt, static_cast<__nv_bfloat16*>(o),
+                                        static_cast<float*>(ws), splits, static_cast<cudaStream_t>(stream)),
+                     "decode attention");
+}
+
+}  // extern "C"

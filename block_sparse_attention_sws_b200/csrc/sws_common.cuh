@@ -1,0 +1,151 @@
+// Internal declarations shared by the libsws translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sws.h"
+
+struct sws_handle {
+  sws_config cfg;
+  int device;
+  int num_sms;
+  double* hd;    // [d, k] row-major
+  double* hdt;   // [k, d] row-major (transpose, for contiguous per-output reads)
+  int32_t* err;  // device error word (guard code of the first failure, 0 = none)
+};
+
+namespace sws {
+
+// Codes recorded in the device error word.
+enum Guard : int32_t {
+  GUARD_NONE = 0,
+  GUARD_MBAR_TIMEOUT = 1,  // a bounded mbarrier wait ran out
+  GUARD_BAD_CSR = 2,       // a CSR entry outside [0, i] or a non-ascending row
+  GUARD_BAD_SELECT = 3,    // top-tau bookkeeping inconsistent
+  GUARD_BAD_LEN = 4,       // a sequence length outside [1, max_len]
+  GUARD_TMEM = 5           // tensor memory allocation failed
+};
+
+__device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// ---- mbarrier / bulk-copy helpers (sm_90+ PTX, used on sm_100a) -------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: about a second at most (each try_wait suspends for a short,
+// hardware-chosen time). Returns false, after recording the guard, on timeout.
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  record_error(err, GUARD_MBAR_TIMEOUT);
+  return false;
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---- conversions ------------------------------------------------------------
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---- integer helpers shared by host and device -------------------------------
+
+__host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// tau_i = ceil((i+1) * num / den): key blocks kept for query block i.
+__host__ __device__ __forceinline__ int32_t tau_of_row(int64_t i, int32_t num, int32_t den) {
+  return static_cast<int32_t>(((i + 1) * static_cast<int64_t>(num) + den - 1) / den);
+}
+
+// ---- launchers (defined in the kernel translation units) ----------------------
+
+// Counts queued kernels (sws_launch_count); every launcher calls it per launch.
+void note_launches(int count);
+
+cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* x, sws_dtype dt, int64_t n, int32_t heads,
+                                       double* out, cudaStream_t st);
+cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,
+                                 int32_t hkv, double* scores, cudaStream_t st);
+
+cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int64_t b, int32_t hq, double* A,
+                                 cudaStream_t st);
+cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st);
+cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32_t hq, double* walk_state,
+                          int32_t* row_ptr, int32_t* col_idx, cudaStream_t st);
+
+cudaError_t launch_attn_prefill_simt(const sws_handle* h, const void* q, const void* k, const void* v, sws_dtype dt,
+                                     int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
+                                     const int32_t* col_idx, void* o, cudaStream_t st);
+
+cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, int32_t batch, int32_t hkv,
+                                     int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+                                     cudaStream_t st);
+cudaError_t launch_decode_advance(int32_t* seq_lens, int32_t batch, cudaStream_t st);
+cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
+                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                 const int32_t* seq_lens, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
+                                 double* k_psum, double* k_sketch, int first_layer, double* walk_state,
+                                 int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
+                                 int32_t* sel_cnt, cudaStream_t st);
+int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group);
+size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
+cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,
+                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                               const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
+                               const int32_t* sel_cnt, __nv_bfloat16* o, float* partial, int32_t splits,
+                               cudaStream_t st);
+
+}  // namespace sws

@@ -1,0 +1,210 @@
+/*
+ * sws.h -- C ABI of libsws, the B200 (sm_100a) Sketch&Walk sparse-attention hot path.
+ *
+ * Source of the method: "Scout Before You Attend: Sketch-and-Walk Sparse Attention
+ * for Efficient LLM Inference" (blog deep-dive of arXiv 2602.07397). Section numbers
+ * below refer to that page.
+ *
+ * Conventions shared by every call
+ *  - Pointers marked (device) are CUDA device pointers on the handle's device; (host)
+ *    pointers are ordinary host memory. The caller owns every buffer. The library
+ *    allocates device memory only in sws_create (the projection matrix) and never in
+ *    a compute call.
+ *  - Every device pointer must be 16-byte aligned; tensors are dense, row-major,
+ *    with the layouts stated per call (no strides).
+ *  - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and return after the launches were queued. A call that fails its host-side
+ *    validation returns a status and queues nothing. Launch failures return SWS_ERR_CUDA.
+ *  - Device-side guards (bounded waits, index checks) never trap: they record a code in
+ *    a per-device error word; sws_sync_check reads and clears it.
+ *  - No C++ exception crosses this boundary.
+ *
+ * Notation: n tokens, B block size, b = ceil(n/B) blocks, d head dim, k sketch dim,
+ * s walk power, hq query heads, hkv KV heads (query head h reads KV head h/(hq/hkv)),
+ * density num/den, tau_i = ceil((i+1)*num/den) key blocks for query block i.
+ */
+#ifndef SWS_H_
+#define SWS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SWS_OK = 0,
+  SWS_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, inconsistent shapes */
+  SWS_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement */
+  SWS_ERR_WORKSPACE = 3,    /* workspace smaller than sws_workspace_size reports */
+  SWS_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  SWS_ERR_DEVICE_CHECK = 5  /* a device-side guard fired (see sws_sync_check) */
+} sws_status;
+
+typedef enum { SWS_BF16 = 0, SWS_FP32 = 1 } sws_dtype;
+
+/* What (A_block)^s of §4 means: the matrix power (default), or the entrywise power
+ * with rows renormalised to sum 1 (the alternative reading of "sparsity exponent"). */
+typedef enum { SWS_WALK_MATRIX_POWER = 0, SWS_WALK_ELEMENTWISE = 1 } sws_walk_mode;
+
+/* Operations whose workspace can be queried. */
+typedef enum {
+  SWS_OP_SKETCH = 0,
+  SWS_OP_WALK_SELECT = 1,
+  SWS_OP_PREFILL_ATTN = 2,
+  SWS_OP_DECODE_ATTN = 3
+} sws_op;
+
+typedef struct {
+  int32_t head_dim;    /* d: 64 or 128 */
+  int32_t block_size;  /* B: 64 or 128 */
+  int32_t sketch_dim;  /* k: 1..d (the page's default is 64; its ablation uses 16-32) */
+  int32_t walk_power;  /* s: 1..64 (default 8, §7) */
+  int32_t walk_mode;   /* sws_walk_mode */
+  int32_t density_num; /* 0 < num <= den; 1/5 = the page's 20% density */
+  int32_t density_den;
+  int32_t reserved;    /* must be 0 */
+  uint64_t seed;       /* seeds the random signs and columns of H_d */
+} sws_config;
+
+typedef struct sws_handle sws_handle;
+
+/* ---------------------------------------------------------------- host-only --- */
+
+const char* sws_status_string(sws_status s);
+
+/* Checks a config against the limits above. Host only; never touches a GPU. */
+sws_status sws_config_check(const sws_config* cfg);
+
+/* Number of blocks b = ceil(n/B), or -1 for an invalid config or n < 1. */
+int64_t sws_num_blocks(const sws_config* cfg, int64_t n);
+
+/* Key blocks kept per head over all query blocks: sum over i < b of tau_i, or -1. */
+int64_t sws_csr_nnz(const sws_config* cfg, int64_t n);
+
+/* The Hadamard projection H_d of §3.2 (d x k, row-major doubles, host memory):
+ * H_d = sqrt(d/k) * D * (H/sqrt(d)) * P, H the Sylvester Hadamard matrix, D random
+ * signs, P k distinct columns. Signs and columns come from the splitmix64 stream
+ * started at seed XOR 0x5357535F48414431: draws 0..d-1 give the signs (+1 when the
+ * top bit is 0), the next d-1 draws a Fisher-Yates shuffle of [0, d) (for r = d-1
+ * down to 1 swap r and draw mod (r+1)); P is the first k shuffled entries.
+ * `hd` receives d*k doubles. */
+sws_status sws_build_projection_host(const sws_config* cfg, double* hd);
+
+/* Workspace bytes that `op` needs for the given sizes (batch is used by decode only). */
+sws_status sws_workspace_size(const sws_config* cfg, sws_op op, int64_t n, int32_t hq, int32_t hkv,
+                              int32_t batch, size_t* bytes);
+
+/* --------------------------------------------------------------- handle --- */
+
+/* Validates cfg and uploads H_d to the current CUDA device (the only allocation the
+ * library makes). On failure *out is NULL. */
+sws_status sws_create(const sws_config* cfg, sws_handle** out);
+sws_status sws_destroy(sws_handle* h);
+
+/* Device copy of H_d (d x k doubles, row-major), owned by the handle. */
+const double* sws_projection_device(const sws_handle* h);
+
+/* Number of kernels this library has queued in this process since it was loaded
+ * (all devices, all threads). Host only; used to count launches in a timed region. */
+uint64_t sws_launch_count(void);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns SWS_OK, SWS_ERR_DEVICE_CHECK (with *code = the recorded guard code), or SWS_ERR_CUDA. */
+sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code);
+
+/* ---------------------------------------------------------------- prefill --- */
+
+/* sw_sketch. §3.1 block means (a partial last block divides by its row count),
+ * §3.2 projection q~_i = q_bar_i H_d, k~_j = k_bar_j H_d and the sketched block scores
+ * S[h,i,j] = q~_i(h) . k~_j(h/(hq/hkv)) / sqrt(k) for j <= i (causal block mask).
+ *   q      (device) [hq, n, d]   dtype
+ *   k      (device) [hkv, n, d]  dtype
+ *   q_sk   (device) [hq, b, k]   double, written
+ *   k_sk   (device) [hkv, b, k]  double, written
+ *   scores (device) [hq, b, b]   double; entries j <= i written, j > i left untouched
+ * Reads Q and K once. */
+sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n,
+                      int32_t hq, int32_t hkv, double* q_sk, double* k_sk, double* scores, void* stream);
+
+/* sw_walk_select. §4: A = row softmax of scores over j <= i (the sketched block
+ * attention matrix), M = A^s, R = M on the first layer, else R = R_prev * M; then for
+ * each query block i the tau_i largest R[i, j], j <= i (ties to the lower j), listed in
+ * ascending order as CSR.
+ *   scores     (device) [hq, b, b] double (lower triangle read)
+ *   walk_state (device) [hq, b, b] double: R_prev in (ignored if first_layer), R out.
+ *              Lower triangle written; entries above the diagonal are written as 0.
+ *   row_ptr    (device) [hq, b+1] int32, written: offsets into the head's col_idx slice
+ *   col_idx    (device) [hq, nnz] int32, written (nnz = sws_csr_nnz)
+ *   ws         (device) sws_workspace_size(SWS_OP_WALK_SELECT) bytes
+ * The walk runs in fp64: R spans hundreds of decades after a few layers. */
+sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n, int32_t hq, int first_layer,
+                           double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* sw_sparse_attn_prefill. §4/§5: exact softmax attention on the original Q, K, V
+ * restricted to the selected key blocks; query token t attends to the tokens u of the
+ * blocks listed for its block with u <= t. Online softmax, fp32 accumulation.
+ *   q (device) [hq, n, d], k, v (device) [hkv, n, d], o (device) [hq, n, d]: all dtype
+ *   row_ptr, col_idx: the CSR of sws_walk_select (each row ascending, within [0, i])
+ * bf16 runs on the tensor cores (fp32 accumulate, output rounded to nearest);
+ * fp32 runs in fp32 FMA. */
+sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const void* k, const void* v,
+                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
+                                   const int32_t* col_idx, void* o, void* ws, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------------- decode --- */
+/* §5: each decode step scores its single new query token against the cached key
+ * blocks with the same sketch. The query is a block of one row; cached key blocks are
+ * their means (the last, partial block by its count). A 1 x b row has no matrix
+ * power, so over the layers of one step the walk is the entrywise product of the
+ * per-layer rows raised to s, kept as logarithms:
+ *   rho^l_j = rho^{l-1}_j + s * (z^l_j - logsumexp_j z^l),  z_j = q~ . k~_j / sqrt(k).
+ * The new token is appended to the cache before it attends.
+ *
+ * Per-layer state (device, caller-owned):
+ *   k_cache, v_cache [batch, hkv, max_len, d] bf16
+ *   k_psum           [batch, hkv, d] double: sum of the keys of the last block
+ *   k_sketch         [batch, hkv, max_blocks, k] double: sketched means of the cached blocks
+ * with max_blocks = ceil(max_len/B). seq_lens (device, int32 [batch]) counts the tokens
+ * of each sequence. */
+
+/* Builds k_psum and k_sketch for caches that already hold seq_lens[i] tokens. */
+sws_status sws_decode_init_cache(const sws_handle* h, const void* k_cache, int32_t batch, int32_t hkv,
+                                 int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+                                 void* stream);
+
+/* Adds 1 to each of the batch entries of seq_lens (device). */
+sws_status sws_decode_advance(const sws_handle* h, int32_t* seq_lens, int32_t batch, void* stream);
+
+/* One layer of the decode-side sketch, walk and selection. seq_lens counts the tokens
+ * INCLUDING this step's token, which is written at position seq_lens[i]-1.
+ *   q_tok [batch, hq, d], k_tok / v_tok [batch, hkv, d] (device, bf16)
+ *   walk_state [batch, hq, max_blocks] double: rho in (ignored if first_layer), out
+ *   head_sel   [batch, hq, max_blocks] int32: each head's blocks, ascending; head_cnt [batch, hq]
+ *   sel        [batch, hkv, max_blocks] int32: union over the GQA group, ascending
+ *   sel_mask   [batch, hkv, max_blocks] uint8: bit r set = query head hkv_index*group + r chose it
+ *   sel_cnt    [batch, hkv] int32
+ * group = hq/hkv must be <= 8. */
+sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                           int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
+                           void* k_cache, void* v_cache, double* k_psum, double* k_sketch, int first_layer,
+                           double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
+                           uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
+
+/* sw_sparse_attn_decode: one query token per (sequence, head) over the tokens
+ * (< seq_lens[i]) of the blocks its head selected. Each KV block of the group's union is
+ * read once for all the group's heads (split over the union, then combined).
+ *   q_tok [batch, hq, d] bf16; o [batch, hq, d] bf16 (device)
+ *   ws    sws_workspace_size(SWS_OP_DECODE_ATTN) bytes */
+sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const void* k_cache,
+                                  const void* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                  const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
+                                  const int32_t* sel_cnt, void* o, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWS_H_ */

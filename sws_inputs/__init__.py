@@ -152,7 +152,7 @@ def ar1(n: int, d: int, rho: float, gen: torch.Generator, device) -> torch.Tenso
     work = torch.float64 if torch.device(device).type == "cpu" else torch.float32
     eps = torch.randn(n, d, generator=gen, device=device, dtype=work)
     eps[1:] *= math.sqrt(1.0 - rho * rho)
-    return _linear_scan(eps, rho)
+    return _linear_scan(eps, rho, chunk=256 if work == torch.float64 else 16)
 
 
 def hub_layout(b: int, hubs: int, d: int, seed: int, layer: int, g: int, device, seq: int = 0):
@@ -196,6 +196,22 @@ def prefill_layer_inputs(w: PrefillWorkload, layer: int, device="cpu"):
             Q[h] = qx.to(out_dt)
             del qx
     return Q, K, V
+
+
+def prefill_head_inputs(w: PrefillWorkload, layer: int, h: int, device="cpu"):
+    """Q[h] [n, d] and K[g], V[g] [n, d] of query head h (g = its KV head): the
+    same streams as prefill_layer_inputs, for callers that need one head only."""
+    out_dt = _dtype(w.dtype)
+    g = h // (w.hq // w.hkv)
+    work = torch.float64 if torch.device(device).type == "cpu" else torch.float32
+    pos, off = hub_layout(w.b, w.hubs, w.d, w.seed, layer, g, device)
+    kx = ar1(w.n, w.d, w.rho, _gen(device, stream_seed(w.seed, layer, KIND_K, g)), device)
+    _add_structure(kx, w.B, pos, off)
+    gv = _gen(device, stream_seed(w.seed, layer, KIND_V, g))
+    v = torch.randn(w.n, w.d, generator=gv, device=device, dtype=work)
+    qx = ar1(w.n, w.d, w.rho, _gen(device, stream_seed(w.seed, layer, KIND_Q, h)), device)
+    _add_structure(qx, w.B, pos, off)
+    return qx.to(out_dt), kx.to(out_dt), v.to(out_dt)
 
 
 def decode_cache_inputs(w: DecodeWorkload, seq: int, layer: int, device="cpu"):

@@ -1,0 +1,153 @@
+"""Parity of the decode path (sws_decode_step, sws_sparse_attn_decode) against
+the oracle, through the C ABI, on seeded synthetic caches.
+
+Every step appends one token per sequence; every layer's selection (each
+head's blocks, the log-domain walk state, the GQA union and its head mask)
+and its attention output are compared with the oracle for the checked
+sequences. Cache slots beyond a sequence's length hold NaN, so any read of a
+token that should be masked shows up in the output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_sws_b200 as S
+import oracle
+import sws_inputs as W
+from oracle import sws_oracle as so
+from parity import compare_attention, compare_selection
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None):
+    dev = "cuda"
+    batch = len(n0s)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    max_len = max(n0s) + steps
+    path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev)
+    group = w.hq // w.hkv
+    check_seqs = list(range(batch)) if check_seqs is None else list(check_seqs)
+    KV, Qs = {}, {}
+    for layer in range(w.layers):
+        path.k_cache[layer].fill_(float("nan"))
+        path.v_cache[layer].fill_(float("nan"))
+        for s_, n0 in enumerate(n0s):
+            ws_ = w.scaled(n0=n0, steps=steps)
+            K, V = W.decode_cache_inputs(ws_, s_, layer, dev)
+            path.k_cache[layer][s_, :, :n0] = K[:, :n0]
+            path.v_cache[layer][s_, :, :n0] = V[:, :n0]
+            KV[(s_, layer)] = (K, V)
+            Qs[(s_, layer)] = W.decode_queries(ws_, s_, layer, dev)
+    path.init_cache(torch.tensor(n0s, dtype=torch.int32, device=dev))
+    Hd = oracle.srht_matrix(w.d, w.k, w.seed)
+    host = {key: (K.double().cpu().numpy(), V.double().cpu().numpy()) for key, (K, V) in KV.items()
+            if key[0] in check_seqs}
+    swaps = []
+    for t in range(steps):
+        path.begin_step()
+        rho_prev = {s_: None for s_ in check_seqs}
+        for layer in range(w.layers):
+            q_tok = torch.stack([Qs[(s_, layer)][:, t] for s_ in range(batch)]).contiguous()
+            k_tok = torch.stack([KV[(s_, layer)][0][:, n0s[s_] + t] for s_ in range(batch)]).contiguous()
+            v_tok = torch.stack([KV[(s_, layer)][1][:, n0s[s_] + t] for s_ in range(batch)]).contiguous()
+            o = path.layer(layer, q_tok, k_tok, v_tok)
+            torch.cuda.synchronize()
+            assert S.sws_sync_check(h) == 0
+            hs = path.head_sel.cpu().numpy()
+            hc = path.head_cnt.cpu().numpy()
+            rho_gpu = path.walk_state.cpu().numpy()
+            sel = path.sel.cpu().numpy()
+            msk = path.sel_mask.cpu().numpy()
+            cnt = path.sel_cnt.cpu().numpy()
+            og = o.float().cpu().numpy()
+            for s_ in check_seqs:
+                length = n0s[s_] + t + 1
+                nb = -(-length // w.B)
+                Kh, Vh = host[(s_, layer)]
+                q = Qs[(s_, layer)][:, t].double().cpu().numpy()
+                rho, z, osel = so.decode_layer_select(q, Kh, length, Hd, w.B, w.s, w.density, rho_prev[s_])
+                rho_prev[s_] = rho
+                assert np.allclose(rho_gpu[s_, :, :nb], rho, rtol=1e-9, atol=1e-9 * np.abs(rho).max())
+                union = {}
+                for hh in range(w.hq):
+                    tau = hc[s_, hh]
+                    gsel = hs[s_, hh, :tau]
+                    assert tau == so.tau_of_row(nb - 1, *w.density)
+                    assert np.all(np.diff(gsel) > 0) and gsel.max() < nb
+                    swaps += [(t, layer, s_, hh) + x for x in compare_selection(gsel, osel[hh], rho[hh],
+                                                                                 log_domain=True)]
+                    for j in gsel:
+                        union[int(j)] = union.get(int(j), 0) | (1 << (hh % group))
+                    g = hh // group
+                    want = so.decode_attention(q[hh], Kh[g], Vh[g], length, gsel, w.B)
+                    compare_attention(og[s_, hh], want)
+                for g in range(w.hkv):
+                    u = {j: m >> 0 for j, m in union.items()}
+                    # union of this KV head's group only
+                    ug = {}
+                    for hh in range(g * group, (g + 1) * group):
+                        for j in hs[s_, hh, :hc[s_, hh]]:
+                            ug[int(j)] = ug.get(int(j), 0) | (1 << (hh - g * group))
+                    n = cnt[s_, g]
+                    assert n == len(ug)
+                    assert list(sel[s_, g, :n]) == sorted(ug)
+                    assert [int(m) for m in msk[s_, g, :n]] == [ug[j] for j in sorted(ug)]
+    h.close()
+    return swaps
+
+
+def test_decode_small_ragged():
+    """Three sequences of different lengths with partial blocks, crossing a block boundary."""
+    w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
+    swaps = run_decode(w, [1000, 1500, 638], steps=5)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
+def test_decode_group_sizes():
+    for hq, hkv in ((4, 4), (4, 2), (8, 1)):
+        w = W.DECODE_128K.scaled(layers=2, hq=hq, hkv=hkv, hubs=3)
+        run_decode(w, [700, 333], steps=3)
+
+
+def test_decode_dense_density():
+    w = W.DECODE_128K.scaled(layers=2, hq=4, hkv=1, hubs=2, density=(1, 1))
+    run_decode(w, [500], steps=2)
+
+
+def test_decode_first_token_of_block():
+    """n0 a multiple of B: the first decode token opens a new block holding only itself."""
+    w = W.DECODE_128K.scaled(layers=2, hq=4, hkv=1, hubs=2)
+    run_decode(w, [1024, 64], steps=2)
+
+
+def test_decode_full_size_sampled():
+    """The full decode workload (16 sequences, 131072 cached tokens, 8 layers)
+    for a few steps; the oracle recomputes two sampled sequences."""
+    w = W.DECODE_128K
+    swaps = run_decode(w, [w.n0] * w.batch, steps=2, check_seqs=[0, w.batch - 1])
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
+def test_decode_bad_length_guard():
+    """A sequence length beyond the cache is rejected by the kernel's own check
+    and reported through the device error word."""
+    w = W.DECODE_128K.scaled(layers=1, hq=4, hkv=1)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    path = S.DecodePath(h, 1, 4, 1, 256, 1)
+    path.k_cache[0].zero_()
+    path.v_cache[0].zero_()
+    path.init_cache(torch.tensor([10], dtype=torch.int32, device="cuda"))
+    assert S.sws_sync_check(h) == 0
+    path.seq_lens.fill_(999)
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, 1, 128, dtype=torch.bfloat16, device="cuda")
+    L = S
+    L.sws_decode_step(h, q, kv, kv, path.seq_lens, path.k_cache[0], path.v_cache[0], path.k_psum[0],
+                      path.k_sketch[0], True, path.walk_state, path.head_sel, path.head_cnt, path.sel, path.sel_mask,
+                      path.sel_cnt)
+    assert S.sws_sync_check(h) == 4  # GUARD_BAD_LEN

@@ -56,3 +56,11 @@ def test_decode_inputs():
     assert Q.shape == (4, 4, 128)
     K2, _ = W.decode_cache_inputs(w, 1, 0)
     assert not torch.equal(K, K2)
+
+
+def test_head_inputs_match_layer_inputs():
+    w = W.TINY.scaled(hq=4, hkv=2, n=300, d=16, dtype="fp32")
+    Q, K, V = W.prefill_layer_inputs(w, 1)
+    for h in range(4):
+        q, k, v = W.prefill_head_inputs(w, 1, h)
+        assert torch.equal(q, Q[h]) and torch.equal(k, K[h // 2]) and torch.equal(v, V[h // 2])
