@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to run (default: the workload's 64)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -330,6 +331,8 @@ def bench_prefill_e2e(args, world, S, torch, pf):
 
 def bench_decode(args, world, S, W, torch, peaks):
     wd = W.DECODE_128K
+    if args.decode_steps is not None:
+        wd = wd.scaled(steps=max(2, min(wd.steps, args.decode_steps)))
     cfg = S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed)
     h = S.Handle(cfg)
     path = S.DecodePath(h, wd.batch, wd.hq, wd.hkv, wd.max_len, wd.layers)

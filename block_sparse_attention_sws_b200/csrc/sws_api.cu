@@ -309,8 +309,11 @@ sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const voi
     return SWS_ERR_INVALID_ARG;
   if (ceil_div64(n, h->cfg.block_size) > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
   auto st = static_cast<cudaStream_t>(stream);
+  if (dtype == SWS_BF16)
+    return cuda_status(launch_attn_prefill_tc(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st),
+                       "prefill attention (tensor cores)");
   return cuda_status(launch_attn_prefill_simt(h, q, k, v, dtype, n, hq, hkv, row_ptr, col_idx, o, st),
-                     "prefill attention");
+                     "prefill attention (fp32)");
 }
 
 sws_status sws_decode_init_cache(const sws_handle* h, const void* k_cache, int32_t batch, int32_t hkv,

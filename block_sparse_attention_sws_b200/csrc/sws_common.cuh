@@ -130,6 +130,10 @@ cudaError_t launch_attn_prefill_simt(const sws_handle* h, const void* q, const v
                                      int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
                                      const int32_t* col_idx, void* o, cudaStream_t st);
 
+cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
+                                   int32_t hq, int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                                   cudaStream_t st);
+
 cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, int32_t batch, int32_t hkv,
                                      int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
                                      cudaStream_t st);

@@ -92,6 +92,9 @@ def test_scaled_workloads_in_full(w):
     (W.TINY.scaled(name="one_row_tail", n=65), 0),
     (W.PREFILL_16K.scaled(name="bf16_d64_B128", d=64, B=128, k=16, n=3000, hq=4, hkv=2, layers=2), 0),
     (W.PREFILL_16K.scaled(name="gqa8", n=1500, hq=8, hkv=1, layers=2), 0),
+    (W.PREFILL_16K.scaled(name="odd_blocks_B64", n=1050, hq=2, hkv=1, layers=2), 0),
+    (W.PREFILL_16K.scaled(name="bf16_one_block", n=100, hq=2, hkv=1, layers=1, hubs=0), 0),
+    (W.PREFILL_64K.scaled(name="bf16_B128_dense", n=700, hq=2, hkv=1, layers=1, density=(1, 1)), 0),
 ], ids=lambda x: x.name if hasattr(x, "name") else str(x))
 def test_edge_cases(w, mode):
     run_case(w, mode=mode)
@@ -108,6 +111,23 @@ def test_dense_density_equals_dense_attention():
     ref = torch.nn.functional.scaled_dot_product_attention(Q.double()[None], K.double()[None], V.double()[None],
                                                            is_causal=True)[0]
     assert (o.double() - ref).abs().max().item() < 1e-4
+
+
+def test_dense_density_equals_dense_attention_bf16():
+    """Density 100% on the tensor-core path: equals dense causal attention (fp64 SDPA) within bf16 tolerance."""
+    for w in (W.PREFILL_16K.scaled(density=(1, 1), n=1000, hq=4, hkv=2, layers=1),
+              W.PREFILL_64K.scaled(density=(1, 1), n=1000, hq=2, hkv=1, layers=1)):
+        cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+        h = S.Handle(cfg)
+        path = S.PrefillPath(h, w.n, w.hq, w.hkv, torch.bfloat16)
+        Q, K, V = W.prefill_layer_inputs(w, 0, "cuda")
+        o = path.layer(Q, K, V, True)
+        g = w.hq // w.hkv
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q.double()[None], K.double().repeat_interleave(g, 0)[None], V.double().repeat_interleave(g, 0)[None],
+            is_causal=True)[0]
+        err = (o.double() - ref).abs()
+        assert err.max().item() < 2e-2 and err.mean().item() < 5e-3
 
 
 FULL = [W.PREFILL_16K, W.PREFILL_64K, W.PREFILL_128K, W.PREFILL_128K_D10]
