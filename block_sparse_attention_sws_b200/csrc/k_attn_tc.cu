@@ -158,15 +158,24 @@ struct Smem {
   static constexpr uint32_t total = bars + sizeof(Bars);
 };
 
-// Bounded wait that also gives up when another role has aborted.
+// Bounded wait (wall time) that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int32_t* err) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 63 && bs->abort) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, kSuspendNs)) return true;
+    if (bs->abort) return false;
+    if (global_ns() - t0 > kWaitNs) break;
   }
   record_error(err, GUARD_MBAR_TIMEOUT);
   bs->abort = 1;
   return false;
+}
+
+// The softmax warps run warp-collective tcgen05.ld/st: a wait's outcome is
+// made uniform across the warp before any of them.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* bs, int32_t* err) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, bs, err));
 }
 
 // Walks the key tiles of one item: for B = 128 the CSR row of query block m;
@@ -429,10 +438,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
       bool first_tile = true;
       while (true) {
         const int st = kv_it & 1;
-        if (!(ok = wait_bar(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
+        if (!(ok = warp_wait(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
         const TileMeta tm = bs->meta[st];
         const int sb = gt & 1;
-        if (!(ok = wait_bar(&bs->s_full[sb], (gt >> 1) & 1, bs, err))) break;
+        if (!(ok = warp_wait(&bs->s_full[sb], (gt >> 1) & 1, bs, err))) break;
         tc_fence_after();
         float s[kTileN];
 #pragma unroll
@@ -471,22 +480,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
           mx = fmaxf(mx, s[c]);
         }
         const float m_new = mx * qscale;
-        if (mx != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2)) {
-          const float alpha = fast_exp2(m_used - m_new);  // 0 when m_used = -inf
-          if (!first_tile) {
-            // O holds earlier tiles at the old reference: wait for them, then rescale this row
-            if (!(ok = wait_bar(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
-            tc_fence_after();
+        const bool need = mx != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2);
+        const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;  // 0 when m_used = -inf
+        if (!first_tile && __any_sync(0xffffffffu, need)) {
+          // O holds earlier tiles at the old reference: wait for them, then the
+          // whole warp rescales its rows (alpha = 1 for rows that keep theirs)
+          if (!(ok = warp_wait(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
+          tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float v[32];
-              tmem_ld32(trow + 256 + c * 32, v);
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(trow + 256 + c * 32, v);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= alpha;
-              tmem_st32(trow + 256 + c * 32, v);
-            }
-            tmem_wait_st();
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st32(trow + 256 + c * 32, v);
           }
+          tmem_wait_st();
+        }
+        if (need) {
           l *= alpha;
           m_used = m_new;
         }
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         }
         l += psum;
         // the P buffer was last read by the PV of tile gt - 2
-        if (gt >= 2 && !(ok = wait_bar(&bs->pv_done[sb], ((gt - 2) >> 1) & 1, bs, err))) break;
+        if (gt >= 2 && !(ok = warp_wait(&bs->pv_done[sb], ((gt - 2) >> 1) & 1, bs, err))) break;
         uint8_t* prow = smem + L::p0 + sb * L::kP + r * 128;
 #pragma unroll
         for (int ch = 0; ch < kTileN / 8; ++ch) {
@@ -520,7 +531,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
       }
       if (!ok) break;
       // epilogue: O / l for this row, once every PV of the item has completed
-      if (!(ok = wait_bar(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
+      if (!(ok = warp_wait(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = o + (static_cast<int64_t>(h) * n + tok) * D;

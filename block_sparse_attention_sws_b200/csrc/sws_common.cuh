@@ -67,13 +67,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: about a second at most (each try_wait suspends for a short,
-// hardware-chosen time). Returns false, after recording the guard, on timeout.
-constexpr uint32_t kWaitLimit = 1u << 22;
+// try_wait that suspends at most `hint_ns` nanoseconds before reporting "not yet".
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits are bounded in wall time (the global nanosecond timer), never by an
+// iteration count: a wait that has not completed after kWaitNs gives up.
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
+constexpr uint32_t kSuspendNs = 20000;       // at most 20 us per try
+
+// Bounded wait. Returns false, after recording the guard, on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, kSuspendNs)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
   }
   record_error(err, GUARD_MBAR_TIMEOUT);
   return false;
