@@ -69,7 +69,7 @@ def load() -> ctypes.CDLL:
         "sws_projection_device": (P, [P]),
         "sws_launch_count": (U64, []),
         "sws_sync_check": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
-        "sws_sketch": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P]),
+        "sws_sketch": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, SZ, P]),
         "sws_walk_select": (ctypes.c_int, [P, P, I64, I32, ctypes.c_int, P, P, P, P, SZ, P]),
         "sws_sparse_attn_prefill": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, SZ, P]),
         "sws_decode_init_cache": (ctypes.c_int, [P, P, I32, I32, I64, P, P, P, P]),
@@ -198,11 +198,11 @@ def sws_sync_check(h: Handle, stream=None) -> int:
 
 # --------------------------------------------------------------- prefill ----
 
-def sws_sketch(h: Handle, q, k, q_sk, k_sk, scores, stream=None) -> None:
+def sws_sketch(h: Handle, q, k, q_sk, k_sk, scores, ws, stream=None) -> None:
     hq, n, _ = q.shape
     hkv = k.shape[0]
     _check(load().sws_sketch(h.ptr, _ptr(q), _ptr(k), _dtype_code(q), n, hq, hkv, _ptr(q_sk), _ptr(k_sk),
-                             _ptr(scores), _stream(stream)), "sws_sketch")
+                             _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sws_sketch")
 
 
 def sws_walk_select(h: Handle, scores, n: int, first_layer: bool, walk_state, row_ptr, col_idx, ws,

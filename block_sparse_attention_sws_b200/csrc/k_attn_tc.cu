@@ -4,22 +4,24 @@
 // Q, K, V restricted to the key blocks selected for each query block (query
 // token t sees key token u of a selected block iff u <= t).
 //
-// One persistent CTA per SM walks (head, 128-row query tile) work items, longest
-// first. A tile is one query block (B = 128) or two adjacent query blocks
-// (B = 64, whose selections overlap almost entirely): their CSR rows are merged
-// and consecutive key blocks of the union are paired into 128-key tiles with a
-// per-(query half, key half) selection mask.
+// One persistent CTA per SM walks (head, 256-row query slab) work items,
+// longest first. A slab is two 128-row query tiles that share one stream of
+// 128-key tiles: the merged CSR rows of its query blocks (4 blocks of 64 or 2
+// of 128; adjacent query blocks select almost the same key blocks), each key
+// tile carrying a selection bit per (key block, query block) pair.
 //
-// Warp roles (192 threads):
-//   warp 0    TMA producer: Q tile once per item, K and V tiles into a 2-stage
-//             ring (3-D tensor maps, 128-byte swizzle, zero fill past n);
-//   warp 1    owns 512 TMEM columns and issues tcgen05.mma from one thread:
-//             S = Q K^T into one of two TMEM S buffers, then O += P V;
-//   warps 2-5 softmax, one query row per thread (TMEM lane = row): reads S,
-//             masks, keeps a running max that is only moved when it grows by
-//             more than 2^8 (then the row of O in TMEM is rescaled), writes
-//             P = 2^(s - m) as bf16 into one of two swizzled shared buffers,
-//             and finally writes O / l.
+// Warp roles (320 threads):
+//   warp 0    TMA producer: both Q tiles once per item, then K and V tiles into
+//             a 2-stage ring (3-D tensor maps, 128-byte swizzle, zero fill past n);
+//   warp 1    owns the 512 TMEM columns and issues tcgen05.mma from one thread,
+//             alternating between the two query tiles w: S_w = Q_w K^T into TMEM,
+//             then O_w += P_w V with P_w read from TMEM (it overwrites S_w);
+//   warps 2-5 and 6-9: one softmax warpgroup per query tile, one query row per
+//             thread (TMEM lane = row). While one group works on its S, the
+//             tensor cores run the other group's products. A row keeps a running
+//             max that only moves when it grows by more than 2^8 (then its row of
+//             O in TMEM is rescaled); P = 2^(s - m) is written back to TMEM as
+//             bf16; the group finally writes O / l.
 // Every wait is bounded; a timeout records a guard code and all roles leave.
 #include <cuda.h>
 
@@ -30,9 +32,10 @@
 namespace sws {
 namespace {
 
-constexpr int kTcThreads = 192;
-constexpr int kTileM = 128;  // query rows per item
-constexpr int kTileN = 128;  // keys per S tile
+constexpr int kTcThreads = 320;
+constexpr int kTileM = 128;   // query rows per tile (two tiles per item)
+constexpr int kTileN = 128;   // keys per S tile
+constexpr int kGroup = 128;   // threads per softmax warpgroup
 constexpr float kRescaleLog2 = 8.0f;
 
 // ---- PTX wrappers --------------------------------------------------------------
@@ -127,19 +130,38 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
          (static_cast<uint32_t>(kTileM >> 4) << 24);
 }
 
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Stores 16 packed words into 16 consecutive columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 // ---- shared state ----------------------------------------------------------------
 
 struct TileMeta {
-  int32_t u0, u1;  // key blocks of the two key halves (B = 64) or the key block (B = 128)
-  int32_t mask;    // bit (2 * key_half + query_half): that query block selected that key block
+  int32_t u0, u1;  // key blocks of the two 64-key halves (B = 64), or the key block twice (B = 128)
+  int32_t mask;    // bit (key_block_slot * QB + query_block_slot): that query block selected that key block
   int32_t last;    // last key tile of the item
 };
 
 struct Bars {
-  uint64_t q_full, q_empty, o_empty;
+  uint64_t q_full, q_empty;
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_empty[2];  // per query tile
   TileMeta meta[2];
   uint32_t tmem_base;
   volatile int32_t abort;
@@ -147,16 +169,18 @@ struct Bars {
 
 template <int D>
 struct Smem {
-  static constexpr uint32_t kQ = kTileM * D * 2;
+  static constexpr uint32_t kQ = kTileM * D * 2;  // one query tile
   static constexpr uint32_t kK = kTileN * D * 2;
-  static constexpr uint32_t kP = kTileM * kTileN * 2;
-  static constexpr uint32_t q = 0;
-  static constexpr uint32_t k0 = q + kQ;
+  static constexpr uint32_t q = 0;                // two query tiles
+  static constexpr uint32_t k0 = q + 2 * kQ;
   static constexpr uint32_t v0 = k0 + 2 * kK;
-  static constexpr uint32_t p0 = v0 + 2 * kK;
-  static constexpr uint32_t bars = p0 + 2 * kP;
+  static constexpr uint32_t bars = v0 + 2 * kK;
   static constexpr uint32_t total = bars + sizeof(Bars);
 };
+
+// TMEM columns: S_w at 128 w (P_w packed over its first 64 columns), O_w at 256 + 128 w.
+__host__ __device__ constexpr uint32_t tcol_s(int w) { return 128u * w; }
+__host__ __device__ constexpr uint32_t tcol_o(int w) { return 256u + 128u * w; }
 
 // Bounded wait (wall time) that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int32_t* err) {
@@ -178,85 +202,79 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
   return __all_sync(0xffffffffu, wait_bar(bar, parity, bs, err));
 }
 
-// Walks the key tiles of one item: for B = 128 the CSR row of query block m;
-// for B = 64 the merge of rows 2m and 2m+1, two union blocks per tile.
+// Walks the key tiles of one item: the merge of the CSR rows of its QB query
+// blocks; B = 128: one key block per tile, B = 64: two union blocks per tile.
 template <int BLK>
 struct TileWalker {
-  const int32_t* c0;
-  const int32_t* c1;
-  int32_t n0, n1, p0, p1, last0, last1, i0, i1;
+  static constexpr int QB = 256 / BLK;
+  const int32_t* c[QB];
+  int32_t cnt[QB], pos[QB], last[QB], row[QB];
   int32_t* err;
 
-  __device__ void init(const int32_t* row_ptr, const int32_t* cols, int64_t b, int64_t nnz, int32_t m, int32_t* e) {
+  __device__ void init(const int32_t* row_ptr, const int32_t* cols, int64_t b, int64_t nnz, int32_t p, int32_t* e) {
     err = e;
-    if constexpr (BLK == 128) {
-      i0 = m;
-      i1 = -1;
-    } else {
-      i0 = 2 * m;
-      i1 = (2 * m + 1 < b) ? 2 * m + 1 : -1;
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      const int64_t i = static_cast<int64_t>(p) * QB + q;
+      row[q] = static_cast<int32_t>(i);
+      pos[q] = 0;
+      last[q] = -1;
+      c[q] = cols;
+      cnt[q] = 0;
+      if (i < b) {
+        int32_t a = row_ptr[i], z = row_ptr[i + 1];
+        if (a < 0 || z < a || z > nnz) {
+          record_error(err, GUARD_BAD_CSR);
+          a = z = 0;
+        }
+        c[q] = cols + a;
+        cnt[q] = z - a;
+      }
     }
-    auto row = [&](int32_t i, const int32_t*& c, int32_t& cnt) {
-      if (i < 0) {
-        c = cols;
-        cnt = 0;
-        return;
-      }
-      int32_t a = row_ptr[i], z = row_ptr[i + 1];
-      if (a < 0 || z < a || z > nnz) {
-        record_error(err, GUARD_BAD_CSR);
-        a = z = 0;
-      }
-      c = cols + a;
-      cnt = z - a;
-    };
-    row(i0, c0, n0);
-    row(i1, c1, n1);
-    p0 = p1 = 0;
-    last0 = last1 = -1;
   }
-  // next valid entry of a row (in [0, i], strictly ascending), or INT_MAX
-  __device__ int32_t peek(const int32_t* c, int32_t n, int32_t& p, int32_t& last, int32_t i) {
-    while (p < n) {
-      const int32_t v = c[p];
-      if (v >= 0 && v <= i && v > last) return v;
+  // next valid entry of row q (in [0, i], strictly ascending), or INT_MAX
+  __device__ int32_t peek(int q) {
+    while (pos[q] < cnt[q]) {
+      const int32_t v = c[q][pos[q]];
+      if (v >= 0 && v <= row[q] && v > last[q]) return v;
       record_error(err, GUARD_BAD_CSR);
-      ++p;
+      ++pos[q];
     }
     return 0x7fffffff;
   }
-  // next union block and its 2-bit mask (bit 0: row i0, bit 1: row i1); false when done
+  // next union block and its QB-bit mask; false when done
   __device__ bool next_block(int32_t& blk, int32_t& msk) {
-    const int32_t a = peek(c0, n0, p0, last0, i0);
-    const int32_t z = (i1 >= 0) ? peek(c1, n1, p1, last1, i1) : 0x7fffffff;
-    if (a == 0x7fffffff && z == 0x7fffffff) return false;
-    blk = min(a, z);
+    int32_t h[QB];
+    int32_t mn = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      h[q] = peek(q);
+      mn = min(mn, h[q]);
+    }
+    if (mn == 0x7fffffff) return false;
+    blk = mn;
     msk = 0;
-    if (a == blk) {
-      msk |= 1;
-      last0 = a;
-      ++p0;
-    }
-    if (z == blk) {
-      msk |= 2;
-      last1 = z;
-      ++p1;
-    }
+#pragma unroll
+    for (int q = 0; q < QB; ++q)
+      if (h[q] == mn) {
+        msk |= 1 << q;
+        last[q] = mn;
+        ++pos[q];
+      }
     return true;
   }
-  // next key tile; returns false when the item has no tile left
   __device__ bool next_tile(TileMeta& t) {
     int32_t b0, m0;
     if (!next_block(b0, m0)) return false;
     t.u0 = b0;
     if constexpr (BLK == 128) {
       t.u1 = b0;
-      t.mask = 1;
+      t.mask = m0;
     } else {
       int32_t b1, m1;
       if (next_block(b1, m1)) {
         t.u1 = b1;
-        t.mask = m0 | (m1 << 2);
+        t.mask = m0 | (m1 << QB);
       } else {
         t.u1 = b0;
         t.mask = m0;
@@ -272,25 +290,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmv, int64_t n, int32_t hq, int32_t group, const int32_t* __restrict__ row_ptr,
     const int32_t* __restrict__ col_idx, int64_t nnz, __nv_bfloat16* __restrict__ o, float qscale, int32_t* err) {
   using L = Smem<D>;
+  constexpr int QB = 256 / BLK;  // query blocks per item
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bs = reinterpret_cast<Bars*>(smem + L::bars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = ceil_div64(n, BLK);
-  const int32_t ntiles = static_cast<int32_t>(ceil_div64(n, kTileM));
-  const int64_t items = static_cast<int64_t>(ntiles) * hq;
+  const int32_t nslab = static_cast<int32_t>(ceil_div64(n, 2 * kTileM));
+  const int64_t items = static_cast<int64_t>(nslab) * hq;
 
   if (threadIdx.x == 0) {
     mbar_init(&bs->q_full, 1);
     mbar_init(&bs->q_empty, 1);
-    mbar_init(&bs->o_empty, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bs->kv_full[s], 1);
       mbar_init(&bs->kv_empty[s], 1);
       mbar_init(&bs->s_full[s], 1);
-      mbar_init(&bs->s_empty[s], 128);
-      mbar_init(&bs->p_full[s], 128);
+      mbar_init(&bs->p_full[s], kGroup);
       mbar_init(&bs->pv_done[s], 1);
+      mbar_init(&bs->o_empty[s], kGroup);
     }
     bs->abort = 0;
     mbar_fence_init();
@@ -305,8 +323,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
   tc_fence_after();
   const uint32_t tmem = bs->tmem_base;
 
-  auto item_of = [&](int64_t t, int32_t& h, int32_t& m) {
-    m = ntiles - 1 - static_cast<int32_t>(t / hq);  // longest rows first
+  auto item_of = [&](int64_t t, int32_t& h, int32_t& p) {
+    p = nslab - 1 - static_cast<int32_t>(t / hq);  // longest rows first
     h = static_cast<int32_t>(t % hq);
   };
 
@@ -315,19 +333,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     if (lane == 0) {
       uint32_t kv_it = 0, item_cnt = 0;
       for (int64_t t = blockIdx.x; t < items && !bs->abort; t += gridDim.x, ++item_cnt) {
-        int32_t h, m;
-        item_of(t, h, m);
+        int32_t h, p;
+        item_of(t, h, p);
         const int32_t g = h / group;
         if (!wait_bar(&bs->q_empty, (item_cnt & 1) ^ 1, bs, err)) break;
-        mbar_arrive_expect_tx(&bs->q_full, L::kQ);
+        mbar_arrive_expect_tx(&bs->q_full, 2 * L::kQ);
 #pragma unroll
-        for (int a = 0; a < D / 64; ++a)
-          tma_load_3d(smem + L::q + a * (kTileM * 128), &tmq, a * 64, m * kTileM, h, &bs->q_full);
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(smem + L::q + w * L::kQ + a * (kTileM * 128), &tmq, a * 64, p * 2 * kTileM + w * kTileM, h,
+                        &bs->q_full);
         TileWalker<BLK> wk;
-        wk.init(row_ptr + static_cast<int64_t>(h) * (b + 1), col_idx + static_cast<int64_t>(h) * nnz, b, nnz, m, err);
+        wk.init(row_ptr + static_cast<int64_t>(h) * (b + 1), col_idx + static_cast<int64_t>(h) * nnz, b, nnz, p, err);
         TileMeta cur, nxt;
         bool have = wk.next_tile(cur);
-        if (!have) {  // a corrupt CSR row: keep the pipeline shape with one fully masked tile
+        if (!have) {  // a corrupt CSR: keep the pipeline shape with one fully masked tile
           cur.u0 = cur.u1 = 0;
           cur.mask = 0;
         }
@@ -336,10 +357,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
           const bool more = have && wk.next_tile(nxt);
           cur.last = more ? 0 : 1;
           const int st = kv_it & 1;
-          if (!wait_bar(&bs->kv_empty[st], ((kv_it >> 1) & 1) ^ 1, bs, err)) {
-            done = true;
-            break;
-          }
+          if (!wait_bar(&bs->kv_empty[st], ((kv_it >> 1) & 1) ^ 1, bs, err)) break;
           bs->meta[st] = cur;
           mbar_arrive_expect_tx(&bs->kv_full[st], 2 * L::kK);
           uint8_t* ks = smem + L::k0 + st * L::kK;
@@ -367,195 +385,186 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileN, false);
       constexpr uint32_t idPV = idesc_bf16(D, true);
-      const uint32_t sq = smem_u32(smem + L::q);
       uint32_t kv_it = 0, gt = 0, item_cnt = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x, ++item_cnt) {
         if (!(ok = wait_bar(&bs->q_full, item_cnt & 1, bs, err))) break;
-        int32_t prev_st = -1;
-        uint32_t prev_gt = 0;
-        bool first_pv = true;
-        auto issue_pv = [&](int st, uint32_t tile) -> bool {
-          const int pb = tile & 1;
-          if (!wait_bar(&bs->p_full[pb], (tile >> 1) & 1, bs, err)) return false;
-          if (first_pv && !wait_bar(&bs->o_empty, (item_cnt & 1) ^ 1, bs, err)) return false;
-          tc_fence_after();
-          const uint32_t sp = smem_u32(smem + L::p0 + pb * L::kP);
-          const uint32_t sv = smem_u32(smem + L::v0 + st * L::kK);
-#pragma unroll
-          for (int kk = 0; kk < kTileN / 16; ++kk) {
-            const uint64_t ad = sw128_desc(sp + (kk >> 2) * (kTileM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(sv + kk * 16 * 128, kTileN * 128, 1024);
-            tc_mma(tmem + 256, ad, bd, idPV, (first_pv && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(&bs->pv_done[pb]);
-          tc_commit(&bs->kv_empty[st]);
-          first_pv = false;
-          return true;
-        };
-        while (true) {
+        bool first = true;
+        while (ok) {
           const int st = kv_it & 1;
           if (!(ok = wait_bar(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
           const bool last = bs->meta[st].last != 0;
-          const int sb = gt & 1;
-          if (!(ok = wait_bar(&bs->s_empty[sb], ((gt >> 1) & 1) ^ 1, bs, err))) break;
-          tc_fence_after();
           const uint32_t sk = smem_u32(smem + L::k0 + st * L::kK);
+          const uint32_t sv = smem_u32(smem + L::v0 + st * L::kK);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
-            const uint32_t koff = (kk >> 2) * (kTileN * 128) + (kk & 3) * 32;
-            tc_mma(tmem + sb * kTileN, sw128_desc(sq + off, 16, 1024), sw128_desc(sk + koff, 16, 1024), idS,
-                   kk > 0 ? 1u : 0u);
+          for (int w = 0; w < 2; ++w) {
+            // S_w overwrites the columns that held P_w of the previous tile
+            if (gt > 0 && !(ok = wait_bar(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + L::q + w * L::kQ);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
+              const uint32_t koff = (kk >> 2) * (kTileN * 128) + (kk & 3) * 32;
+              tc_mma(tmem + tcol_s(w), sw128_desc(sq + off, 16, 1024), sw128_desc(sk + koff, 16, 1024), idS,
+                     kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bs->s_full[w]);
           }
-          tc_commit(&bs->s_full[sb]);
+          if (!ok) break;
           if (last) tc_commit(&bs->q_empty);
-          if (prev_st >= 0 && !(ok = issue_pv(prev_st, prev_gt))) break;
-          prev_st = st;
-          prev_gt = gt;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            if (!(ok = wait_bar(&bs->p_full[w], gt & 1, bs, err))) break;
+            if (first && !(ok = wait_bar(&bs->o_empty[w], (item_cnt & 1) ^ 1, bs, err))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTileN / 16; ++kk)
+              tc_mma_ts(tmem + tcol_o(w), tmem + tcol_s(w) + kk * 8, sw128_desc(sv + kk * 16 * 128, kTileN * 128, 1024),
+                        idPV, (first && kk == 0) ? 0u : 1u);
+            tc_commit(&bs->pv_done[w]);
+          }
+          if (!ok) break;
+          tc_commit(&bs->kv_empty[st]);
+          first = false;
           ++kv_it;
           ++gt;
-          if (last) {
-            ok = issue_pv(prev_st, prev_gt);
-            break;
-          }
+          if (last) break;
         }
       }
     }
   } else {
     // -------------------------------------------------------------- softmax --
-    const int q4 = warp & 3;        // TMEM lane quarter of this warp
-    const int r = q4 * 32 + lane;   // query row of the tile
+    const int w = (warp - 2) >> 2;          // query tile of this warpgroup
+    const int q4 = warp & 3;                // TMEM lane quarter of this warp
+    const int r = q4 * 32 + lane;           // query row of the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    uint32_t kv_it = 0, gt = 0;
+    const uint32_t ts = trow + tcol_s(w), to = trow + tcol_o(w);
+    const int qslot = (w * kTileM + r) / BLK;  // query block slot within the item
+    uint32_t kv_it = 0, gt = 0, item_cnt = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x) {
-      int32_t h, m;
-      item_of(t, h, m);
-      const int64_t tok = static_cast<int64_t>(m) * kTileM + r;
-      const int qh = r >> 6;  // query half (B = 64)
+    for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x, ++item_cnt) {
+      int32_t h, p;
+      item_of(t, h, p);
+      const int64_t tok = static_cast<int64_t>(p) * 2 * kTileM + w * kTileM + r;
+      const int64_t qi = static_cast<int64_t>(p) * QB + qslot;  // query block of this row
       float m_used = -INFINITY, l = 0.f;
       bool first_tile = true;
       while (true) {
         const int st = kv_it & 1;
         if (!(ok = warp_wait(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
         const TileMeta tm = bs->meta[st];
-        const int sb = gt & 1;
-        if (!(ok = warp_wait(&bs->s_full[sb], (gt >> 1) & 1, bs, err))) break;
+        if (!(ok = warp_wait(&bs->s_full[w], gt & 1, bs, err))) break;
         tc_fence_after();
         float s[kTileN];
 #pragma unroll
         for (int c = 0; c < kTileN / 32; ++c) {
           float v[32];
-          tmem_ld32(trow + sb * kTileN + c * 32, v);
+          tmem_ld32(ts + c * 32, v);  // the wait is inside: registers valid on return
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
         }
-        tc_fence_before();
-        mbar_arrive(&bs->s_empty[sb]);
-        // masks: 0 = none, 1 = all, 2 = causal (key offset <= query offset)
-        int mode[2];
-        int limit[2];
-        if constexpr (BLK == 128) {
-          mode[0] = mode[1] = (tm.u0 < m) ? 1 : 2;
-          limit[0] = r;
-          limit[1] = r - 64;
-        } else {
-          const int qi = 2 * m + qh;
+        // masks per key block slot: 0 = none, 1 = all, 2 = causal (key offset <= query offset)
+        constexpr int KBS = kTileN / BLK;
+        int mode[KBS];
 #pragma unroll
-          for (int kh = 0; kh < 2; ++kh) {
-            const int kb = kh ? tm.u1 : tm.u0;
-            const bool sel = (tm.mask >> (2 * kh + qh)) & 1;
-            mode[kh] = !sel ? 0 : (kb < qi ? 1 : (kb == qi ? 2 : 0));
-            limit[kh] = r & 63;
+        for (int kb = 0; kb < KBS; ++kb) {
+          const int64_t ub = kb ? tm.u1 : tm.u0;
+          const bool sel = (tm.mask >> (kb * QB + qslot)) & 1;
+          mode[kb] = !sel ? 0 : (ub < qi ? 1 : (ub == qi ? 2 : 0));
+        }
+        const int qoff = r & (BLK - 1);  // offset of the row inside its query block
+#pragma unroll
+        for (int kb = 0; kb < KBS; ++kb) {
+          if (mode[kb] != 1) {
+#pragma unroll
+            for (int c = 0; c < BLK; ++c)
+              s[kb * BLK + c] = (mode[kb] == 2 && c <= qoff) ? s[kb * BLK + c] : -INFINITY;
           }
         }
-        float mx = -INFINITY;
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kTileN; ++c) {
-          const int kh = c >> 6;
-          const int cc = (BLK == 128) ? c : (c & 63);
-          const bool valid = mode[kh] == 1 || (mode[kh] == 2 && cc <= ((BLK == 128) ? r : limit[kh]));
-          s[c] = valid ? s[c] : -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
+        for (int u = 0; u < 8; ++u) mx8[u] = s[u];
+#pragma unroll
+        for (int c = 8; c < kTileN; c += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], s[c + u]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = mx * qscale;
         const bool need = mx != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2);
         const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;  // 0 when m_used = -inf
-        if (!first_tile && __any_sync(0xffffffffu, need)) {
-          // O holds earlier tiles at the old reference: wait for them, then the
-          // whole warp rescales its rows (alpha = 1 for rows that keep theirs)
-          if (!(ok = warp_wait(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float v[32];
-            tmem_ld32(trow + 256 + c * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= alpha;
-            tmem_st32(trow + 256 + c * 32, v);
-          }
-          tmem_wait_st();
-        }
         if (need) {
           l *= alpha;
           m_used = m_new;
         }
-        // P = 2^(s * qscale - m_used); masked entries and an unset reference give 0
-        float psum = 0.f;
-        uint32_t pk[kTileN / 2];
+        // P = 2^(s * qscale - m_used), bf16, over the first 64 columns of S_w
+        const bool live = m_used != -INFINITY;
+        const float nm = live ? -m_used : 0.f;
+        float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kTileN; c += 2) {
-          const float p0 = (m_used == -INFINITY) ? 0.f : fast_exp2(fmaf(s[c], qscale, -m_used));
-          const float p1 = (m_used == -INFINITY) ? 0.f : fast_exp2(fmaf(s[c + 1], qscale, -m_used));
-          psum += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        l += psum;
-        // the P buffer was last read by the PV of tile gt - 2
-        if (gt >= 2 && !(ok = warp_wait(&bs->pv_done[sb], ((gt - 2) >> 1) & 1, bs, err))) break;
-        uint8_t* prow = smem + L::p0 + sb * L::kP + r * 128;
+        for (int qt = 0; qt < 4; ++qt) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int ch = 0; ch < kTileN / 8; ++ch) {
-          const int atom = ch >> 3, cc = ch & 7;
-          uint4 v = make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-          *reinterpret_cast<uint4*>(prow + atom * (kTileM * 128) + ((cc ^ (r & 7)) << 4)) = v;
+          for (int i = 0; i < 16; ++i) {
+            const int c = qt * 32 + 2 * i;
+            const float p0 = live ? fast_exp2(fmaf(s[c], qscale, nm)) : 0.f;
+            const float p1 = live ? fast_exp2(fmaf(s[c + 1], qscale, nm)) : 0.f;
+            ps8[i & 7] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16u(ts + qt * 16, pk);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        if (!first_tile && __any_sync(0xffffffffu, need)) {
+          // O_w holds earlier tiles at the old reference: wait for them, then the
+          // whole warp rescales its rows (alpha = 1 for rows that keep theirs)
+          if (!(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(to + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st32(to + c * 32, v);
+          }
+        }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bs->p_full[sb]);
+        mbar_arrive(&bs->p_full[w]);
         first_tile = false;
         ++kv_it;
         ++gt;
         if (tm.last) break;
       }
       if (!ok) break;
-      // epilogue: O / l for this row, once every PV of the item has completed
-      if (!(ok = warp_wait(&bs->pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, bs, err))) break;
+      // epilogue: O_w / l for this row, once every PV of the item has completed
+      if (!(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = o + (static_cast<int64_t>(h) * n + tok) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
-        tmem_ld32(trow + 256 + c * 32, v);
+        tmem_ld32(to + c * 32, v);
         if (tok < n) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 w = make_uint4(pack_bf16x2(v[q * 8 + 0] * inv, v[q * 8 + 1] * inv),
+            uint4 u = make_uint4(pack_bf16x2(v[q * 8 + 0] * inv, v[q * 8 + 1] * inv),
                                  pack_bf16x2(v[q * 8 + 2] * inv, v[q * 8 + 3] * inv),
                                  pack_bf16x2(v[q * 8 + 4] * inv, v[q * 8 + 5] * inv),
                                  pack_bf16x2(v[q * 8 + 6] * inv, v[q * 8 + 7] * inv));
-            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = w;
+            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = u;
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&bs->o_empty);
+      mbar_arrive(&bs->o_empty[w]);
     }
   }
   // teardown: the softmax warps waited for the last PV of their last item, and
-  // MMAs complete in issue order, so no MMA is in flight past this barrier
+  // that completion covers every earlier MMA of this CTA
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -610,7 +619,7 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
   const int64_t b = ceil_div64(n, BLK);
   int64_t nnz = 0;
   for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
-  const int64_t items = ceil_div64(n, kTileM) * hq;
+  const int64_t items = ceil_div64(n, 2 * kTileM) * hq;
   const int grid = static_cast<int>(std::min<int64_t>(items, h->num_sms));
   const float qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
   kern<<<grid, kTcThreads, smem, st>>>(mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx, nnz,
@@ -620,8 +629,6 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
 }
 
 }  // namespace
-
-size_t attn_prefill_tc_smem_bytes(int d) { return (d == 128 ? Smem<128>::total : Smem<64>::total) + 1024; }
 
 cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
                                    int32_t hq, int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o,

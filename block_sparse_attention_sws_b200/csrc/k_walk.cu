@@ -38,9 +38,12 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) / sum : 0.0;
 }
 
-// C = A * Bm for lower-triangular b x b matrices, one 64 x 64 output tile per
-// CTA, 64 threads with 8 x 8 accumulators each, k staged 8 at a time.
-constexpr int kTT = 64, kTK = 8;
+// C = A * Bm for lower-triangular b x b matrices. One 32 x 32 output tile per
+// CTA (on or below the diagonal, heaviest first), 64 threads with 4 x 4
+// accumulators each, k staged 16 at a time through shared memory with the next
+// chunk prefetched into registers. Entries above the diagonal of A and Bm are
+// treated as zero whatever the buffers hold.
+constexpr int kTT = 32, kTK = 16, kGemmThreads = 64;
 
 __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int64_t& tj) {
   // heaviest tiles (largest ti - tj) first
@@ -52,8 +55,10 @@ __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int6
   ti = tj = 0;
 }
 
-__global__ void __launch_bounds__(64) tri_gemm_kernel(const double* __restrict__ A, const double* __restrict__ Bm,
-                                                      double* __restrict__ C, int64_t b) {
+__global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __restrict__ A,
+                                                                const double* __restrict__ Bm,
+                                                                double* __restrict__ C, int64_t b) {
+  constexpr int PER = kTT * kTK / kGemmThreads;  // elements of each operand chunk per thread
   __shared__ __align__(16) double As[2][kTK][kTT];  // k-major
   __shared__ __align__(16) double Bs[2][kTK][kTT];
   const int64_t nt = ceil_div64(b, kTT);
@@ -64,37 +69,37 @@ __global__ void __launch_bounds__(64) tri_gemm_kernel(const double* __restrict__
   const double* Bh = Bm + hoff;
   double* Ch = C + hoff;
   const int tid = threadIdx.x;
-  const int tr = tid / 8, tc = tid % 8;
+  const int tr = tid / (kTT / 4), tc = tid % (kTT / 4);
   const int64_t i0 = ti * kTT, j0 = tj * kTT;
   const int64_t kbeg = j0, kend = std::min<int64_t>(b, i0 + kTT);
 
-  double ra[kTK], rb[kTK];
+  double ra[PER], rb[PER];
   auto load = [&](int64_t k0) {
-    // A: thread owns row i0 + tid, 8 consecutive k
-    const int64_t ar = i0 + tid;
 #pragma unroll
-    for (int q = 0; q < kTK; ++q) {
-      const int64_t kk = k0 + q;
-      ra[q] = (ar < b && kk < kend && kk <= ar) ? Ah[ar * b + kk] : 0.0;  // lower triangle only
+    for (int q = 0; q < PER; ++q) {
+      const int e = tid + q * kGemmThreads;
+      // A: element (row e % T, k e / T)
+      const int64_t ar = i0 + e % kTT, ak = k0 + e / kTT;
+      ra[q] = (ar < b && ak < kend && ak <= ar) ? Ah[ar * b + ak] : 0.0;
+      // B: element (k e / T, column e % T)
+      const int64_t bk = k0 + e / kTT, bc = j0 + e % kTT;
+      rb[q] = (bk < kend && bc < b && bc <= bk) ? Bh[bk * b + bc] : 0.0;
     }
-    // B: row k0 + tid/8, 8 consecutive columns starting at (tid%8)*8
-    const int64_t br = k0 + tid / 8;
-    const int64_t bc = j0 + (tid % 8) * 8;
-#pragma unroll
-    for (int q = 0; q < kTK; ++q) rb[q] = (br < kend && bc + q < b && bc + q <= br) ? Bh[br * b + bc + q] : 0.0;
   };
   auto store = [&](int buf) {
 #pragma unroll
-    for (int q = 0; q < kTK; ++q) As[buf][q][tid] = ra[q];
-#pragma unroll
-    for (int q = 0; q < kTK; ++q) Bs[buf][tid / 8][(tid % 8) * 8 + q] = rb[q];
+    for (int q = 0; q < PER; ++q) {
+      const int e = tid + q * kGemmThreads;
+      As[buf][e / kTT][e % kTT] = ra[q];
+      Bs[buf][e / kTT][e % kTT] = rb[q];
+    }
   };
 
-  double acc[8][8];
+  double acc[4][4];
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
+  for (int u = 0; u < 4; ++u)
 #pragma unroll
-    for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
 
   int buf = 0;
   load(kbeg);
@@ -105,21 +110,16 @@ __global__ void __launch_bounds__(64) tri_gemm_kernel(const double* __restrict__
     if (more) load(k0 + kTK);
 #pragma unroll
     for (int q = 0; q < kTK; ++q) {
-      double a[8], bv[8];
-      const double2* ap = reinterpret_cast<const double2*>(&As[buf][q][tr * 8]);
-      const double2* bp = reinterpret_cast<const double2*>(&Bs[buf][q][tc * 8]);
+      const double2 a01 = *reinterpret_cast<const double2*>(&As[buf][q][tr * 4]);
+      const double2 a23 = *reinterpret_cast<const double2*>(&As[buf][q][tr * 4 + 2]);
+      const double2 b01 = *reinterpret_cast<const double2*>(&Bs[buf][q][tc * 4]);
+      const double2 b23 = *reinterpret_cast<const double2*>(&Bs[buf][q][tc * 4 + 2]);
+      const double a[4] = {a01.x, a01.y, a23.x, a23.y};
+      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const double2 x = ap[u], y = bp[u];
-        a[2 * u] = x.x;
-        a[2 * u + 1] = x.y;
-        bv[2 * u] = y.x;
-        bv[2 * u + 1] = y.y;
-      }
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int v = 0; v < 8; ++v) acc[u][v] = fma(a[u], bv[v], acc[u][v]);
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bv[v], acc[u][v]);
     }
     if (more) {
       store(buf ^ 1);
@@ -128,12 +128,12 @@ __global__ void __launch_bounds__(64) tri_gemm_kernel(const double* __restrict__
     }
   }
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int64_t i = i0 + tr * 8 + u;
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = i0 + tr * 4 + u;
     if (i >= b) continue;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const int64_t j = j0 + tc * 8 + v;
+    for (int v = 0; v < 4; ++v) {
+      const int64_t j = j0 + tc * 4 + v;
       if (j < b) Ch[i * b + j] = acc[u][v];
     }
   }
@@ -185,7 +185,7 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
 cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st) {
   const int64_t nt = ceil_div64(b, kTT);
   dim3 grid(static_cast<unsigned>(nt * (nt + 1) / 2), hq);
-  tri_gemm_kernel<<<grid, 64, 0, st>>>(A, Bm, C, b);
+  tri_gemm_kernel<<<grid, kGemmThreads, 0, st>>>(A, Bm, C, b);
   note_launches(1);
   return cudaGetLastError();
 }

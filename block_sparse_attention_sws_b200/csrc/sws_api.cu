@@ -141,6 +141,8 @@ sws_status sws_workspace_size(const sws_config* c, sws_op op, int64_t n, int32_t
   const int64_t b = ceil_div64(n, c->block_size);
   switch (op) {
     case SWS_OP_SKETCH:
+      *bytes = sketch_workspace_bytes(*c, n, hq, hkv);
+      return SWS_OK;
     case SWS_OP_PREFILL_ATTN:
       *bytes = 0;
       return SWS_OK;
@@ -218,17 +220,20 @@ sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code) {
 }
 
 sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n, int32_t hq,
-                      int32_t hkv, double* q_sk, double* k_sk, double* scores, void* stream) {
+                      int32_t hkv, double* q_sk, double* k_sk, double* scores, void* ws, size_t ws_bytes,
+                      void* stream) {
   if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (dtype != SWS_BF16 && dtype != SWS_FP32) return SWS_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sk) || !aligned16(k_sk) || !aligned16(scores))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sk) || !aligned16(k_sk) || !aligned16(scores) ||
+      !aligned16(ws))
     return SWS_ERR_INVALID_ARG;
   const int64_t b = ceil_div64(n, h->cfg.block_size);
   if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
+  if (ws_bytes < sketch_workspace_bytes(h->cfg, n, hq, hkv)) return SWS_ERR_WORKSPACE;
   auto st = static_cast<cudaStream_t>(stream);
-  sws_status s = cuda_status(launch_sketch_pool_project(h, q, dtype, n, hq, q_sk, st), "sketch q");
-  if (s != SWS_OK) return s;
-  s = cuda_status(launch_sketch_pool_project(h, k, dtype, n, hkv, k_sk, st), "sketch k");
+  sws_status s = cuda_status(
+      launch_sketch_means_project(h, q, k, dtype, n, hq, hkv, static_cast<double*>(ws), q_sk, k_sk, st),
+      "sketch means");
   if (s != SWS_OK) return s;
   return cuda_status(launch_sketch_scores(h, q_sk, k_sk, b, hq, hkv, scores, st), "sketch scores");
 }

@@ -30,10 +30,12 @@ class PrefillPath:
         self.col_idx = torch.empty(hq, self.nnz, dtype=torch.int32, device=device)
         ws = L.sws_workspace_size(cfg, L.SWS_OP_WALK_SELECT, n, hq, hkv)
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        wss = L.sws_workspace_size(cfg, L.SWS_OP_SKETCH, n, hq, hkv)
+        self.ws_sketch = torch.empty(max(wss, 16), dtype=torch.uint8, device=device)
         self.o = torch.empty(hq, n, d, dtype=dtype, device=device)
 
     def sketch(self, q, k, stream=None):
-        L.sws_sketch(self.h, q, k, self.q_sk, self.k_sk, self.scores, stream)
+        L.sws_sketch(self.h, q, k, self.q_sk, self.k_sk, self.scores, self.ws_sketch, stream)
 
     def walk_select(self, first_layer: bool, stream=None):
         L.sws_walk_select(self.h, self.scores, self.n, first_layer, self.walk_state, self.row_ptr, self.col_idx,

@@ -96,7 +96,8 @@ def test_projection_matches_oracle(lib, d, k, seed):
 
 def test_workspace_sizes(lib):
     cfg = S.make_config(128, 64, 32)
-    assert S.sws_workspace_size(cfg, S.SWS_OP_SKETCH, 16384, 32, 8) == 0
+    assert S.sws_workspace_size(cfg, S.SWS_OP_SKETCH, 16384, 32, 8) == 40 * 256 * 128 * 8
+    assert S.sws_workspace_size(cfg, S.SWS_OP_PREFILL_ATTN, 16384, 32, 8) == 0
     assert S.sws_workspace_size(cfg, S.SWS_OP_WALK_SELECT, 16384, 32, 8) == 4 * 32 * 256 * 256 * 8
     dec = S.sws_workspace_size(cfg, S.SWS_OP_DECODE_ATTN, 131136, 32, 8, 16)
     assert dec > 0 and dec % (130 * 4) == 0
@@ -109,7 +110,7 @@ def test_workspace_sizes(lib):
 def test_null_handle_rejected_without_launch(lib):
     """Host validation fails before any CUDA call, so this runs without a GPU."""
     P = ctypes.c_void_p
-    assert lib.sws_sketch(None, P(16), P(16), 0, 64, 1, 1, P(16), P(16), P(16), None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_sketch(None, P(16), P(16), 0, 64, 1, 1, P(16), P(16), P(16), P(16), 16, None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_walk_select(None, P(16), 64, 1, 1, P(16), P(16), P(16), P(16), 16, None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_sparse_attn_prefill(None, P(16), P(16), P(16), 0, 64, 1, 1, P(16), P(16), P(16), None, 0,
                                        None) == S.SWS_ERR_INVALID_ARG

@@ -189,7 +189,7 @@ def test_invalid_arguments_queue_nothing():
     kk = torch.zeros(3, 256, 128, dtype=torch.bfloat16, device="cuda")  # 4 % 3 != 0
     out = torch.zeros(4, 4, 32, dtype=torch.float64, device="cuda")
     with pytest.raises(S.SwsError) as e:
-        S.sws_sketch(h, q, kk, out, out, out)
+        S.sws_sketch(h, q, kk, out, out, out, torch.zeros(16, dtype=torch.uint8, device="cuda"))
     assert e.value.status == S.SWS_ERR_INVALID_ARG
     ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
     sc = torch.zeros(4, 4, 4, dtype=torch.float64, device="cuda")
