@@ -20,8 +20,6 @@
 namespace sws {
 namespace {
 
-constexpr int kPoolThreads = 256;
-
 // Block means of Q (heads [0, hq)) and K (heads [hq, hq + hkv)):
 // means[(head * nblk + blk) * D + c]. Every warp streams its own items through
 // a private ring of bulk-copy stages: lane l reads 16-byte vectors l, l + 32,
