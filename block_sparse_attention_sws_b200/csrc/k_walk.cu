@@ -8,7 +8,8 @@
 // Everything here is fp64: after a few layers the entries of R that decide the
 // selection are 1e-20 .. 1e-40 of the row maximum, below what fp32 holds.
 // The b x b matrices are lower-triangular, so the GEMM only visits tiles on or
-// below the diagonal and, inside a tile pair, only k in [tile(j), tile(i)].
+// below the diagonal and, inside a tile pair, only k in [tile(j), tile(i)];
+// it runs on the fp64 tensor path.
 #include <algorithm>
 
 #include "select.cuh"
@@ -38,12 +39,15 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) / sum : 0.0;
 }
 
-// C = A * Bm for lower-triangular b x b matrices. One 32 x 32 output tile per
-// CTA (on or below the diagonal, heaviest first), 64 threads with 4 x 4
-// accumulators each, k staged 16 at a time through shared memory with the next
+// C = A * Bm for lower-triangular b x b matrices on the fp64 tensor path
+// (mma.sync m16n8k4 f64). One 64 x 64 output tile per CTA (on or below the
+// diagonal, heaviest first), four warps of 32 x 32, k staged 16 at a time
+// through padded shared memory (conflict-free fragment loads) with the next
 // chunk prefetched into registers. Entries above the diagonal of A and Bm are
 // treated as zero whatever the buffers hold.
-constexpr int kTT = 32, kTK = 16, kGemmThreads = 64;
+constexpr int kTT = 64, kTK = 16, kGemmThreads = 128;
+constexpr int kApad = kTK + 2;   // A tile row stride (doubles)
+constexpr int kBpad = kTT + 8;   // B tile row stride (doubles)
 
 __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int64_t& tj) {
   // heaviest tiles (largest ti - tj) first
@@ -55,12 +59,19 @@ __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int6
   ti = tj = 0;
 }
 
+__device__ __forceinline__ void dmma_16x8x4(double (&c)[4], double a0, double a1, double b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a0), "d"(a1), "d"(b0));
+}
+
 __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __restrict__ A,
                                                                 const double* __restrict__ Bm,
                                                                 double* __restrict__ C, int64_t b) {
-  constexpr int PER = kTT * kTK / kGemmThreads;  // elements of each operand chunk per thread
-  __shared__ __align__(16) double As[2][kTK][kTT];  // k-major
-  __shared__ __align__(16) double Bs[2][kTK][kTT];
+  constexpr int PER = kTT * kTK / kGemmThreads;  // 8 elements of each operand chunk per thread
+  __shared__ __align__(16) double As[2][kTT][kApad];
+  __shared__ __align__(16) double Bs[2][kTK][kBpad];
   const int64_t nt = ceil_div64(b, kTT);
   int64_t ti, tj;
   tile_of(blockIdx.x, nt, ti, tj);
@@ -68,8 +79,9 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
   const double* Ah = A + hoff;
   const double* Bh = Bm + hoff;
   double* Ch = C + hoff;
-  const int tid = threadIdx.x;
-  const int tr = tid / (kTT / 4), tc = tid % (kTT / 4);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int wm = warp >> 1, wn = warp & 1;
   const int64_t i0 = ti * kTT, j0 = tj * kTT;
   const int64_t kbeg = j0, kend = std::min<int64_t>(b, i0 + kTT);
 
@@ -78,8 +90,8 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int e = tid + q * kGemmThreads;
-      // A: element (row e % T, k e / T)
-      const int64_t ar = i0 + e % kTT, ak = k0 + e / kTT;
+      // A: element (row e / KC, k e % KC): 16 consecutive threads read one row
+      const int64_t ar = i0 + e / kTK, ak = k0 + e % kTK;
       ra[q] = (ar < b && ak < kend && ak <= ar) ? Ah[ar * b + ak] : 0.0;
       // B: element (k e / T, column e % T)
       const int64_t bk = k0 + e / kTT, bc = j0 + e % kTT;
@@ -90,16 +102,18 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int e = tid + q * kGemmThreads;
-      As[buf][e / kTT][e % kTT] = ra[q];
+      As[buf][e / kTK][e % kTK] = ra[q];
       Bs[buf][e / kTT][e % kTT] = rb[q];
     }
   };
 
-  double acc[4][4];
+  double acc[2][4][4];
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
+    for (int n8 = 0; n8 < 4; ++n8)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[mt][n8][v] = 0.0;
 
   int buf = 0;
   load(kbeg);
@@ -109,17 +123,19 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
     const bool more = k0 + kTK < kend;
     if (more) load(k0 + kTK);
 #pragma unroll
-    for (int q = 0; q < kTK; ++q) {
-      const double2 a01 = *reinterpret_cast<const double2*>(&As[buf][q][tr * 4]);
-      const double2 a23 = *reinterpret_cast<const double2*>(&As[buf][q][tr * 4 + 2]);
-      const double2 b01 = *reinterpret_cast<const double2*>(&Bs[buf][q][tc * 4]);
-      const double2 b23 = *reinterpret_cast<const double2*>(&Bs[buf][q][tc * 4 + 2]);
-      const double a[4] = {a01.x, a01.y, a23.x, a23.y};
-      const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+    for (int ks = 0; ks < kTK / 4; ++ks) {
+      double a[2][2], bf[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int mt = 0; mt < 2; ++mt) {
+        a[mt][0] = As[buf][wm * 32 + mt * 16 + g][ks * 4 + t4];
+        a[mt][1] = As[buf][wm * 32 + mt * 16 + g + 8][ks * 4 + t4];
+      }
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bv[v], acc[u][v]);
+      for (int n8 = 0; n8 < 4; ++n8) bf[n8] = Bs[buf][ks * 4 + t4][wn * 32 + n8 * 8 + g];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4(acc[mt][n8], a[mt][0], a[mt][1], bf[n8]);
     }
     if (more) {
       store(buf ^ 1);
@@ -128,13 +144,17 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
     }
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t i = i0 + tr * 4 + u;
-    if (i >= b) continue;
+  for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int64_t j = j0 + tc * 4 + v;
-      if (j < b) Ch[i * b + j] = acc[u][v];
+    for (int hh = 0; hh < 2; ++hh) {
+      const int64_t i = i0 + wm * 32 + mt * 16 + g + 8 * hh;
+      if (i >= b) continue;
+#pragma unroll
+      for (int n8 = 0; n8 < 4; ++n8) {
+        const int64_t j = j0 + wn * 32 + n8 * 8 + 2 * t4;
+        if (j < b) Ch[i * b + j] = acc[mt][n8][2 * hh];
+        if (j + 1 < b) Ch[i * b + j + 1] = acc[mt][n8][2 * hh + 1];
+      }
     }
   }
 }
