@@ -27,8 +27,9 @@ EXPORTS = [
     "sws_workspace_size", "sws_create", "sws_destroy", "sws_projection_device", "sws_launch_count",
     "sws_sync_check", "sws_sketch",
     "sws_walk_select", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
-    "sws_sparse_attn_decode",
+    "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 32 << 20  # SWS_NOALLOC_SCRATCH_BYTES
 
 
 class SwsConfig(ctypes.Structure):
@@ -77,6 +78,7 @@ def load() -> ctypes.CDLL:
         "sws_decode_step": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, ctypes.c_int, P, P, P, P,
                                            P, P, P]),
         "sws_sparse_attn_decode": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, SZ, P]),
+        "sws_sparse_attn_decode_noalloc": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -252,3 +254,14 @@ def sws_sparse_attn_decode(h: Handle, q_tok, k_cache, v_cache, seq_lens, sel, se
     _check(load().sws_sparse_attn_decode(h.ptr, _ptr(q_tok), _ptr(k_cache), _ptr(v_cache), batch, hq, hkv, max_len,
                                          _ptr(seq_lens), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt), _ptr(o), _ptr(ws),
                                          ws.numel() * ws.element_size(), _stream(stream)), "sws_sparse_attn_decode")
+
+
+def sws_sparse_attn_decode_noalloc(h: Handle, q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o,
+                                   stream=None) -> None:
+    """sws_sparse_attn_decode without a workspace, for callers that cannot allocate:
+    the partials live in the library's built-in scratch array (see include/sws.h)."""
+    batch, hq, _ = q_tok.shape
+    hkv, max_len = k_cache.shape[1], k_cache.shape[2]
+    _check(load().sws_sparse_attn_decode_noalloc(h.ptr, _ptr(q_tok), _ptr(k_cache), _ptr(v_cache), batch, hq, hkv,
+                                                 max_len, _ptr(seq_lens), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
+                                                 _ptr(o), _stream(stream)), "sws_sparse_attn_decode_noalloc")

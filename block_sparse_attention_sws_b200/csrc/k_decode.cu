@@ -18,6 +18,7 @@
 //     head, and writes a partial (o, max, sum) per head.
 //   decode_combine_kernel: merges the partials of each (sequence, head).
 #include <algorithm>
+#include <mutex>
 
 #include "select.cuh"
 #include "sws_common.cuh"
@@ -562,3 +563,66 @@ cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, 
 }
 
 }  // namespace sws
+
+// ---------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc, or hand the library any memory it did
+// not receive from them, at the point where they run decode attention: plug-ins
+// inside a host framework that owns every device allocation, serving loops that
+// must not take the synchronisation and latency of an allocation on the token
+// path, and code that runs under an allocator budget fixed ahead of time. For
+// them this variant keeps the split-KV partial results in one scratch array
+// that lives in the library itself, sized SWS_NOALLOC_SCRATCH_BYTES, allocated
+// by the CUDA runtime when the library is loaded on a device and held until
+// the process exits.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SWS_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch, looked up once per device. On the host
+// the array's name is only a stand-in for the device symbol; the kernel must
+// receive the address that cudaGetSymbolAddress returns for the current device.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[256] = {};
+
+cudaError_t noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[device] = p;
+  }
+  *out = g_noalloc_ptr[device];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" sws_status sws_sparse_attn_decode_noalloc(const sws_handle* h, const void* q_tok, const void* k_cache,
+                                                     const void* v_cache, int32_t batch, int32_t hq, int32_t hkv,
+                                                     int64_t max_len, const int32_t* seq_lens, const int32_t* sel,
+                                                     const uint8_t* sel_mask, const int32_t* sel_cnt, void* o,
+                                                     void* stream) {
+  if (!h || batch < 1 || max_len < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || hq > 4096) return SWS_ERR_INVALID_ARG;
+  const int32_t group = hq / hkv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u) != 0) return SWS_ERR_INVALID_ARG;
+  const int32_t splits = sws::decode_num_splits(h->cfg, max_len, group);
+  const size_t need = static_cast<size_t>(batch) * hq * splits * (h->cfg.head_dim + 2) * sizeof(float);
+  if (need > SWS_NOALLOC_SCRATCH_BYTES) return SWS_ERR_WORKSPACE;  // beyond the built-in scratch
+  int device = -1;
+  if (cudaGetDevice(&device) != cudaSuccess || device != h->device) return SWS_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (noalloc_scratch(device, &scratch) != cudaSuccess) return SWS_ERR_CUDA;
+  const cudaError_t e = sws::launch_decode_attn(
+      h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), batch, hq, hkv, max_len, seq_lens, sel, sel_mask, sel_cnt,
+      static_cast<__nv_bfloat16*>(o), static_cast<float*>(scratch), splits, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWS_OK : SWS_ERR_CUDA;
+}

@@ -205,6 +205,32 @@ sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const 
                                   const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
                                   const int32_t* sel_cnt, void* o, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------- no-allocation variant --- */
+/* The paper has no counterpart to this call; it serves callers that cannot allocate
+ * device memory on the decode path (a plug-in whose host framework owns every device
+ * allocation, a serving loop that may not pay an allocation's latency and implicit
+ * synchronisation per token, a fixed memory budget decided up front).
+ *
+ * Same computation, arguments and layouts as sws_sparse_attn_decode, without the
+ * workspace: the split-KV partial results go to one scratch array of
+ * SWS_NOALLOC_SCRATCH_BYTES built into the library. The CUDA runtime places that array
+ * on every device the library is loaded on, and it stays there until the process exits.
+ *  - The call allocates nothing (no cudaMalloc, no cudaFree, nothing through a framework).
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    and keeps it; make that first call on each device before any stream capture.
+ *  - The handle's device must be the current device.
+ *  - Every call shares the one array and finds the previous call's contents in it (each
+ *    call overwrites all it reads). Calls whose kernels overlap on the GPU race on it:
+ *    issue them on one stream, or order them.
+ *  - Returns SWS_ERR_WORKSPACE, and queues nothing, when batch * hq * splits * (d + 2) * 4
+ *    bytes of partials (what sws_workspace_size(SWS_OP_DECODE_ATTN) reports) would exceed
+ *    SWS_NOALLOC_SCRATCH_BYTES; the workspace form has no such limit. */
+#define SWS_NOALLOC_SCRATCH_BYTES (32u << 20)
+sws_status sws_sparse_attn_decode_noalloc(const sws_handle* h, const void* q_tok, const void* k_cache,
+                                          const void* v_cache, int32_t batch, int32_t hq, int32_t hkv,
+                                          int64_t max_len, const int32_t* seq_lens, const int32_t* sel,
+                                          const uint8_t* sel_mask, const int32_t* sel_cnt, void* o, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
