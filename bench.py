@@ -43,8 +43,34 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to run (default: the workload's 64)")
+    ap.add_argument("--decode-batch", type=int, default=None, help="smaller decode batch (profiling only)")
+    ap.add_argument("--decode-n0", type=int, default=None, help="shorter cached prompt (profiling only)")
+    ap.add_argument("--decode-layers", type=int, default=None, help="fewer decode layers (profiling only)")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement (profiling only)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
+
+
+def profiled_traffic(name: str, source: str):
+    """DRAM bytes per launch (read + write) recorded in profiles/<name>.md by an
+    ncu capture, if that capture was taken of the current kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", name + ".md")
+    src = os.path.join(ROOT, "block_sparse_attention_sws_b200", "csrc", source)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    fields = {}
+    for line in open(path):
+        if line.startswith("- ") and ": " in line:
+            k, v = line[2:].split(": ", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel source sha256") != digest:
+        return None
+    try:
+        return float(fields["dram bytes per launch (read + write)"])
+    except (KeyError, ValueError):
+        return None
 
 
 def load_peaks():
@@ -333,6 +359,12 @@ def bench_decode(args, world, S, W, torch, peaks):
     wd = W.DECODE_128K
     if args.decode_steps is not None:
         wd = wd.scaled(steps=max(2, min(wd.steps, args.decode_steps)))
+    if args.decode_batch is not None:
+        wd = wd.scaled(batch=args.decode_batch)
+    if args.decode_n0 is not None:
+        wd = wd.scaled(n0=args.decode_n0)
+    if args.decode_layers is not None:
+        wd = wd.scaled(layers=args.decode_layers)
     cfg = S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed)
     h = S.Handle(cfg)
     path = S.DecodePath(h, wd.batch, wd.hq, wd.hkv, wd.max_len, wd.layers)
@@ -409,7 +441,8 @@ def bench_decode(args, world, S, W, torch, peaks):
         "stages_us_per_layer": {"decode_step": statistics.mean(sel_ms) * 1e3, "attention": attn_launch_ms * 1e3},
         "roofline": {"kernel": "sws_sparse_attn_decode (split + combine)", "bound": "hbm",
                      "achieved": attn_bytes / (attn_launch_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                     "frac": attn_bytes / (attn_launch_ms * 1e-3) / 1e9 / hbm, "traffic": None},
+                     "frac": attn_bytes / (attn_launch_ms * 1e-3) / 1e9 / hbm,
+                     "traffic": profiled_traffic("decode_attn_b16_n131072", "k_decode.cu")},
     }
     h.close()
     return out
@@ -429,6 +462,16 @@ def main():
     import sws_inputs as W
     S.load()
     peaks, peak_kind = load_peaks()
+    if args.no_prefill:
+        # profiling run of the decode path alone: not a benchmark line
+        out = {"profiling_only": True, "decode": bench_decode(args, world, S, W, torch, peaks)}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
     pf = bench_prefill(args, world, S, W, torch)
     w = pf["w"]
     ms_step = pf["ms"] / args.steps
@@ -445,7 +488,8 @@ def main():
                    "l2": f"inputs larger than L2 ({pf['in_bytes'] / 1e6:.0f} MB per step)"},
         "stages_ms_per_step": pf["stage"],
         "roofline": {"kernel": "sws_sparse_attn_prefill", "bound": "tensor", "achieved": attn_tflops, "peak": peak_t,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak_t, "traffic": None,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
+                     "traffic": profiled_traffic("attn_tc_prefill_n16384_B64", "k_attn_tc.cu"),
                      "peak_source": f"{peak_kind} bf16 sustained", "flops_per_launch": pf["flops"],
                      "ms_per_launch": pf["attn_ms"]},
         "sketch_roofline": {"bound": "hbm", "achieved": pf["sketch_bytes"] / (pf["stage"]["sketch"] / w.layers * 1e-3) / 1e9,

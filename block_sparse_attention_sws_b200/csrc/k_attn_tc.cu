@@ -29,10 +29,6 @@
 
 #include "sws_common.cuh"
 
-#ifndef SWS_PACK_INT
-#define SWS_PACK_INT 0
-#endif
-
 namespace sws {
 namespace {
 
@@ -40,29 +36,14 @@ constexpr int kTcThreads = 320;
 constexpr int kTileM = 128;   // query rows per tile (two tiles per item)
 constexpr int kTileN = 128;   // keys per S tile
 constexpr int kGroup = 128;   // threads per softmax warpgroup
-#ifndef SWS_WARP_ARRIVE
-#define SWS_WARP_ARRIVE 1
-#endif
-// arrivals per softmax-group barrier phase: one per warp (after __syncwarp) or one per thread
-constexpr int kArrivals = SWS_WARP_ARRIVE ? kGroup / 32 : kGroup;
+// arrivals per softmax-group barrier phase: one per warp, after __syncwarp
+constexpr int kArrivals = kGroup / 32;
 
 __device__ __forceinline__ void group_arrive(uint64_t* bar) {
-#if SWS_WARP_ARRIVE
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-#else
-  mbar_arrive(bar);
-#endif
 }
 constexpr float kRescaleLog2 = 8.0f;
-#ifndef SWS_POLY_EVERY
-#define SWS_POLY_EVERY 0
-#endif
-#ifndef SWS_LD128
-#define SWS_LD128 0
-#endif
-
-constexpr int kPolyEvery = SWS_POLY_EVERY;  // every kPolyEvery-th exponential on the FMA pipe (0: none)
 
 // ---- PTX wrappers --------------------------------------------------------------
 
@@ -134,41 +115,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 8.5: round x to the nearest integer j with the
-// 1.5 * 2^23 shift, evaluate a cubic for 2^f on f = x - j in [-1/2, 1/2], and add
-// j to the exponent field. The cubic is a minimax-style fit of 2^f on
-// [-1/2, 1/2] (iteratively reweighted least squares on Chebyshev nodes):
-// relative error below 7.5e-5, far under the bf16 rounding of P. Arguments
-// below -126 (masked scores included) return about 2^-126: negligible next to
-// the row maximum's 2^0.
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.05517168715596199f, f, 0.2426111400127411f), f, 0.6932609677314758f), f,
-                       0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two non-negative floats to bf16x2 on the integer pipe (round half up: add half
-// an ulp of bf16, keep the high halves), leaving the conversion unit to exp2.
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
-#if SWS_PACK_INT
-  return pack_bf16x2_pos(lo, hi);
-#else
-  return pack_bf16x2(lo, hi);
-#endif
-}
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 "version 1").
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -196,18 +149,6 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint
       : "memory");
 }
 
-// 128 consecutive columns of this thread's lane in one load; the wait for it is
-// in the same statement, so all 128 registers are valid on return.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
-  uint32_t r[128];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // Stores 16 packed words into 16 consecutive columns of this thread's lane.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
@@ -251,34 +192,12 @@ struct Smem {
 __host__ __device__ constexpr uint32_t tcol_s(int w) { return 128u * w; }
 __host__ __device__ constexpr uint32_t tcol_o(int w) { return 256u + 128u * w; }
 
-#ifndef SWS_WAIT_MODE
-#define SWS_WAIT_MODE 1
-#endif
-
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait (wall time) that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bs, int32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
-#if SWS_WAIT_MODE == 0
-    if (mbar_try_wait_hint(bar, parity, kSuspendNs)) return true;
-#elif SWS_WAIT_MODE == 1
     if (mbar_try_wait(bar, parity)) return true;
-#else
-    if (mbar_test_wait(bar, parity)) return true;
-#endif
     if ((it & 15) == 0) {
       if (bs->abort) return false;
       if (global_ns() - t0 > kWaitNs) break;
@@ -571,9 +490,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         if (!(ok = warp_wait(&bs->s_full[w], gt & 1, bs, err))) break;
         tc_fence_after();
         float s[kTileN];
-#if SWS_LD128
-        tmem_ld128(ts, s);
-#else
 #pragma unroll
         for (int c = 0; c < kTileN / 32; ++c) {
           float v[32];
@@ -581,7 +497,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
         }
-#endif
         // masks per key block slot: 0 = none, 1 = all, 2 = causal (key offset <= query offset)
         constexpr int KBS = kTileN / BLK;
         int mode[KBS];
@@ -630,10 +545,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = qt * 32 + 2 * i;
-              constexpr int kPE = kPolyEvery > 0 ? kPolyEvery : 1;
-              const bool poly = kPolyEvery > 0 && ((c + 1) % kPE) == kPE - 1;  // compile-time per element
               const float p0 = fast_exp2(fmaf(s[c], qscale, nm));
-              const float p1 = poly ? poly_exp2(fmaf(s[c + 1], qscale, nm)) : fast_exp2(fmaf(s[c + 1], qscale, nm));
+              const float p1 = fast_exp2(fmaf(s[c + 1], qscale, nm));
               ps8[i & 7] += p0 + p1;
               pk[i] = pack_p(p0, p1);
             }
