@@ -26,6 +26,7 @@ import subprocess
 import sys
 import threading
 import time
+import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -36,7 +37,7 @@ METRIC = "prefill tokens/s + % tensor peak at 20% density; decode step µs + HBM
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
@@ -99,12 +100,18 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
         self.th = threading.Thread(target=self._read, daemon=True)
         self.th.start()
+        # nvidia-smi takes a moment to start: wait for its first sample so that
+        # the samples cover the timed region that follows
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.skip = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -121,7 +128,7 @@ class ClockSampler:
         self.th.join(timeout=2)
         mhz, mx, reasons, watts = [], [], set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[max(0, getattr(self, "skip", 0) - 1):]:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -139,6 +146,11 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
                 "power_w_max": max(watts) if watts else None, "samples": len(mhz), "reasons": sorted(reasons)}
+
+
+def gpu_bus_id(torch) -> str:
+    p = torch.cuda.get_device_properties(torch.cuda.current_device())
+    return f"{getattr(p, 'pci_domain_id', 0):08x}:{getattr(p, 'pci_bus_id', 0):02x}:{getattr(p, 'pci_device_id', 0):02x}.0"
 
 
 # ------------------------------------------------------------- distributed --
@@ -176,31 +188,36 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------ cpu baseline --
 
-def oracle_prefill_sample(w, budget_s: float, max_heads=None):
-    """Times the oracle on whole heads (all layers, every query block) until the
-    budget is spent; returns (seconds, heads done)."""
-    import numpy as np
+def oracle_head_layers(w):
+    """The oracle over the workload one (head, layer) at a time, head by head,
+    each head's walk state carried through its layers; yields the seconds each
+    head-layer took (input generation excluded)."""
     import oracle
     import sws_inputs as W
     from oracle import sws_oracle as so
     Hd = oracle.srht_matrix(w.d, w.k, w.seed)
-    t0 = time.perf_counter()
-    heads = 0
-    limit = w.hq if max_heads is None else max_heads
-    gen_time = 0.0
-    while heads < limit:
+    h = 0
+    while True:
         st = so.PrefillState()
-        h = heads
         for layer in range(w.layers):
-            g0 = time.perf_counter()
-            q, k, v = W.prefill_head_inputs(w, layer, h)
+            q, k, v = W.prefill_head_inputs(w, layer, h % w.hq)
             q64, k64, v64 = (x.double().numpy()[None] for x in (q, k, v))
-            gen_time += time.perf_counter() - g0
+            t0 = time.perf_counter()
             so.prefill_layer(q64, k64, v64, Hd, w.B, w.s, w.density, st, heads=[0], attention_blocks="all")
-        heads += 1
-        if time.perf_counter() - t0 - gen_time >= budget_s:
+            yield time.perf_counter() - t0
+        h += 1
+
+
+def oracle_prefill_sample(w, budget_s: float):
+    """Times the oracle on whole heads (all layers, every query block) until the
+    budget is spent; returns (seconds, heads done)."""
+    secs, done = 0.0, 0
+    for t in oracle_head_layers(w):
+        secs += t
+        done += 1
+        if done % w.layers == 0 and (secs >= budget_s or done // w.layers >= w.hq):
             break
-    return time.perf_counter() - t0 - gen_time, heads
+    return secs, done // w.layers
 
 
 def blas_threads() -> int:
@@ -228,13 +245,13 @@ def run_reference(args, world, rank):
     if rank != 0:
         return 0
     w = W.PREFILL_16K
+    # one step = one (head, layer) of the pass, heads in turn with their walk
+    # state carried across steps; scaled by the hq x layers head-layers of a pass
+    it = oracle_head_layers(w)
     for _ in range(args.warmup):
-        oracle_prefill_sample(w, 0.0, max_heads=1)
-    times = []
-    for _ in range(args.steps):
-        secs, heads = oracle_prefill_sample(w, 0.0, max_heads=1)
-        times.append(secs * w.hq / heads)
-    step = statistics.mean(times)
+        next(it)
+    times = [next(it) for _ in range(args.steps)]
+    step = statistics.mean(times) * w.hq * w.layers
     value = w.n / step
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -243,8 +260,9 @@ def run_reference(args, world, rank):
         "config": {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
                    "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
-                         "sample": f"each step: the oracle on 1 of {w.hq} query heads x {w.layers} layers, "
-                                   f"scaled by heads to the whole pass"},
+                         "sample": f"each step: the oracle (fp64 numpy) on one head-layer (1 of {w.hq} query heads, "
+                                   f"1 of {w.layers} layers, every query block), scaled by the {w.hq * w.layers} "
+                                   f"head-layers of one pass"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -282,10 +300,7 @@ def bench_prefill(args, world, S, W, torch):
     assert S.sws_sync_check(h) == 0
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(w.layers)]
            for _ in range(args.steps)]
-    dev_props = torch.cuda.get_device_properties(0)
-    bus = f"{getattr(dev_props, 'pci_domain_id', 0):08x}:{getattr(dev_props, 'pci_bus_id', 0):02x}:" \
-          f"{getattr(dev_props, 'pci_device_id', 0):02x}.0"
-    clocks = ClockSampler(bus)
+    clocks = ClockSampler(gpu_bus_id(torch))
     clocks.start()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -407,13 +422,18 @@ def bench_decode(args, world, S, W, torch, peaks):
     for t in range(warm):
         step(t, False)
     torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_bus_id(torch))
+    clocks.start()
     barrier(world)
+    torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for t in range(warm, wd.steps):
         step(t, True)
     b.record(stream)
     torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
     assert S.sws_sync_check(h) == 0
     timed = wd.steps - warm
     step_ms = max_over_ranks(a.elapsed_time(b), world) / timed
@@ -434,7 +454,7 @@ def bench_decode(args, world, S, W, torch, peaks):
     hbm = peaks["hbm_gbs"]
     dense_bytes = units * (wd.n0 + wd.steps) * wd.d * 4
     out = {
-        "workload": wd.name, "step_us": step_ms * 1e3, "steps_timed": timed,
+        "workload": wd.name, "step_us": step_ms * 1e3, "steps_timed": timed, "clocks": clk,
         "hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
         "bytes_per_step": step_bytes, "kv_bytes_per_step": kv_bytes, "dense_kv_bytes_per_step": dense_bytes,
         "union_blocks_per_unit": float(u.mean().item()),
@@ -477,7 +497,14 @@ def main():
     ms_step = pf["ms"] / args.steps
     value = world * w.n / (ms_step * 1e-3)
     attn_tflops = pf["flops"] / (pf["attn_ms"] * 1e-3) / 1e12
-    peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # The burst GEMM peak was measured at full SM clocks, the sustained one under
+    # the power cap at lower clocks: take the one whose clocks the timed region saw.
+    sm, smx = pf["clocks"].get("sm_mhz"), pf["clocks"].get("sm_max_mhz")
+    burst = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    at_full_clock = sm is None or smx is None or sm >= 0.9 * smx
+    peak_t = burst if at_full_clock else sustained
+    peak_name = "bf16 burst" if at_full_clock else "bf16 sustained"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -490,7 +517,8 @@ def main():
         "roofline": {"kernel": "sws_sparse_attn_prefill", "bound": "tensor", "achieved": attn_tflops, "peak": peak_t,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
                      "traffic": profiled_traffic("attn_tc_prefill_n16384_B64", "k_attn_tc.cu"),
-                     "peak_source": f"{peak_kind} bf16 sustained", "flops_per_launch": pf["flops"],
+                     "peak_source": f"{peak_kind} {peak_name}",
+                     "frac_of_burst": attn_tflops / burst, "frac_of_sustained": attn_tflops / sustained, "flops_per_launch": pf["flops"],
                      "ms_per_launch": pf["attn_ms"]},
         "sketch_roofline": {"bound": "hbm", "achieved": pf["sketch_bytes"] / (pf["stage"]["sketch"] / w.layers * 1e-3) / 1e9,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s"},
