@@ -8,9 +8,10 @@
 //   decode_select_kernel (one CTA per (sequence, KV head)):
 //     1. appends the token's K/V to the cache, adds K to the running sum of the
 //        last block and refreshes that block's sketch k~ = mean * H_d;
-//     2. for each query head of the GQA group (one warp each): q~ = q H_d,
-//        z_j = q~ . k~_j / sqrt(k) over the cached blocks, the log-domain walk
-//        rho_j += s * (z_j - logsumexp(z)), and the top-tau blocks of rho;
+//     2. q~ = q H_d for the query heads of the GQA group and z_j = q~ . k~_j /
+//        sqrt(k) over the cached blocks (one thread per block, all heads); then
+//        per head, on 8 / group warps: the log-domain walk rho_j += s * (z_j -
+//        logsumexp(z)) and the top-tau blocks of rho (8-bit radix select);
 //     3. the union of the group's choices, ascending, with a per-block head mask.
 //   decode_attn_kernel (split over the union): each CTA streams a slice of the
 //     union's K/V blocks (cp.async, 3 stages), scores all heads of the group
@@ -67,8 +68,114 @@ __global__ void advance_kernel(int32_t* seq_lens, int32_t batch) {
 
 // -------------------------------------------------------------- select ------
 constexpr int kSelThreads = 256;
-constexpr int kChunk = 64;  // k~ rows staged per pass
+constexpr int kSelWarps = kSelThreads / 32;
 
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Output o of a length-D row times H_d, computed by one warp: lane l sums the
+// terms t = l, l + 32, ..., then a shuffle tree adds the lanes.
+template <int D>
+__device__ __forceinline__ double warp_dot_hdt(const double* row_smem, const double* __restrict__ hdt_row, int lane) {
+  double a = 0.0;
+#pragma unroll
+  for (int t = lane; t < D; t += 32) a = fma(row_smem[t], __ldg(hdt_row + t), a);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+  return a;
+}
+
+// Exact top-tau of keys[0, m) (ties to the lower index) by nthr threads (whole
+// warps, the first of them warp `w0`) that share named barrier `bar_id`:
+// eight passes of an 8-bit radix select on the 64-bit keys (a 256-bin shared
+// histogram of the keys that still match the prefix found so far), then an
+// ordered compaction by the first warp that writes the chosen indices
+// ascending to out[] and ORs `bit` into mark[j].
+__device__ void group_top_tau(const uint64_t* keys, int m, int tau, int* hist, int* ctl, int t, int nthr, int bar_id,
+                              int32_t* out, uint32_t* mark, uint32_t bit, int32_t* err) {
+  uint64_t prefix = 0, pm = 0;
+  int need = tau;
+  bool all_cands = false;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int x = t; x < 256; x += nthr) hist[x] = 0;
+    if (t == 0) ctl[0] = ctl[1] = ctl[2] = 0;
+    named_bar(bar_id, nthr);
+    for (int j = t; j < m; j += nthr) {
+      const uint64_t key = keys[j];
+      if ((key & pm) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    named_bar(bar_id, nthr);
+    if (t < 32) {
+      // lane l owns bins 255 - 8l - u, u = 0..7 (descending key order)
+      int c[8], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        c[u] = hist[255 - 8 * t - u];
+        sum += c[u];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (t >= off) incl += y;
+      }
+      const int excl = incl - sum;
+      if (excl < need && need <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (run + c[u] >= need) {
+            ctl[0] = 255 - 8 * t - u;
+            ctl[1] = need - run;
+            ctl[2] = c[u];
+            break;
+          }
+          run += c[u];
+        }
+      }
+    }
+    named_bar(bar_id, nthr);
+    const int digit = ctl[0];
+    need = ctl[1];
+    const int cnt = ctl[2];
+    prefix |= static_cast<uint64_t>(digit) << shift;
+    pm |= 255ull << shift;
+    named_bar(bar_id, nthr);  // ctl and hist are rewritten by the next pass
+    if (cnt == need) {
+      all_cands = true;
+      break;
+    }
+  }
+  if (t >= 32) return;
+  const unsigned lt = lanemask_lt();
+  int base = 0, ties = 0;
+  for (int j0 = 0; j0 < m; j0 += 32) {
+    const int j = j0 + t;
+    const bool valid = j < m;
+    const uint64_t km = valid ? (keys[j] & pm) : 0;
+    const bool above = valid && km > prefix;
+    const bool cand = valid && km == prefix;
+    const unsigned cb = __ballot_sync(0xffffffffu, cand);
+    bool take = cand;
+    if (!all_cands) {
+      take = cand && (ties + __popc(cb & lt)) < need;
+      ties += __popc(cb);
+    }
+    const bool sel = above || take;
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = base + __popc(sb & lt);
+      if (pos < tau) out[pos] = j;
+      atomicOr(&mark[j], bit);
+    }
+    base += __popc(sb);
+  }
+  if (t == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
+}
+
+// One CTA per (sequence, KV head); the query heads of the group split the
+// warps between them (8 / group warps each) for their walk and selection.
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_tok,
@@ -80,12 +187,15 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     int32_t B, int32_t s_pow, int32_t num, int32_t den, int32_t* err) {
   const int group = hq / hkv;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                 // [group][max_blocks] (z, then keys)
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                       // [group][max_blocks] (z, then keys)
   uint32_t* mark = reinterpret_cast<uint32_t*>(keys + group * max_blocks);  // [max_blocks]
   double* qt = reinterpret_cast<double*>(mark + ((max_blocks + 1) & ~int64_t(1)));  // [group][k]
-  double* ks = qt + group * k;                                        // [kChunk][k + 1]
-  double* mean = ks + kChunk * (k + 1);                               // [D]
-  int* wsum = reinterpret_cast<int*>(mean + D);                       // [kSelThreads / 32 + 1]
+  double* mean = qt + group * k;                                            // [D]
+  double* qrow = mean + D;                                                  // [group][D]
+  double* red = qrow + group * D;                                           // [kSelWarps]
+  int* hist = reinterpret_cast<int*>(red + kSelWarps);                      // [group][256]
+  int* ctl = hist + group * 256;                                            // [group][4]
+  int* wsum = ctl + group * 4;                                              // [kSelWarps + 1]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t unit = blockIdx.x;
@@ -98,10 +208,11 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
   const int64_t pos = len - 1;
   const int64_t blk = pos / B;
   const int cnt = static_cast<int>(pos % B) + 1;
-  const int64_t nb = blk + 1;
-  for (int64_t j = tid; j < nb; j += kSelThreads) mark[j] = 0u;
+  const int nb = static_cast<int>(blk + 1);
+  for (int j = tid; j < nb; j += kSelThreads) mark[j] = 0u;
 
-  // 1. append the token and refresh the last block's sketch
+  // 1. append the token, update the last block's running key sum; stage the
+  //    block mean and the group's query rows
   if (tid < D) {
     const __nv_bfloat16 kt = k_tok[unit * D + tid];
     k_cache[(unit * max_len + pos) * D + tid] = kt;
@@ -111,70 +222,85 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     k_psum[unit * D + tid] = ps;
     mean[tid] = ps / cnt;
   }
+  for (int x = tid; x < group * D; x += kSelThreads)
+    qrow[x] = static_cast<double>(__bfloat162float(q_tok[((int64_t)bi * hq + (int64_t)g * group) * D + x]));
   __syncthreads();
+  // the last block's sketch k~ = mean H_d and q~ = q H_d, one warp per output
   double* ksk = k_sketch + unit * max_blocks * k;
-  for (int c = tid; c < k; c += kSelThreads) {
-    double acc = 0.0;
-    for (int t = 0; t < D; ++t) acc += mean[t] * hdt[(size_t)c * D + t];
-    ksk[blk * k + c] = acc;
-  }
-  // q~ = q H_d for every head of the group
-  for (int x = tid; x < group * k; x += kSelThreads) {
-    const int r = x / k, c = x % k;
-    const __nv_bfloat16* qr = q_tok + ((int64_t)bi * hq + g * group + r) * D;
-    double acc = 0.0;
-    for (int t = 0; t < D; ++t) acc += static_cast<double>(__bfloat162float(qr[t])) * hdt[(size_t)c * D + t];
-    qt[r * k + c] = acc;
+  for (int o = warp; o < (group + 1) * k; o += kSelWarps) {
+    const int r = o / k, c = o % k;  // r == group: the key block
+    const double v = warp_dot_hdt<D>(r == group ? mean : qrow + r * D, hdt + (size_t)c * D, lane);
+    if (lane == 0) {
+      if (r == group) ksk[blk * k + c] = v;
+      else qt[r * k + c] = v;
+    }
   }
   __syncthreads();
 
-  // 2a. z_j for every head, k~ staged through shared memory
+  // 2. z_j = q~ . k~_j / sqrt(k) for every head, one thread per key block
   double* z = reinterpret_cast<double*>(keys);
   const double inv_sqrt_k = 1.0 / sqrt((double)k);
-  for (int64_t j0 = 0; j0 < nb; j0 += kChunk) {
-    const int rows = static_cast<int>(std::min<int64_t>(kChunk, nb - j0));
-    for (int x = tid; x < rows * k; x += kSelThreads) ks[(x / k) * (k + 1) + x % k] = ksk[j0 * k + x];
-    __syncthreads();
-    for (int x = tid; x < group * rows; x += kSelThreads) {
-      const int r = x / rows, jj = x % rows;
-      double acc = 0.0;
-      for (int c = 0; c < k; ++c) acc += qt[r * k + c] * ks[jj * (k + 1) + c];
-      z[r * max_blocks + j0 + jj] = acc * inv_sqrt_k;
+  for (int j = tid; j < nb; j += kSelThreads) {
+    const double* kr = ksk + (int64_t)j * k;
+    double acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
+    for (int c = 0; c < k; ++c) {
+      const double kv = kr[c];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < group) acc[r] = fma(qt[r * k + c], kv, acc[r]);
     }
-    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < group) z[r * max_blocks + j] = acc[r] * inv_sqrt_k;
   }
+  __syncthreads();
 
-  // 2b. log-domain walk and top-tau, one warp per head
+  // 3. per head: log-domain walk, then top-tau (its share of the warps)
   const int tau = tau_of_row(nb - 1, num, den);
-  for (int r = warp; r < group; r += kSelThreads / 32) {
+  const int wph = kSelWarps / group;  // >= 1 since group <= 8
+  const int r = warp / wph;
+  if (r < group) {
+    const int t = tid - r * wph * 32, nthr = wph * 32, bar_id = 1 + r;
     const int h = g * group + r;
     double* zr = z + r * max_blocks;
     double mx = -INFINITY;
-    for (int64_t j = lane; j < nb; j += 32) mx = fmax(mx, zr[j]);
+    for (int j = t; j < nb; j += nthr) mx = fmax(mx, zr[j]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
+    named_bar(bar_id, nthr);
+    mx = red[r * wph];
+    for (int w = 1; w < wph; ++w) mx = fmax(mx, red[r * wph + w]);
+    named_bar(bar_id, nthr);
     double se = 0.0;
-    for (int64_t j = lane; j < nb; j += 32) se += exp(zr[j] - mx);
+    for (int j = t; j < nb; j += nthr) se += exp(zr[j] - mx);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
+    if (lane == 0) red[warp] = se;
+    named_bar(bar_id, nthr);
+    se = 0.0;
+    for (int w = 0; w < wph; ++w) se += red[r * wph + w];
     const double lse = mx + log(se);
     double* rho = walk_state + ((int64_t)bi * hq + h) * max_blocks;
     uint64_t* kr = keys + r * max_blocks;
-    for (int64_t j = lane; j < nb; j += 32) {
+    for (int j = t; j < nb; j += nthr) {
       const double val = (first_layer ? 0.0 : rho[j]) + s_pow * (zr[j] - lse);
       rho[j] = val;
       kr[j] = order_key(val);
     }
-    __syncwarp();
-    warp_top_tau(kr, static_cast<int>(nb), tau, head_sel + ((int64_t)bi * hq + h) * max_blocks, err, mark, 1u << r);
-    if (lane == 0) head_cnt[(int64_t)bi * hq + h] = tau;
+    named_bar(bar_id, nthr);
+    group_top_tau(kr, nb, tau, hist + r * 256, ctl + r * 4, t, nthr, bar_id,
+                  head_sel + ((int64_t)bi * hq + h) * max_blocks, mark, 1u << r, err);
+    if (t == 0) head_cnt[(int64_t)bi * hq + h] = tau;
   }
   __syncthreads();
 
-  // 3. ordered compaction of the union
+  // 4. ordered compaction of the union
   int base = 0;
-  for (int64_t j0 = 0; j0 < nb; j0 += kSelThreads) {
-    const int64_t j = j0 + tid;
+  for (int j0 = 0; j0 < nb; j0 += kSelThreads) {
+    const int j = j0 + tid;
     const uint32_t mk = (j < nb) ? mark[j] : 0u;
     const unsigned bal = __ballot_sync(0xffffffffu, mk != 0u);
     if (lane == 0) wsum[warp] = __popc(bal);
@@ -182,7 +308,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     int off = base;
     for (int w = 0; w < warp; ++w) off += wsum[w];
     int tot = 0;
-    for (int w = 0; w < kSelThreads / 32; ++w) tot += wsum[w];
+    for (int w = 0; w < kSelWarps; ++w) tot += wsum[w];
     if (mk != 0u) {
       const int p = off + __popc(bal & lanemask_lt());
       sel[unit * max_blocks + p] = static_cast<int32_t>(j);
@@ -482,7 +608,8 @@ cudaError_t launch_attn2(int32_t group, const __nv_bfloat16* q, const __nv_bfloa
 size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group) {
   const int64_t k = cfg.sketch_dim, D = cfg.head_dim;
   return (size_t)group * max_blocks * 8 + (size_t)((max_blocks + 1) & ~int64_t(1)) * 4 + (size_t)group * k * 8 +
-         (size_t)kChunk * (k + 1) * 8 + (size_t)D * 8 + (kSelThreads / 32 + 1) * 4;
+         (size_t)D * 8 + (size_t)group * D * 8 + kSelWarps * 8 + (size_t)group * 256 * 4 + (size_t)group * 4 * 4 +
+         (kSelWarps + 1) * 4;
 }
 
 int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group) {

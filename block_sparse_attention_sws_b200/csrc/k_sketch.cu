@@ -4,15 +4,11 @@
 // (feature-space sketch: projection by H_d and the sketched block scores
 // Q~ K~^T / sqrt(k) under the causal block mask).
 //
-// 1. pool_mean_kernel: one streaming pass over Q and K (one launch for both).
-//    One CTA per SM; each warp walks its own (head, block) items; each item is
-//    one contiguous B x d tile fetched by a 1-D bulk copy into the warp's ring
-//    of shared-memory stages (mbarrier completion), summed per column (fp32
-//    partials over four bf16 rows, fp64 beyond) and scaled by 1 / (rows of the
-//    block). HBM-bound: Q and K are read exactly once; the fp64 means go to
-//    the workspace.
-// 2. project_kernel: q~ = q_bar H_d and k~ = k_bar H_d (b x d x k MACs).
-// 3. scores_kernel: S = Q~ K~^T / sqrt(k) on and below the block diagonal.
+// 1. pool_project_kernel: one streaming pass over Q and K (one launch for
+//    both): 16-byte loads of each contiguous B x d block, per-column sums,
+//    the means, and their projection q~ = q_bar H_d, k~ = k_bar H_d. HBM-bound:
+//    Q and K are read exactly once and only the b x k sketches are written.
+// 2. scores_kernel: S = Q~ K~^T / sqrt(k) on and below the block diagonal.
 #include <algorithm>
 
 #include "sws_common.cuh"
@@ -20,105 +16,83 @@
 namespace sws {
 namespace {
 
-// Block means of Q (heads [0, hq)) and K (heads [hq, hq + hkv)):
-// means[(head * nblk + blk) * D + c]. Every warp streams its own items through
-// a private ring of bulk-copy stages: lane l reads 16-byte vectors l, l + 32,
-// ... of the tile, so it always holds the same 16 bytes of columns over a
-// strided set of rows; one shuffle level per factor of two finishes the column
-// sums, and no CTA-wide barrier is needed.
+// 16 bytes from global memory that this kernel reads exactly once: bypass L1.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+constexpr int kPoolWarps = 8;   // warps per CTA
+constexpr int kPoolBatch = 8;   // 16-byte loads in flight per lane
+
+// Block means of Q (heads [0, hq)) and K (heads [hq, hq + hkv)) and their
+// projection by H_d, in one pass over Q and K. One warp per (head, block)
+// item, items dealt round-robin over all warps of the grid; a block is one
+// contiguous rows x D tile, so lane l always reads the same 16 bytes of
+// columns (vector l mod VR of a row) on rows l / VR, l / VR + 32 / VR, ...,
+// kPoolBatch of them in flight at a time. bf16 columns are summed in fp32 over
+// one batch of rows, then in fp64; fp32 inputs are summed in fp64 throughout.
+// The column sums meet in a shuffle tree, the means (sum / rows, as the
+// definition divides) go to a per-warp shared row, and lane j forms output
+// column j of q~ = q_bar H_d (k~ for K heads) from it and column j of H_d.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) pool_mean_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n,
-                                                        int32_t hq, int32_t hkv, int32_t B, int64_t nblk,
-                                                        double inv_B, double* __restrict__ means, int stages,
-                                                        uint32_t stage_bytes, int32_t* err) {
+__global__ void __launch_bounds__(kPoolWarps * 32, 3)
+    pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
+                        int32_t B, int64_t nblk, const double* __restrict__ hd, int32_t ksk,
+                        double* __restrict__ q_sk, double* __restrict__ k_sk) {
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte vector
   constexpr int VR = D / VE;          // vectors per row
   static_assert(VR <= 32 && 32 % VR == 0, "row must map onto a whole number of lanes");
-  constexpr int LPC = 32 / VR;        // lanes sharing a column group
+  constexpr int LPC = 32 / VR;        // rows covered by one warp-wide load
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ double mean_row[kPoolWarps][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  uint8_t* tiles = smem + (size_t)warp * stages * stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)nwarps * stages * stage_bytes) + warp * 8;
-
+  const int vc = lane % VR, rl = lane / VR;
   const int64_t total = (int64_t)(hq + hkv) * nblk;
-  const int64_t gw = (int64_t)blockIdx.x * nwarps + warp;  // global warp index
-  const int64_t nw = (int64_t)gridDim.x * nwarps;
-  const int64_t my_count = gw < total ? (total - gw + nw - 1) / nw : 0;
-
-  auto item_src = [&](int64_t it, uint32_t& bytes) -> const T* {
+  const int64_t nw = (int64_t)gridDim.x * kPoolWarps;
+  for (int64_t it = (int64_t)blockIdx.x * kPoolWarps + warp; it < total; it += nw) {
     const int64_t head = it / nblk, blk = it % nblk;
     const int64_t r0 = blk * B;
-    const int64_t rows = (n - r0 < B ? n - r0 : (int64_t)B);
-    bytes = static_cast<uint32_t>(rows * D * sizeof(T));
-    return head < hq ? q + (head * n + r0) * D : k + ((head - hq) * n + r0) * D;
-  };
-
-  if (lane == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
-    mbar_fence_init();
-    for (int s = 0; s < stages && s < my_count; ++s) {
-      uint32_t bytes;
-      const T* src = item_src(gw + (int64_t)s * nw, bytes);
-      mbar_arrive_expect_tx(&full[s], bytes);
-      bulk_g2s(tiles + (size_t)s * stage_bytes, src, bytes, &full[s]);
-    }
-  }
-  __syncwarp();
-
-  const int vc = lane % VR, r_lane = lane / VR;
-  for (int64_t m = 0; m < my_count; ++m) {
-    const int s = static_cast<int>(m % stages);
-    const uint32_t parity = static_cast<uint32_t>((m / stages) & 1);
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], parity, err))) return;
-
-    const int64_t it = gw + m * nw;
-    const int64_t blk = it % nblk;
-    const int rows = static_cast<int>(n - blk * B < B ? n - blk * B : (int64_t)B);
-    const T* tile = reinterpret_cast<const T*>(tiles + (size_t)s * stage_bytes);
+    const int rows = static_cast<int>(n - r0 < B ? n - r0 : (int64_t)B);
+    const T* src = (head < hq ? q + (head * n + r0) * D : k + ((head - hq) * n + r0) * D) + vc * VE;
 
     double acc[VE];
 #pragma unroll
     for (int e = 0; e < VE; ++e) acc[e] = 0.0;
-    if constexpr (sizeof(T) == 2) {
-      // bf16: fp32 partial over groups of four rows, then fp64
-      for (int r0 = r_lane; r0 < rows; r0 += 4 * LPC) {
+    for (int rb = rl; rb < rows; rb += kPoolBatch * LPC) {
+      uint4 v[kPoolBatch];
+#pragma unroll
+      for (int u = 0; u < kPoolBatch; ++u) {
+        const int r = rb + u * LPC;
+        v[u] = r < rows ? ld_stream16(src + (size_t)r * D) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if constexpr (sizeof(T) == 2) {
         float part[VE];
 #pragma unroll
         for (int e = 0; e < VE; ++e) part[e] = 0.f;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int r = r0 + qq * LPC;
-          if (r < rows) {
-            const uint4 v = *reinterpret_cast<const uint4*>(tile + (size_t)r * D + vc * VE);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int u = 0; u < kPoolBatch; ++u) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              part[2 * e] += __uint_as_float(w[e] << 16);
-              part[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
-            }
+          for (int e = 0; e < 4; ++e) {
+            part[2 * e] += __uint_as_float(w[e] << 16);
+            part[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
           }
         }
 #pragma unroll
         for (int e = 0; e < VE; ++e) acc[e] += static_cast<double>(part[e]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < kPoolBatch; ++u) {
+          acc[0] += static_cast<double>(__uint_as_float(v[u].x));
+          acc[1] += static_cast<double>(__uint_as_float(v[u].y));
+          acc[2] += static_cast<double>(__uint_as_float(v[u].z));
+          acc[3] += static_cast<double>(__uint_as_float(v[u].w));
+        }
       }
-    } else {
-      for (int r = r_lane; r < rows; r += LPC) {
-        const float4 v = *reinterpret_cast<const float4*>(tile + (size_t)r * D + vc * VE);
-        acc[0] += v.x;
-        acc[1] += v.y;
-        acc[2] += v.z;
-        acc[3] += v.w;
-      }
-    }
-    __syncwarp();  // every lane is done with the stage
-    if (lane == 0 && m + stages < my_count) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      uint32_t bytes;
-      const T* src = item_src(gw + (m + stages) * nw, bytes);
-      mbar_arrive_expect_tx(&full[s], bytes);
-      bulk_g2s(tiles + (size_t)s * stage_bytes, src, bytes, &full[s]);
     }
 #pragma unroll
     for (int off = VR; off < 32; off <<= 1) {
@@ -126,41 +100,23 @@ __global__ void __launch_bounds__(128) pool_mean_kernel(const T* __restrict__ q,
       for (int e = 0; e < VE; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
     }
     if (lane < VR) {
-      const double sc = rows == B ? inv_B : 1.0 / rows;
-      double* dst = means + it * D + vc * VE;
+      const double cnt = static_cast<double>(rows);
 #pragma unroll
-      for (int e = 0; e < VE; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(acc[e] * sc, acc[e + 1] * sc);
+      for (int e = 0; e < VE; e += 2)
+        *reinterpret_cast<double2*>(&mean_row[warp][vc * VE + e]) = make_double2(acc[e] / cnt, acc[e + 1] / cnt);
     }
-  }
-}
-
-// q~ (rows < q_rows) and k~ from the block means: one warp per (head, block).
-// The row of means is held four values per lane and broadcast by shuffles;
-// four independent accumulators per output column.
-__global__ void __launch_bounds__(256) project_kernel(const double* __restrict__ means, int64_t rows, int64_t q_rows,
-                                                      const double* __restrict__ hd, int D, int k,
-                                                      double* __restrict__ q_sk, double* __restrict__ k_sk) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const double* mr = means + row * D;
-  double mv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) mv[i] = (lane + 32 * i < D) ? mr[lane + 32 * i] : 0.0;
-  double* out = row < q_rows ? q_sk + row * k : k_sk + (row - q_rows) * k;
-  for (int c0 = 0; c0 < k; c0 += 32) {
-    const int c = c0 + lane;
-    double a[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (32 * g >= D) break;
+    __syncwarp();
+    double* out = head < hq ? q_sk + it * ksk : k_sk + (it - (int64_t)hq * nblk) * ksk;
+    for (int j = lane; j < ksk; j += 32) {
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 8
-      for (int j = 0; j < 32; ++j) {
-        const double m = __shfl_sync(0xffffffffu, mv[g], j);
-        if (c < k) a[j & 3] = fma(m, hd[(size_t)(32 * g + j) * k + c], a[j & 3]);
+      for (int c = 0; c < D; c += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = fma(mean_row[warp][c + u], __ldg(hd + (size_t)(c + u) * ksk + j), a[u]);
       }
+      out[j] = (a[0] + a[1]) + (a[2] + a[3]);
     }
-    if (c < k) out[c] = (a[0] + a[1]) + (a[2] + a[3]);
+    __syncwarp();  // the row is rewritten by the next item
   }
 }
 
@@ -221,54 +177,35 @@ __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ 
 }
 
 template <typename T, int D>
-cudaError_t launch_pool(const sws_handle* h, const T* q, const T* k, int64_t n, int32_t hq, int32_t hkv,
-                        double* means, cudaStream_t st) {
+cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int64_t n, int32_t hq, int32_t hkv,
+                                double* q_sk, double* k_sk, cudaStream_t st) {
   const int32_t B = h->cfg.block_size;
   const int64_t nblk = ceil_div64(n, B);
-  const uint32_t stage_bytes = static_cast<uint32_t>(B) * D * sizeof(T);
-  // about 192 KB of copies in flight per SM: warps x stages x tile
-  const int stages = stage_bytes <= (16u << 10) ? 3 : 2;
-  const int warps = std::max(1, std::min(4, static_cast<int>((192u << 10) / (stages * stage_bytes))));
-  const size_t smem = (size_t)warps * stages * stage_bytes + (size_t)warps * 8 * sizeof(uint64_t);
-  auto kern = pool_mean_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const int64_t total = (int64_t)(hq + hkv) * nblk;
-  const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, warps), (int64_t)h->num_sms));
-  kern<<<grid, warps * 32, smem, st>>>(q, k, n, hq, hkv, B, nblk, 1.0 / B, means, stages, stage_bytes, h->err);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 3 * (int64_t)h->num_sms));
+  pool_project_kernel<T, D><<<grid, kPoolWarps * 32, 0, st>>>(q, k, n, hq, hkv, B, nblk, h->hd, h->cfg.sketch_dim,
+                                                              q_sk, k_sk);
   note_launches(1);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t sketch_workspace_bytes(const sws_config& c, int64_t n, int32_t hq, int32_t hkv) {
-  return (size_t)(hq + hkv) * ceil_div64(n, c.block_size) * c.head_dim * sizeof(double);
-}
+size_t sketch_workspace_bytes(const sws_config&, int64_t, int32_t, int32_t) { return 0; }
 
-cudaError_t launch_sketch_means_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
-                                        int32_t hq, int32_t hkv, double* means, double* q_sk, double* k_sk,
-                                        cudaStream_t st) {
+cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
+                                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, cudaStream_t st) {
   const int d = h->cfg.head_dim;
-  cudaError_t e;
   if (dt == SWS_BF16) {
     const auto* pq = static_cast<const __nv_bfloat16*>(q);
     const auto* pk = static_cast<const __nv_bfloat16*>(k);
-    e = d == 128 ? launch_pool<__nv_bfloat16, 128>(h, pq, pk, n, hq, hkv, means, st)
-                 : launch_pool<__nv_bfloat16, 64>(h, pq, pk, n, hq, hkv, means, st);
-  } else {
-    const auto* pq = static_cast<const float*>(q);
-    const auto* pk = static_cast<const float*>(k);
-    e = d == 128 ? launch_pool<float, 128>(h, pq, pk, n, hq, hkv, means, st)
-                 : launch_pool<float, 64>(h, pq, pk, n, hq, hkv, means, st);
+    return d == 128 ? launch_pool_project<__nv_bfloat16, 128>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st)
+                    : launch_pool_project<__nv_bfloat16, 64>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st);
   }
-  if (e != cudaSuccess) return e;
-  const int64_t b = ceil_div64(n, h->cfg.block_size);
-  const int64_t rows = (int64_t)(hq + hkv) * b;
-  project_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(means, rows, (int64_t)hq * b, h->hd, d,
-                                                                             h->cfg.sketch_dim, q_sk, k_sk);
-  note_launches(1);
-  return cudaGetLastError();
+  const auto* pq = static_cast<const float*>(q);
+  const auto* pk = static_cast<const float*>(k);
+  return d == 128 ? launch_pool_project<float, 128>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st)
+                  : launch_pool_project<float, 64>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st);
 }
 
 cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,

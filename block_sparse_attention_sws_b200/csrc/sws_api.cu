@@ -232,8 +232,7 @@ sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dty
   if (ws_bytes < sketch_workspace_bytes(h->cfg, n, hq, hkv)) return SWS_ERR_WORKSPACE;
   auto st = static_cast<cudaStream_t>(stream);
   sws_status s = cuda_status(
-      launch_sketch_means_project(h, q, k, dtype, n, hq, hkv, static_cast<double*>(ws), q_sk, k_sk, st),
-      "sketch means");
+      launch_sketch_pool_project(h, q, k, dtype, n, hq, hkv, q_sk, k_sk, st), "sketch pool+project");
   if (s != SWS_OK) return s;
   return cuda_status(launch_sketch_scores(h, q_sk, k_sk, b, hq, hkv, scores, st), "sketch scores");
 }

@@ -140,9 +140,8 @@ __host__ __device__ __forceinline__ int32_t tau_of_row(int64_t i, int32_t num, i
 void note_launches(int count);
 
 size_t sketch_workspace_bytes(const sws_config& c, int64_t n, int32_t hq, int32_t hkv);
-cudaError_t launch_sketch_means_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
-                                        int32_t hq, int32_t hkv, double* means, double* q_sk, double* k_sk,
-                                        cudaStream_t st);
+cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
+                                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, cudaStream_t st);
 cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,
                                  int32_t hkv, double* scores, cudaStream_t st);
 

@@ -124,8 +124,9 @@ sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code);
  *   q_sk   (device) [hq, b, k]   double, written
  *   k_sk   (device) [hkv, b, k]  double, written
  *   scores (device) [hq, b, b]   double; entries j <= i written, j > i left untouched
- *   ws     (device) sws_workspace_size(SWS_OP_SKETCH) bytes: the fp64 block means
- * Reads Q and K once. */
+ *   ws     (device) sws_workspace_size(SWS_OP_SKETCH) bytes, currently 0: the block
+ *          means stay on chip (may be NULL while the size is 0)
+ * Reads Q and K once: one fused pass forms the block means and projects them. */
 sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n,
                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, double* scores, void* ws,
                       size_t ws_bytes, void* stream);
