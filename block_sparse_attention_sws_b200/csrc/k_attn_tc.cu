@@ -123,6 +123,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
+// Two fp32 lanes in one 64-bit register for the packed fp32x2 instructions.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 "version 1").
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -515,15 +540,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
               s[kb * BLK + c] = (mode[kb] == 2 && c <= qoff) ? s[kb * BLK + c] : -INFINITY;
           }
         }
-        float mx8[8];
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = s[u];
+        for (int c = 0; c < kTileN; c += 8)
 #pragma unroll
-        for (int c = 8; c < kTileN; c += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], s[c + u]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int u = 0; u < 4; ++u) mx4[u] = max3f(mx4[u], s[c + 2 * u], s[c + 2 * u + 1]);
+        const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
         const float m_new = mx * qscale;
         const bool need = mx != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2);
         const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;  // 0 when m_used = -inf
@@ -535,39 +557,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         // Masked scores are -inf and give exactly 0. The branch is warp-uniform
         // (tcgen05.st is warp-collective): the straight-line path when every row
         // of the warp has a finite reference, a per-row select otherwise.
-        float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const bool live = m_used != -INFINITY;
-        const float nm = live ? -m_used : 0.f;
-        if (__all_sync(0xffffffffu, live)) {
+        const float nm = m_used != -INFINITY ? -m_used : 0.f;
+        const uint64_t sc2 = f2(qscale, qscale), nm2 = f2(nm, nm);
+        uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int qt = 0; qt < 4; ++qt) {
-            uint32_t pk[16];
+        for (int qt = 0; qt < 4; ++qt) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = qt * 32 + 2 * i;
-              const float p0 = fast_exp2(fmaf(s[c], qscale, nm));
-              const float p1 = fast_exp2(fmaf(s[c + 1], qscale, nm));
-              ps8[i & 7] += p0 + p1;
-              pk[i] = pack_p(p0, p1);
-            }
-            tmem_st16u(ts + qt * 16, pk);
+          for (int i = 0; i < 16; ++i) {
+            const int c = qt * 32 + 2 * i;
+            float x0, x1;
+            f2_split(f2_fma(f2(s[c], s[c + 1]), sc2, nm2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            acc2[i & 3] = f2_add(acc2[i & 3], f2(p0, p1));
+            pk[i] = pack_p(p0, p1);
           }
-        } else {
-#pragma unroll
-          for (int qt = 0; qt < 4; ++qt) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = qt * 32 + 2 * i;
-              const float p0 = live ? fast_exp2(fmaf(s[c], qscale, nm)) : 0.f;
-              const float p1 = live ? fast_exp2(fmaf(s[c + 1], qscale, nm)) : 0.f;
-              ps8[i & 7] += p0 + p1;
-              pk[i] = pack_p(p0, p1);
-            }
-            tmem_st16u(ts + qt * 16, pk);
-          }
+          tmem_st16u(ts + qt * 16, pk);
         }
-        l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        {
+          float a0, a1, b0, b1;
+          f2_split(f2_add(acc2[0], acc2[1]), a0, a1);
+          f2_split(f2_add(acc2[2], acc2[3]), b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
         if (!first_tile && __any_sync(0xffffffffu, need)) {
           // O_w holds earlier tiles at the old reference: wait for them, then the
           // whole warp rescales its rows (alpha = 1 for rows that keep theirs)
