@@ -10,18 +10,25 @@
 // of 128; adjacent query blocks select almost the same key blocks), each key
 // tile carrying a selection bit per (key block, query block) pair.
 //
-// Warp roles (320 threads):
-//   warp 0    TMA producer: both Q tiles once per item, then K and V tiles into
-//             a 2-stage ring (3-D tensor maps, 128-byte swizzle, zero fill past n);
-//   warp 1    owns the 512 TMEM columns and issues tcgen05.mma from one thread,
-//             alternating between the two query tiles w: S_w = Q_w K^T into TMEM,
-//             then O_w += P_w V with P_w read from TMEM (it overwrites S_w);
+// Warp roles (352 threads):
+//   warp 0    TMA producer: both Q tiles once per item, then K tiles into a
+//             3-stage ring and V tiles into a 2-stage ring (3-D tensor maps,
+//             128-byte swizzle, zero fill past n); the score products run ahead
+//             of the PV products, so K is needed before V;
+//   warp 1    owns the 512 TMEM columns and issues the score products
+//             S_w = Q_w K^T of the two query tiles w, S_0(g), S_1(g), S_0(g+1),
+//             ..., into the one score buffer the tiles share; each waits until
+//             the softmax group of the previous product has copied the buffer
+//             to registers;
+//   warp 10   issues O_w += P_w V with P_w read from the tile's own TMEM
+//             columns, once the softmax group has written it. With two issuing
+//             threads the tensor cores are fed while either one waits, and no
+//             product ever waits for another product to finish;
 //   warps 2-5 and 6-9: one softmax warpgroup per query tile, one query row per
-//             thread (TMEM lane = row). While one group works on its S, the
-//             tensor cores run the other group's products. A row keeps a running
-//             max that only moves when it grows by more than 2^8 (then its row of
-//             O in TMEM is rescaled); P = 2^(s - m) is written back to TMEM as
-//             bf16; the group finally writes O / l.
+//             thread (TMEM lane = row). A row keeps a running max that only
+//             moves when it grows by more than 2^8 (then its row of O in TMEM is
+//             rescaled); P = 2^(s - m) goes to the group's P columns as bf16 once
+//             its previous PV has read them; the group finally writes O / l.
 // Every wait is bounded; a timeout records a guard code and all roles leave.
 #include <cuda.h>
 
@@ -32,10 +39,12 @@
 namespace sws {
 namespace {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 352;  // 11 warps
 constexpr int kTileM = 128;   // query rows per tile (two tiles per item)
 constexpr int kTileN = 128;   // keys per S tile
 constexpr int kGroup = 128;   // threads per softmax warpgroup
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kPvWarp = 10;   // issues the PV products
 // arrivals per softmax-group barrier phase: one per warp, after __syncwarp
 constexpr int kArrivals = kGroup / 32;
 
@@ -148,6 +157,16 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// 32 columns of this thread's lane into r[]; the registers become valid only
+// after tmem_wait_ld4 below, which names them as operands so that no use can
+// move above it.
+__device__ __forceinline__ void tmem_ld32_nw(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];" : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]) : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld4(uint32_t (&a)[32], uint32_t (&b)[32], uint32_t (&c)[32], uint32_t (&d)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(a[0]), "+r"(b[0]), "+r"(c[0]), "+r"(d[0]), "+r"(a[1]), "+r"(b[1]), "+r"(c[1]), "+r"(d[1]), "+r"(a[2]), "+r"(b[2]), "+r"(c[2]), "+r"(d[2]), "+r"(a[3]), "+r"(b[3]), "+r"(c[3]), "+r"(d[3]), "+r"(a[4]), "+r"(b[4]), "+r"(c[4]), "+r"(d[4]), "+r"(a[5]), "+r"(b[5]), "+r"(c[5]), "+r"(d[5]), "+r"(a[6]), "+r"(b[6]), "+r"(c[6]), "+r"(d[6]), "+r"(a[7]), "+r"(b[7]), "+r"(c[7]), "+r"(d[7]), "+r"(a[8]), "+r"(b[8]), "+r"(c[8]), "+r"(d[8]), "+r"(a[9]), "+r"(b[9]), "+r"(c[9]), "+r"(d[9]), "+r"(a[10]), "+r"(b[10]), "+r"(c[10]), "+r"(d[10]), "+r"(a[11]), "+r"(b[11]), "+r"(c[11]), "+r"(d[11]), "+r"(a[12]), "+r"(b[12]), "+r"(c[12]), "+r"(d[12]), "+r"(a[13]), "+r"(b[13]), "+r"(c[13]), "+r"(d[13]), "+r"(a[14]), "+r"(b[14]), "+r"(c[14]), "+r"(d[14]), "+r"(a[15]), "+r"(b[15]), "+r"(c[15]), "+r"(d[15]), "+r"(a[16]), "+r"(b[16]), "+r"(c[16]), "+r"(d[16]), "+r"(a[17]), "+r"(b[17]), "+r"(c[17]), "+r"(d[17]), "+r"(a[18]), "+r"(b[18]), "+r"(c[18]), "+r"(d[18]), "+r"(a[19]), "+r"(b[19]), "+r"(c[19]), "+r"(d[19]), "+r"(a[20]), "+r"(b[20]), "+r"(c[20]), "+r"(d[20]), "+r"(a[21]), "+r"(b[21]), "+r"(c[21]), "+r"(d[21]), "+r"(a[22]), "+r"(b[22]), "+r"(c[22]), "+r"(d[22]), "+r"(a[23]), "+r"(b[23]), "+r"(c[23]), "+r"(d[23]), "+r"(a[24]), "+r"(b[24]), "+r"(c[24]), "+r"(d[24]), "+r"(a[25]), "+r"(b[25]), "+r"(c[25]), "+r"(d[25]), "+r"(a[26]), "+r"(b[26]), "+r"(c[26]), "+r"(d[26]), "+r"(a[27]), "+r"(b[27]), "+r"(c[27]), "+r"(d[27]), "+r"(a[28]), "+r"(b[28]), "+r"(c[28]), "+r"(d[28]), "+r"(a[29]), "+r"(b[29]), "+r"(c[29]), "+r"(d[29]), "+r"(a[30]), "+r"(b[30]), "+r"(c[30]), "+r"(d[30]), "+r"(a[31]), "+r"(b[31]), "+r"(c[31]), "+r"(d[31]) :: "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 "version 1").
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -195,9 +214,9 @@ struct TileMeta {
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_empty[2];  // per query tile
-  TileMeta meta[2];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], o_empty[2];  // per query tile
+  TileMeta meta[kKStages];  // per K stage
   uint32_t tmem_base;
   volatile int32_t abort;
 };
@@ -208,13 +227,15 @@ struct Smem {
   static constexpr uint32_t kK = kTileN * D * 2;
   static constexpr uint32_t q = 0;                // two query tiles
   static constexpr uint32_t k0 = q + 2 * kQ;
-  static constexpr uint32_t v0 = k0 + 2 * kK;
-  static constexpr uint32_t bars = v0 + 2 * kK;
+  static constexpr uint32_t v0 = k0 + kKStages * kK;
+  static constexpr uint32_t bars = v0 + kVStages * kK;
   static constexpr uint32_t total = bars + sizeof(Bars);
 };
 
-// TMEM columns: S_w at 128 w (P_w packed over its first 64 columns), O_w at 256 + 128 w.
-__host__ __device__ constexpr uint32_t tcol_s(int w) { return 128u * w; }
+// TMEM columns: the shared score buffer at 0, P_w (bf16 pairs) at 128 + 64 w,
+// O_w at 256 + 128 w.
+constexpr uint32_t kColS = 0;
+__host__ __device__ constexpr uint32_t tcol_p(int w) { return 128u + 64u * w; }
 __host__ __device__ constexpr uint32_t tcol_o(int w) { return 256u + 128u * w; }
 
 // Bounded wait (wall time) that also gives up as soon as another role has aborted.
@@ -339,10 +360,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
   if (threadIdx.x == 0) {
     mbar_init(&bs->q_full, 1);
     mbar_init(&bs->q_empty, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bs->k_full[s], 1);
+      mbar_init(&bs->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bs->v_full[s], 1);
+      mbar_init(&bs->v_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bs->kv_full[s], 1);
-      mbar_init(&bs->kv_empty[s], 1);
       mbar_init(&bs->s_full[s], 1);
+      mbar_init(&bs->s_free[s], kArrivals);
       mbar_init(&bs->p_full[s], kArrivals);
       mbar_init(&bs->pv_done[s], 1);
       mbar_init(&bs->o_empty[s], kArrivals);
@@ -393,22 +421,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         while (!done) {
           const bool more = have && wk.next_tile(nxt);
           cur.last = more ? 0 : 1;
-          const int st = kv_it & 1;
-          if (!wait_bar(&bs->kv_empty[st], ((kv_it >> 1) & 1) ^ 1, bs, err)) break;
-          bs->meta[st] = cur;
-          mbar_arrive_expect_tx(&bs->kv_full[st], 2 * L::kK);
-          uint8_t* ks = smem + L::k0 + st * L::kK;
-          uint8_t* vs = smem + L::v0 + st * L::kK;
+          const int sk = kv_it % kKStages, sv = kv_it % kVStages;
+          if (!wait_bar(&bs->k_empty[sk], ((kv_it / kKStages) & 1) ^ 1, bs, err)) break;
+          bs->meta[sk] = cur;
+          mbar_arrive_expect_tx(&bs->k_full[sk], L::kK);
+          uint8_t* ks = smem + L::k0 + sk * L::kK;
 #pragma unroll
           for (int a = 0; a < D / 64; ++a) {
             if constexpr (BLK == 128) {
-              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 128, g, &bs->kv_full[st]);
-              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 128, g, &bs->kv_full[st]);
+              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 128, g, &bs->k_full[sk]);
             } else {
-              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 64, g, &bs->kv_full[st]);
-              tma_load_3d(ks + a * (kTileN * 128) + 64 * 128, &tmk, a * 64, cur.u1 * 64, g, &bs->kv_full[st]);
-              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 64, g, &bs->kv_full[st]);
-              tma_load_3d(vs + a * (kTileN * 128) + 64 * 128, &tmv, a * 64, cur.u1 * 64, g, &bs->kv_full[st]);
+              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 64, g, &bs->k_full[sk]);
+              tma_load_3d(ks + a * (kTileN * 128) + 64 * 128, &tmk, a * 64, cur.u1 * 64, g, &bs->k_full[sk]);
+            }
+          }
+          if (!wait_bar(&bs->v_empty[sv], ((kv_it / kVStages) & 1) ^ 1, bs, err)) break;
+          mbar_arrive_expect_tx(&bs->v_full[sv], L::kK);
+          uint8_t* vs = smem + L::v0 + sv * L::kK;
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a) {
+            if constexpr (BLK == 128) {
+              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 128, g, &bs->v_full[sv]);
+            } else {
+              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 64, g, &bs->v_full[sv]);
+              tma_load_3d(vs + a * (kTileN * 128) + 64 * 128, &tmv, a * 64, cur.u1 * 64, g, &bs->v_full[sv]);
             }
           }
           ++kv_it;
@@ -417,87 +453,87 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer --
-    // Issue order per key tile g: S_0(g), PV_1(g-1), S_1(g), PV_0(g). Group 1
-    // gets its scores half a period after group 0, so the two softmax groups
-    // take turns instead of contending for the exponential units. S_w(g)
-    // overwrites the TMEM columns that held P_w(g-1): it waits for PV_w(g-1).
+  } else if (warp == 1 || warp == kPvWarp) {
+    // ------------------------------------------------------------ MMA issuers --
+    // Two threads feed the tensor cores, so that neither stream's waits leave
+    // them idle: warp 1 issues the score products S_0(g), S_1(g), S_0(g+1), ...
+    // into the one score buffer, each once the softmax group of the previous
+    // one has copied the buffer to registers (s_free); warp kPvWarp issues
+    // PV_0(g), PV_1(g), PV_0(g+1), ..., each once its P is in TMEM (p_full) and,
+    // on an item's first tile, once the previous item's epilogue has read O_w
+    // (o_empty). Each thread commits the barriers of its own products.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileN, false);
       constexpr uint32_t idPV = idesc_bf16(D, true);
-      uint32_t kv_it = 0, gt = 0, item_cnt = 0;
+      const bool s_stream = warp == 1;
+      uint32_t g = 0, item_g = 0;
       bool ok = true;
-      // the PV_1 still owed for the previous tile
-      bool owe = false, owe_first = false;
-      int owe_st = 0;
-      uint32_t owe_item = 0;
-      auto issue_s = [&](int w, int st) {
-        const uint32_t sq = smem_u32(smem + L::q + w * L::kQ);
-        const uint32_t sk = smem_u32(smem + L::k0 + st * L::kK);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * (kTileN * 128) + (kk & 3) * 32;
-          tc_mma(tmem + tcol_s(w), sw128_desc(sq + off, 16, 1024), sw128_desc(sk + koff, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bs->s_full[w]);
-      };
-      auto issue_pv = [&](int w, int st, bool first_of_item) {
-        const uint32_t sv = smem_u32(smem + L::v0 + st * L::kK);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
-          tc_mma_ts(tmem + tcol_o(w), tmem + tcol_s(w) + kk * 8, sw128_desc(sv + kk * 16 * 128, kTileN * 128, 1024),
-                    idPV, (first_of_item && kk == 0) ? 0u : 1u);
-        tc_commit(&bs->pv_done[w]);
-      };
-      // PV_1 of the owed tile (tile gt - 1)
-      auto pay = [&]() -> bool {
-        if (!wait_bar(&bs->p_full[1], (gt - 1) & 1, bs, err)) return false;
-        if (owe_first && !wait_bar(&bs->o_empty[1], (owe_item & 1) ^ 1, bs, err)) return false;
-        issue_pv(1, owe_st, owe_first);
-        tc_commit(&bs->kv_empty[owe_st]);
-        owe = false;
-        return true;
-      };
-      for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x, ++item_cnt) {
-        if (!(ok = wait_bar(&bs->q_full, item_cnt & 1, bs, err))) break;
+      for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x, ++item_g) {
+        if (s_stream && !(ok = wait_bar(&bs->q_full, item_g & 1, bs, err))) break;
         bool first = true;
         while (true) {
-          const int st = kv_it & 1;
-          if (!(ok = wait_bar(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
-          const bool last = bs->meta[st].last != 0;
-          if (gt > 0 && !(ok = wait_bar(&bs->pv_done[0], (gt - 1) & 1, bs, err))) break;
-          issue_s(0, st);
-          if (owe && !(ok = pay())) break;
-          if (gt > 0 && !(ok = wait_bar(&bs->pv_done[1], (gt - 1) & 1, bs, err))) break;
-          issue_s(1, st);
-          if (last) tc_commit(&bs->q_empty);
-          if (!(ok = wait_bar(&bs->p_full[0], gt & 1, bs, err))) break;
-          if (first && !(ok = wait_bar(&bs->o_empty[0], (item_cnt & 1) ^ 1, bs, err))) break;
-          issue_pv(0, st, first);
-          owe = true;
-          owe_first = first;
-          owe_st = st;
-          owe_item = item_cnt;
+          const int sk = g % kKStages;
+          if (!(ok = wait_bar(&bs->k_full[sk], (g / kKStages) & 1, bs, err))) break;
+          const bool last = bs->meta[sk].last != 0;
+          if (s_stream) {
+            const uint32_t sq0 = smem_u32(smem + L::q), sq1 = smem_u32(smem + L::q + L::kQ);
+            const uint32_t skk = smem_u32(smem + L::k0 + sk * L::kK);
+            if (g > 0 && !(ok = wait_bar(&bs->s_free[1], (g - 1) & 1, bs, err))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
+              const uint32_t koff = (kk >> 2) * (kTileN * 128) + (kk & 3) * 32;
+              tc_mma(tmem + kColS, sw128_desc(sq0 + off, 16, 1024), sw128_desc(skk + koff, 16, 1024), idS,
+                     kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bs->s_full[0]);
+            if (!(ok = wait_bar(&bs->s_free[0], g & 1, bs, err))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
+              const uint32_t koff = (kk >> 2) * (kTileN * 128) + (kk & 3) * 32;
+              tc_mma(tmem + kColS, sw128_desc(sq1 + off, 16, 1024), sw128_desc(skk + koff, 16, 1024), idS,
+                     kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bs->s_full[1]);
+            if (last) tc_commit(&bs->q_empty);
+          } else {
+            const uint32_t sv = smem_u32(smem + L::v0 + (g % kVStages) * L::kK);
+            if (!(ok = wait_bar(&bs->v_full[g % kVStages], (g / kVStages) & 1, bs, err))) break;
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              if (!(ok = wait_bar(&bs->p_full[w], g & 1, bs, err))) break;
+              if (first && !(ok = wait_bar(&bs->o_empty[w], (item_g & 1) ^ 1, bs, err))) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kTileN / 16; ++kk)
+                tc_mma_ts(tmem + tcol_o(w), tmem + tcol_p(w) + kk * 8,
+                          sw128_desc(sv + kk * 16 * 128, kTileN * 128, 1024), idPV, (first && kk == 0) ? 0u : 1u);
+              tc_commit(&bs->pv_done[w]);
+            }
+            if (!ok) break;
+            // K and V of tile g are free (S_1(g) completed before P_1(g) was
+            // written); a K stage is released only here, after both softmax
+            // groups are done with the tile, because its slot also holds the
+            // tile's metadata
+            tc_commit(&bs->k_empty[sk]);
+            tc_commit(&bs->v_empty[g % kVStages]);
+          }
           first = false;
-          ++kv_it;
-          ++gt;
+          ++g;
           if (last) break;
         }
       }
-      if (ok && owe) pay();
     }
-  } else {
+  } else if (warp >= 2 && warp < 10) {
     // -------------------------------------------------------------- softmax --
     const int w = (warp - 2) >> 2;          // query tile of this warpgroup
     const int q4 = warp & 3;                // TMEM lane quarter of this warp
     const int r = q4 * 32 + lane;           // query row of the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t ts = trow + tcol_s(w), to = trow + tcol_o(w);
+    const uint32_t ts = trow + kColS, tp = trow + tcol_p(w), to = trow + tcol_o(w);
     const int qslot = (w * kTileM + r) / BLK;  // query block slot within the item
     uint32_t kv_it = 0, gt = 0, item_cnt = 0;
     bool ok = true;
@@ -509,19 +545,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
       float m_used = -INFINITY, l = 0.f;
       bool first_tile = true;
       while (true) {
-        const int st = kv_it & 1;
-        if (!(ok = warp_wait(&bs->kv_full[st], (kv_it >> 1) & 1, bs, err))) break;
-        const TileMeta tm = bs->meta[st];
+        const int sk = kv_it % kKStages;
+        if (!(ok = warp_wait(&bs->k_full[sk], (kv_it / kKStages) & 1, bs, err))) break;
+        const TileMeta tm = bs->meta[sk];
         if (!(ok = warp_wait(&bs->s_full[w], gt & 1, bs, err))) break;
         tc_fence_after();
         float s[kTileN];
+        {
+          uint32_t ra[32], rb[32], rc[32], rd[32];
+          tmem_ld32_nw(ts, ra);
+          tmem_ld32_nw(ts + 32, rb);
+          tmem_ld32_nw(ts + 64, rc);
+          tmem_ld32_nw(ts + 96, rd);
+          tmem_wait_ld4(ra, rb, rc, rd);
 #pragma unroll
-        for (int c = 0; c < kTileN / 32; ++c) {
-          float v[32];
-          tmem_ld32(ts + c * 32, v);  // the wait is inside: registers valid on return
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(ra[i]);
+            s[32 + i] = __uint_as_float(rb[i]);
+            s[64 + i] = __uint_as_float(rc[i]);
+            s[96 + i] = __uint_as_float(rd[i]);
+          }
         }
+        // the scores are in registers: the score buffer may take the next product
+        tc_fence_before();
+        group_arrive(&bs->s_free[w]);
         // masks per key block slot: 0 = none, 1 = all, 2 = causal (key offset <= query offset)
         constexpr int KBS = kTileN / BLK;
         int mode[KBS];
@@ -553,26 +600,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
           l *= alpha;
           m_used = m_new;
         }
-        // P = 2^(s * qscale - m_used), bf16, over the first 64 columns of S_w.
-        // Masked scores are -inf and give exactly 0. The branch is warp-uniform
-        // (tcgen05.st is warp-collective): the straight-line path when every row
-        // of the warp has a finite reference, a per-row select otherwise.
+        // P = 2^(s * qscale - m_used) as packed bf16 pairs, kept in registers
+        // until this group's previous PV has read its P columns. Masked scores
+        // are -inf and give exactly 0; a row whose reference is still -inf has
+        // seen only masked scores, so nm = 0 gives 0 there too. Scale, shift and
+        // row sum run on the packed fp32x2 pipe.
         const float nm = m_used != -INFINITY ? -m_used : 0.f;
         const uint64_t sc2 = f2(qscale, qscale), nm2 = f2(nm, nm);
         uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[kTileN / 2];
 #pragma unroll
-        for (int qt = 0; qt < 4; ++qt) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = qt * 32 + 2 * i;
-            float x0, x1;
-            f2_split(f2_fma(f2(s[c], s[c + 1]), sc2, nm2), x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            acc2[i & 3] = f2_add(acc2[i & 3], f2(p0, p1));
-            pk[i] = pack_p(p0, p1);
-          }
-          tmem_st16u(ts + qt * 16, pk);
+        for (int i = 0; i < kTileN / 2; ++i) {
+          const int c = 2 * i;
+          float x0, x1;
+          f2_split(f2_fma(f2(s[c], s[c + 1]), sc2, nm2), x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          acc2[i & 3] = f2_add(acc2[i & 3], f2(p0, p1));
+          pk[i] = pack_p(p0, p1);
         }
         {
           float a0, a1, b0, b1;
@@ -580,11 +624,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
           f2_split(f2_add(acc2[2], acc2[3]), b0, b1);
           l += (a0 + a1) + (b0 + b1);
         }
+        // PV_w(gt-1) has read P_w and written O_w: both may change now. This
+        // group waits for every one of its PV completions in turn, so the wait
+        // is never more than one phase ahead of the barrier.
+        if (gt > 0 && !(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
+        tc_fence_after();
         if (!first_tile && __any_sync(0xffffffffu, need)) {
-          // O_w holds earlier tiles at the old reference: wait for them, then the
-          // whole warp rescales its rows (alpha = 1 for rows that keep theirs)
-          if (!(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
-          tc_fence_after();
+          // O_w holds earlier tiles at the old reference: the whole warp
+          // rescales its rows (alpha = 1 for rows that keep theirs)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float v[32];
@@ -594,6 +641,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
             tmem_st32(to + c * 32, v);
           }
         }
+#pragma unroll
+        for (int qt = 0; qt < kTileN / 32; ++qt) tmem_st16u(tp + qt * 16, pk + 16 * qt);
         tmem_wait_st();
         tc_fence_before();
         group_arrive(&bs->p_full[w]);
