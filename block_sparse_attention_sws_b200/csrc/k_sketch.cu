@@ -6,7 +6,8 @@
 //
 // 1. pool_project_kernel: one streaming pass over Q and K (one launch for
 //    both): 16-byte loads of each contiguous B x d block, per-column sums,
-//    the means, and their projection q~ = q_bar H_d, k~ = k_bar H_d. HBM-bound:
+//    the means, and their projection q~ = q_bar H_d, k~ = k_bar H_d as a
+//    Walsh-Hadamard transform in registers and shuffles. HBM-bound:
 //    Q and K are read exactly once and only the b x k sketches are written.
 // 2. scores_kernel: S = Q~ K~^T / sqrt(k) on and below the block diagonal.
 #include <algorithm>
@@ -35,22 +36,37 @@ constexpr int kPoolBatch = 8;   // 16-byte loads in flight per lane
 // columns (vector l mod VR of a row) on rows l / VR, l / VR + 32 / VR, ...,
 // kPoolBatch of them in flight at a time. bf16 columns are summed in fp32 over
 // one batch of rows, then in fp64; fp32 inputs are summed in fp64 throughout.
-// The column sums meet in a shuffle tree, the means (sum / rows, as the
-// definition divides) go to a per-warp shared row, and lane j forms output
-// column j of q~ = q_bar H_d (k~ for K heads) from it and column j of H_d.
+// The column sums meet in a shuffle tree that leaves every lane with the sums
+// of its columns c = VE (l mod VR) + e. H_d[c][j] = scale sign_c
+// (-1)^popcount(c & col_j), so q_bar H_d is a Walsh-Hadamard transform of
+// sign * q_bar read at the k sampled indices col_j: butterflies over e in
+// registers, then over the lane bits with xor shuffles; lane j fetches
+// transform entry col_j and scales it by scale / rows (the mean divides the
+// sums by the rows the block holds).
 template <typename T, int D>
 __global__ void __launch_bounds__(kPoolWarps * 32, 3)
     pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
-                        int32_t B, int64_t nblk, const double* __restrict__ hd, int32_t ksk,
-                        double* __restrict__ q_sk, double* __restrict__ k_sk) {
+                        int32_t B, int64_t nblk, const double* __restrict__ sign, const int32_t* __restrict__ col,
+                        double scale, int32_t ksk, double* __restrict__ q_sk, double* __restrict__ k_sk) {
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte vector
   constexpr int VR = D / VE;          // vectors per row
   static_assert(VR <= 32 && 32 % VR == 0, "row must map onto a whole number of lanes");
   constexpr int LPC = 32 / VR;        // rows covered by one warp-wide load
 
-  __shared__ double mean_row[kPoolWarps][D];
+  constexpr int kOut = D / 32;  // output columns per lane at most (k <= D)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int vc = lane % VR, rl = lane / VR;
+  double sg[VE];
+#pragma unroll
+  for (int e = 0; e < VE; ++e) sg[e] = sign[vc * VE + e];
+  int olane[kOut], oel[kOut];  // lane and element holding transform entry col_j, j = lane + 32 t
+#pragma unroll
+  for (int t = 0; t < kOut; ++t) {
+    const int j = lane + 32 * t;
+    const int pj = j < ksk ? col[j] : 0;
+    olane[t] = pj / VE;
+    oel[t] = pj % VE;
+  }
   const int64_t total = (int64_t)(hq + hkv) * nblk;
   const int64_t nw = (int64_t)gridDim.x * kPoolWarps;
   for (int64_t it = (int64_t)blockIdx.x * kPoolWarps + warp; it < total; it += nw) {
@@ -99,24 +115,42 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 3)
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
     }
-    if (lane < VR) {
-      const double cnt = static_cast<double>(rows);
+    double v[VE];
 #pragma unroll
-      for (int e = 0; e < VE; e += 2)
-        *reinterpret_cast<double2*>(&mean_row[warp][vc * VE + e]) = make_double2(acc[e] / cnt, acc[e + 1] / cnt);
-    }
-    __syncwarp();
-    double* out = head < hq ? q_sk + it * ksk : k_sk + (it - (int64_t)hq * nblk) * ksk;
-    for (int j = lane; j < ksk; j += 32) {
-      double a[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 8
-      for (int c = 0; c < D; c += 4) {
+    for (int e = 0; e < VE; ++e) v[e] = acc[e] * sg[e];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) a[u] = fma(mean_row[warp][c + u], __ldg(hd + (size_t)(c + u) * ksk + j), a[u]);
+    for (int hb = 1; hb < VE; hb <<= 1) {
+#pragma unroll
+      for (int e = 0; e < VE; ++e) {
+        if ((e & hb) == 0) {
+          const double a = v[e], b2 = v[e + hb];
+          v[e] = a + b2;
+          v[e + hb] = a - b2;
+        }
       }
-      out[j] = (a[0] + a[1]) + (a[2] + a[3]);
     }
-    __syncwarp();  // the row is rewritten by the next item
+#pragma unroll
+    for (int hb = 1; hb < VR; hb <<= 1) {
+      const bool upper = (lane & hb) != 0;
+#pragma unroll
+      for (int e = 0; e < VE; ++e) {
+        const double u = __shfl_xor_sync(0xffffffffu, v[e], hb);
+        v[e] = upper ? u - v[e] : v[e] + u;
+      }
+    }
+    const double f = scale / static_cast<double>(rows);
+    double* out = head < hq ? q_sk + it * ksk : k_sk + (it - (int64_t)hq * nblk) * ksk;
+#pragma unroll
+    for (int t = 0; t < kOut; ++t) {
+      if (32 * t >= ksk) break;  // warp-uniform
+      double w = 0.0;
+#pragma unroll
+      for (int e = 0; e < VE; ++e) {
+        const double x = __shfl_sync(0xffffffffu, v[e], olane[t]);
+        if (oel[t] == e) w = x;
+      }
+      if (lane + 32 * t < ksk) out[lane + 32 * t] = w * f;
+    }
   }
 }
 
@@ -183,8 +217,8 @@ cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int
   const int64_t nblk = ceil_div64(n, B);
   const int64_t total = (int64_t)(hq + hkv) * nblk;
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 3 * (int64_t)h->num_sms));
-  pool_project_kernel<T, D><<<grid, kPoolWarps * 32, 0, st>>>(q, k, n, hq, hkv, B, nblk, h->hd, h->cfg.sketch_dim,
-                                                              q_sk, k_sk);
+  pool_project_kernel<T, D><<<grid, kPoolWarps * 32, 0, st>>>(q, k, n, hq, hkv, B, nblk, h->sign, h->col, h->scale,
+                                                              h->cfg.sketch_dim, q_sk, k_sk);
   note_launches(1);
   return cudaGetLastError();
 }

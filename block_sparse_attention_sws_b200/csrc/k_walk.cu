@@ -40,14 +40,16 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
 }
 
 // C = A * Bm for lower-triangular b x b matrices on the fp64 tensor path
-// (mma.sync m16n8k4 f64). One 64 x 64 output tile per CTA (on or below the
-// diagonal, heaviest first), four warps of 32 x 32, k staged 16 at a time
-// through padded shared memory (conflict-free fragment loads) with the next
-// chunk prefetched into registers. Entries above the diagonal of A and Bm are
+// (mma.sync m16n8k4 f64). One 32 x 32 output tile per CTA of two warps (on or
+// below the diagonal, heaviest first; many small CTAs keep every SM busy and
+// waste less of the triangle than large tiles), each warp a 16 x 32 slice;
+// k staged 16 at a time through padded shared memory (row strides of 20 and
+// 36 doubles make the fragment loads conflict-free) with the next chunk
+// prefetched into registers. Entries above the diagonal of A and Bm are
 // treated as zero whatever the buffers hold.
-constexpr int kTT = 64, kTK = 16, kGemmThreads = 128;
-constexpr int kApad = kTK + 2;   // A tile row stride (doubles)
-constexpr int kBpad = kTT + 8;   // B tile row stride (doubles)
+constexpr int kTT = 32, kTK = 16, kGemmThreads = 64;
+constexpr int kApad = kTK + 4;   // A tile row stride (doubles)
+constexpr int kBpad = kTT + 4;   // B tile row stride (doubles)
 
 __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int64_t& tj) {
   // heaviest tiles (largest ti - tj) first
@@ -66,7 +68,7 @@ __device__ __forceinline__ void dmma_16x8x4(double (&c)[4], double a0, double a1
       : "d"(a0), "d"(a1), "d"(b0));
 }
 
-__global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __restrict__ A,
+__global__ void __launch_bounds__(kGemmThreads, 8) tri_gemm_kernel(const double* __restrict__ A,
                                                                 const double* __restrict__ Bm,
                                                                 double* __restrict__ C, int64_t b) {
   constexpr int PER = kTT * kTK / kGemmThreads;  // 8 elements of each operand chunk per thread
@@ -81,7 +83,6 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
   double* Ch = C + hoff;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
-  const int wm = warp >> 1, wn = warp & 1;
   const int64_t i0 = ti * kTT, j0 = tj * kTT;
   const int64_t kbeg = j0, kend = std::min<int64_t>(b, i0 + kTT);
 
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
       // A: element (row e / KC, k e % KC): 16 consecutive threads read one row
       const int64_t ar = i0 + e / kTK, ak = k0 + e % kTK;
       ra[q] = (ar < b && ak < kend && ak <= ar) ? Ah[ar * b + ak] : 0.0;
-      // B: element (k e / T, column e % T)
+      // B: element (k e / T, column e % T): a warp reads one row
       const int64_t bk = k0 + e / kTT, bc = j0 + e % kTT;
       rb[q] = (bk < kend && bc < b && bc <= bk) ? Bh[bk * b + bc] : 0.0;
     }
@@ -107,13 +108,11 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
     }
   };
 
-  double acc[2][4][4];
+  double acc[4][4];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int n8 = 0; n8 < 4; ++n8)
 #pragma unroll
-    for (int n8 = 0; n8 < 4; ++n8)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[mt][n8][v] = 0.0;
+    for (int v = 0; v < 4; ++v) acc[n8][v] = 0.0;
 
   int buf = 0;
   load(kbeg);
@@ -124,18 +123,13 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
     if (more) load(k0 + kTK);
 #pragma unroll
     for (int ks = 0; ks < kTK / 4; ++ks) {
-      double a[2][2], bf[4];
+      const double a0 = As[buf][warp * 16 + g][ks * 4 + t4];
+      const double a1 = As[buf][warp * 16 + g + 8][ks * 4 + t4];
+      double bf[4];
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        a[mt][0] = As[buf][wm * 32 + mt * 16 + g][ks * 4 + t4];
-        a[mt][1] = As[buf][wm * 32 + mt * 16 + g + 8][ks * 4 + t4];
-      }
+      for (int n8 = 0; n8 < 4; ++n8) bf[n8] = Bs[buf][ks * 4 + t4][n8 * 8 + g];
 #pragma unroll
-      for (int n8 = 0; n8 < 4; ++n8) bf[n8] = Bs[buf][ks * 4 + t4][wn * 32 + n8 * 8 + g];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4(acc[mt][n8], a[mt][0], a[mt][1], bf[n8]);
+      for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4(acc[n8], a0, a1, bf[n8]);
     }
     if (more) {
       store(buf ^ 1);
@@ -144,17 +138,14 @@ __global__ void __launch_bounds__(kGemmThreads) tri_gemm_kernel(const double* __
     }
   }
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
+  for (int hh = 0; hh < 2; ++hh) {
+    const int64_t i = i0 + warp * 16 + g + 8 * hh;
+    if (i >= b) continue;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int64_t i = i0 + wm * 32 + mt * 16 + g + 8 * hh;
-      if (i >= b) continue;
-#pragma unroll
-      for (int n8 = 0; n8 < 4; ++n8) {
-        const int64_t j = j0 + wn * 32 + n8 * 8 + 2 * t4;
-        if (j < b) Ch[i * b + j] = acc[mt][n8][2 * hh];
-        if (j + 1 < b) Ch[i * b + j + 1] = acc[mt][n8][2 * hh + 1];
-      }
+    for (int n8 = 0; n8 < 4; ++n8) {
+      const int64_t j = j0 + n8 * 8 + 2 * t4;
+      if (j < b) Ch[i * b + j] = acc[n8][2 * hh];
+      if (j + 1 < b) Ch[i * b + j + 1] = acc[n8][2 * hh + 1];
     }
   }
 }

@@ -107,15 +107,15 @@ int64_t sws_csr_nnz(const sws_config* c, int64_t n) {
   return nnz;
 }
 
-sws_status sws_build_projection_host(const sws_config* c, double* hd) {
-  sws_status s = sws_config_check(c);
-  if (s != SWS_OK) return s;
-  if (!hd) return SWS_ERR_INVALID_ARG;
-  const int d = c->head_dim, k = c->sketch_dim;
+// Signs and the column permutation of the projection (its first k entries
+// are the sampled columns), from the splitmix64 stream of the seed.
+static void projection_draws(const sws_config* c, std::vector<int>& sign, std::vector<int>& perm) {
+  const int d = c->head_dim;
   uint64_t state = c->seed ^ kProjectionTag;
   std::vector<uint64_t> draws(2 * d - 1);
   for (auto& x : draws) x = splitmix_next(state);
-  std::vector<int> sign(d), perm(d);
+  sign.assign(d, 1);
+  perm.resize(d);
   for (int r = 0; r < d; ++r) sign[r] = (draws[r] >> 63) ? -1 : 1;
   for (int r = 0; r < d; ++r) perm[r] = r;
   int next = d;
@@ -123,8 +123,23 @@ sws_status sws_build_projection_host(const sws_config* c, double* hd) {
     const int j = static_cast<int>(draws[next++] % static_cast<uint64_t>(r + 1));
     std::swap(perm[r], perm[j]);
   }
+}
+
+// 1/sqrt(k), formed as sqrt(d/k)/sqrt(d) like every entry of H_d
+static double projection_scale(const sws_config* c) {
+  const int d = c->head_dim, k = c->sketch_dim;
+  return std::sqrt(static_cast<double>(d) / k) / std::sqrt(static_cast<double>(d));
+}
+
+sws_status sws_build_projection_host(const sws_config* c, double* hd) {
+  sws_status s = sws_config_check(c);
+  if (s != SWS_OK) return s;
+  if (!hd) return SWS_ERR_INVALID_ARG;
+  const int d = c->head_dim, k = c->sketch_dim;
+  std::vector<int> sign, perm;
+  projection_draws(c, sign, perm);
   // H_d[r][c] = sqrt(d/k) * sign[r] * (-1)^popcount(r & perm[c]) / sqrt(d) = sign * (+-1) / sqrt(k)
-  const double scale = std::sqrt(static_cast<double>(d) / k) / std::sqrt(static_cast<double>(d));
+  const double scale = projection_scale(c);
   for (int r = 0; r < d; ++r)
     for (int cc = 0; cc < k; ++cc) {
       const int par = popcount32(static_cast<uint32_t>(r & perm[cc])) & 1;
@@ -174,18 +189,29 @@ sws_status sws_create(const sws_config* c, sws_handle** out) {
   h->cfg = *c;
   cudaError_t e = cudaGetDevice(&h->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  std::vector<int> sign_i, perm;
+  projection_draws(c, sign_i, perm);
+  std::vector<double> sign(sign_i.begin(), sign_i.end());
+  std::vector<int32_t> col(perm.begin(), perm.begin() + k);
+  h->scale = projection_scale(c);
   void* mem = nullptr;
   const size_t hd_bytes = hd.size() * sizeof(double);
-  if (e == cudaSuccess) e = cudaMalloc(&mem, 2 * hd_bytes + 256);
+  const size_t sign_bytes = static_cast<size_t>(d) * sizeof(double);
+  const size_t col_bytes = (static_cast<size_t>(k) * sizeof(int32_t) + 15) & ~size_t(15);
+  if (e == cudaSuccess) e = cudaMalloc(&mem, 2 * hd_bytes + sign_bytes + col_bytes + 256);
   if (e != cudaSuccess) {
     delete h;
     return cuda_status(e, "sws_create");
   }
   h->hd = static_cast<double*>(mem);
   h->hdt = h->hd + hd.size();
-  h->err = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mem) + 2 * hd_bytes);
+  h->sign = h->hdt + hd.size();
+  h->col = reinterpret_cast<int32_t*>(h->sign + d);
+  h->err = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(mem) + 2 * hd_bytes + sign_bytes + col_bytes);
   e = cudaMemcpy(h->hd, hd.data(), hd_bytes, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(h->hdt, hdt.data(), hd_bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->sign, sign.data(), sign_bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->col, col.data(), k * sizeof(int32_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int32_t));
   if (e != cudaSuccess) {
     cudaFree(mem);

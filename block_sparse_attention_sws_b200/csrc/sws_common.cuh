@@ -13,6 +13,9 @@ struct sws_handle {
   int num_sms;
   double* hd;    // [d, k] row-major
   double* hdt;   // [k, d] row-major (transpose, for contiguous per-output reads)
+  double* sign;  // [d] the random signs D of H_d (+1 / -1)
+  int32_t* col;  // [k] the sampled Hadamard columns P of H_d
+  double scale;  // 1/sqrt(k): H_d[r][c] = scale * sign[r] * (-1)^popcount(r & col[c])
   int32_t* err;  // device error word (guard code of the first failure, 0 = none)
 };
 
