@@ -67,7 +67,7 @@ __global__ void advance_kernel(int32_t* seq_lens, int32_t batch) {
 }
 
 // -------------------------------------------------------------- select ------
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {

@@ -27,7 +27,7 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
 }
 
 constexpr int kPoolWarps = 8;   // warps per CTA
-constexpr int kPoolBatch = 8;   // 16-byte loads in flight per lane
+constexpr int kPoolBatch = 16;  // 16-byte loads in flight per lane
 
 // Block means of Q (heads [0, hq)) and K (heads [hq, hq + hkv)) and their
 // projection by H_d, in one pass over Q and K. One warp per (head, block)
@@ -44,7 +44,7 @@ constexpr int kPoolBatch = 8;   // 16-byte loads in flight per lane
 // transform entry col_j and scales it by scale / rows (the mean divides the
 // sums by the rows the block holds).
 template <typename T, int D>
-__global__ void __launch_bounds__(kPoolWarps * 32, 3)
+__global__ void __launch_bounds__(kPoolWarps * 32, 2)
     pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
                         int32_t B, int64_t nblk, const double* __restrict__ sign, const int32_t* __restrict__ col,
                         double scale, int32_t ksk, double* __restrict__ q_sk, double* __restrict__ k_sk) {
@@ -177,11 +177,22 @@ __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ 
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   double acc[4][4] = {};
   for (int c0 = 0; c0 < k; c0 += kSC) {
-    for (int e = threadIdx.x; e < kST * kSC; e += 256) {
+    // all loads of the chunk in flight before any store to shared memory
+    constexpr int kPerThread = kST * kSC / 256;
+    double qv[kPerThread], kv[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int e = threadIdx.x + 256 * u;
       const int r = e / kSC, c = e % kSC;
       const int64_t qi = ti * kST + r, kj = tj * kST + r;
-      qs[r][c] = (qi < b && c0 + c < k) ? qh[qi * k + c0 + c] : 0.0;
-      ks[r][c] = (kj < b && c0 + c < k) ? kh[kj * k + c0 + c] : 0.0;
+      qv[u] = (qi < b && c0 + c < k) ? qh[qi * k + c0 + c] : 0.0;
+      kv[u] = (kj < b && c0 + c < k) ? kh[kj * k + c0 + c] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int e = threadIdx.x + 256 * u;
+      qs[e / kSC][e % kSC] = qv[u];
+      ks[e / kSC][e % kSC] = kv[u];
     }
     __syncthreads();
 #pragma unroll 4
@@ -216,7 +227,7 @@ cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int
   const int32_t B = h->cfg.block_size;
   const int64_t nblk = ceil_div64(n, B);
   const int64_t total = (int64_t)(hq + hkv) * nblk;
-  const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 3 * (int64_t)h->num_sms));
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 2 * (int64_t)h->num_sms));
   pool_project_kernel<T, D><<<grid, kPoolWarps * 32, 0, st>>>(q, k, n, hq, hkv, B, nblk, h->sign, h->col, h->scale,
                                                               h->cfg.sketch_dim, q_sk, k_sk);
   note_launches(1);

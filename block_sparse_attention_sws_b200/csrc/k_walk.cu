@@ -20,8 +20,49 @@ namespace {
 
 // One warp per row. temp = 1 for the softmax of §4; temp = s gives the
 // entrywise power with renormalised rows (softmax(S)^s / sum = softmax(s S)).
+// Each lane keeps its exponentials (j = lane + 32 u) in registers between the
+// sum and the normalisation, so every entry takes one exponential.
+constexpr int kSoftmaxPerLane = 32;  // rows up to 1024 blocks wide
+
 __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __restrict__ S, int64_t b, int64_t rows,
                                                             double temp, double* __restrict__ A) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t i = row % b;
+  const double* s = S + row * b;
+  double* a = A + row * b;
+  double x[kSoftmaxPerLane];
+  double mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+    const int64_t j = lane + 32 * u;
+    x[u] = j <= i ? temp * s[j] : -INFINITY;
+    mx = fmax(mx, x[u]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  double sum = 0.0;
+#pragma unroll
+  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+    if (32 * u > i) break;  // warp-uniform: no entry j <= i left for any lane
+    x[u] = exp(x[u] - mx);  // exp(-inf) = 0 for j > i
+    sum += x[u];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const double inv = 1.0 / sum;
+#pragma unroll
+  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+    const int64_t j = lane + 32 * u;
+    if (j < b) a[j] = j <= i ? x[u] * inv : 0.0;
+  }
+}
+
+// The same for rows wider than 32 x kSoftmaxPerLane blocks: two passes over
+// the row, the exponentials recomputed for the normalisation.
+__global__ void __launch_bounds__(256) block_softmax_wide_kernel(const double* __restrict__ S, int64_t b,
+                                                                 int64_t rows, double temp, double* __restrict__ A) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -36,7 +77,8 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   for (int64_t j = lane; j <= i; j += 32) sum += exp(temp * s[j] - mx);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-  for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) / sum : 0.0;
+  const double inv = 1.0 / sum;
+  for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) * inv : 0.0;
 }
 
 // C = A * Bm for lower-triangular b x b matrices on the fp64 tensor path
@@ -161,6 +203,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= rows) return;
   uint64_t* keys = keys_all + (size_t)warp * b;
+  int* hist = reinterpret_cast<int*>(keys_all + (size_t)(blockDim.x >> 5) * b) + warp * 256;
   const int64_t h = row / b, i = row % b;
   const double* r = R + row * b;
   double* ws = walk_state + row * b;
@@ -179,7 +222,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
     if (i == b - 1) row_ptr[h * (b + 1) + b] = static_cast<int32_t>(rp + tau);
   }
   __syncwarp();
-  warp_top_tau(keys, static_cast<int>(i + 1), tau, col_idx + h * nnz + rp, err);
+  warp_top_tau8(keys, static_cast<int>(i + 1), tau, col_idx + h * nnz + rp, hist, err);
 }
 
 }  // namespace
@@ -188,7 +231,10 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
                                  cudaStream_t st) {
   const int64_t rows = (int64_t)hq * b;
   const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
-  block_softmax_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
+  if (b <= 32 * kSoftmaxPerLane)
+    block_softmax_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
+  else
+    block_softmax_wide_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -205,7 +251,7 @@ cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32
                           int32_t* row_ptr, int32_t* col_idx, cudaStream_t st) {
   const int64_t rows = (int64_t)hq * b;
   int warps = static_cast<int>(std::min<int64_t>(8, std::max<int64_t>(1, (160 << 10) / (b * 8))));
-  const size_t smem = (size_t)warps * b * sizeof(uint64_t);
+  const size_t smem = (size_t)warps * (b * sizeof(uint64_t) + 256 * sizeof(int));
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int64_t nnz = 0;

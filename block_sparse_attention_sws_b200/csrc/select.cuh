@@ -80,4 +80,90 @@ __device__ __forceinline__ void warp_top_tau(const uint64_t* keys, int m, int ta
   if (lane == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
 }
 
+// The same selection with 8-bit digits: eight passes, each counting the keys
+// that still match the prefix found so far in a 256-bin histogram hist[]
+// (shared memory owned by this warp), then the ordered compaction above.
+__device__ __forceinline__ void warp_top_tau8(const uint64_t* keys, int m, int tau, int32_t* out, int* hist,
+                                              int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  uint64_t prefix = 0, pmask = 0;
+  int need = tau;
+  bool all_cands = false;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0;
+    __syncwarp();
+    for (int j = lane; j < m; j += 32) {
+      const uint64_t key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncwarp();
+    // lane l owns bins 255 - 8 l - u (u = 0..7), in descending key order
+    int c[8], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      c[u] = hist[255 - 8 * lane - u];
+      sum += c[u];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int excl = incl - sum;
+    int digit = 0, rest = 0, cnt = 0;
+    const bool here = excl < need && need <= incl;
+    if (here) {
+      int run = excl;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (run + c[u] >= need) {
+          digit = 255 - 8 * lane - u;
+          rest = need - run;
+          cnt = c[u];
+          break;
+        }
+        run += c[u];
+      }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, here);
+    const int src = who ? __ffs(who) - 1 : 0;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    rest = __shfl_sync(0xffffffffu, rest, src);
+    cnt = __shfl_sync(0xffffffffu, cnt, src);
+    __syncwarp();  // every lane has read hist before the next pass clears it
+    prefix |= static_cast<uint64_t>(digit) << shift;
+    pmask |= 255ull << shift;
+    need = rest;
+    if (cnt == need) {
+      all_cands = true;
+      break;
+    }
+  }
+  const unsigned lt = lanemask_lt();
+  int base = 0, ties = 0;
+  for (int j0 = 0; j0 < m; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < m;
+    const uint64_t km = valid ? (keys[j] & pmask) : 0;
+    const bool above = valid && km > prefix;
+    const bool cand = valid && km == prefix;
+    const unsigned cb = __ballot_sync(0xffffffffu, cand);
+    bool take = cand;
+    if (!all_cands) {
+      take = cand && (ties + __popc(cb & lt)) < need;
+      ties += __popc(cb);
+    }
+    const bool sel = above || take;
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = base + __popc(sb & lt);
+      if (pos < tau) out[pos] = j;
+    }
+    base += __popc(sb);
+  }
+  if (lane == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
+}
+
 }  // namespace sws
