@@ -9,7 +9,8 @@
 //    the means, and their projection q~ = q_bar H_d, k~ = k_bar H_d as a
 //    Walsh-Hadamard transform in registers and shuffles. HBM-bound:
 //    Q and K are read exactly once and only the b x k sketches are written.
-// 2. scores_kernel: S = Q~ K~^T / sqrt(k) on and below the block diagonal.
+// 2. scores_kernel: S = Q~ K~^T / sqrt(k) on and below the block diagonal, on
+//    the fp64 tensor path.
 #include <algorithm>
 
 #include "sws_common.cuh"
@@ -154,16 +155,25 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
   }
 }
 
-// S[h, i, j] = q~_i . k~_j / sqrt(k) for j <= i, fp64, 64 x 64 tiles on and
-// below the diagonal; 256 threads, 4 x 4 outputs each.
-constexpr int kST = 64;
-constexpr int kSC = 32;  // sketch-dimension chunk staged in shared memory
+// S[h, i, j] = q~_i . k~_j / sqrt(k) for j <= i, fp64, on the fp64 tensor path
+// (mma.sync m16n8k4 f64): one 32 x 32 tile on or below the block diagonal per
+// CTA of two warps (each a 16 x 32 slice), the sketch dimension staged 16 at a
+// time through padded shared memory (conflict-free fragment loads, as in the
+// walk's GEMM). Query head h reads the sketches of KV head h / group.
+constexpr int kST = 32, kSC = 16;
 
-__global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ q_sk, const double* __restrict__ k_sk,
-                                                     int64_t b, int32_t hq, int32_t group, int32_t k,
-                                                     double inv_sqrt_k, double* __restrict__ S) {
-  __shared__ double qs[kST][kSC + 1];
-  __shared__ double ks[kST][kSC + 1];
+__device__ __forceinline__ void dmma_16x8x4_s(double (&c)[4], double a0, double a1, double b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a0), "d"(a1), "d"(b0));
+}
+
+__global__ void __launch_bounds__(64) scores_kernel(const double* __restrict__ q_sk, const double* __restrict__ k_sk,
+                                                    int64_t b, int32_t hq, int32_t group, int32_t k,
+                                                    double inv_sqrt_k, double* __restrict__ S) {
+  __shared__ __align__(16) double qs[kST][kSC + 4];  // [query block][sketch dim]
+  __shared__ __align__(16) double ks[kSC][kST + 4];  // [sketch dim][key block]
   const int64_t t = blockIdx.x;
   // tile (ti, tj), tj <= ti, from the linear lower-triangle index
   int64_t ti = static_cast<int64_t>((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
@@ -171,52 +181,52 @@ __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ 
   while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
   const int64_t tj = t - ti * (ti + 1) / 2;
   const int h = blockIdx.y;
-  const int g = h / group;
   const double* qh = q_sk + (size_t)h * b * k;
-  const double* kh = k_sk + (size_t)g * b * k;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  double acc[4][4] = {};
-  for (int c0 = 0; c0 < k; c0 += kSC) {
-    // all loads of the chunk in flight before any store to shared memory
-    constexpr int kPerThread = kST * kSC / 256;
-    double qv[kPerThread], kv[kPerThread];
+  const double* kh = k_sk + (size_t)(h / group) * b * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int64_t i0 = ti * kST, j0 = tj * kST;
+  double acc[4][4];
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-      const int e = threadIdx.x + 256 * u;
-      const int r = e / kSC, c = e % kSC;
-      const int64_t qi = ti * kST + r, kj = tj * kST + r;
+  for (int n8 = 0; n8 < 4; ++n8)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[n8][v] = 0.0;
+  for (int c0 = 0; c0 < k; c0 += kSC) {
+    constexpr int kPer = kST * kSC / 64;  // 8 elements of each operand per thread
+    double qv[kPer], kv[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + 64 * u;
+      const int r = e / kSC, c = e % kSC;  // 16 consecutive threads read one row
+      const int64_t qi = i0 + r, kj = j0 + r;
       qv[u] = (qi < b && c0 + c < k) ? qh[qi * k + c0 + c] : 0.0;
       kv[u] = (kj < b && c0 + c < k) ? kh[kj * k + c0 + c] : 0.0;
     }
+    __syncthreads();  // the previous chunk's fragments have been read
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-      const int e = threadIdx.x + 256 * u;
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + 64 * u;
       qs[e / kSC][e % kSC] = qv[u];
-      ks[e / kSC][e % kSC] = kv[u];
+      ks[e % kSC][e / kSC] = kv[u];
     }
     __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kSC; ++c) {
-      double a[4], bb[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[u] = qs[ty + 16 * u][c];
-        bb[u] = ks[tx + 16 * u][c];
-      }
+    for (int kk = 0; kk < kSC / 4; ++kk) {
+      const double a0 = qs[warp * 16 + g][kk * 4 + t4];
+      const double a1 = qs[warp * 16 + g + 8][kk * 4 + t4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bb[v], acc[u][v]);
+      for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4_s(acc[n8], a0, a1, ks[kk * 4 + t4][n8 * 8 + g]);
     }
-    __syncthreads();
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t i = ti * kST + ty + 16 * u;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int64_t i = i0 + warp * 16 + g + 8 * hh;
+    if (i >= b) continue;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int64_t j = tj * kST + tx + 16 * v;
-      if (i < b && j <= i) S[((size_t)h * b + i) * b + j] = acc[u][v] * inv_sqrt_k;
+    for (int n8 = 0; n8 < 4; ++n8) {
+      const int64_t j = j0 + n8 * 8 + 2 * t4;
+      if (j <= i) S[((size_t)h * b + i) * b + j] = acc[n8][2 * hh] * inv_sqrt_k;
+      if (j + 1 <= i) S[((size_t)h * b + i) * b + j + 1] = acc[n8][2 * hh + 1] * inv_sqrt_k;
     }
   }
 }
@@ -258,7 +268,7 @@ cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const 
   const int64_t nt = ceil_div64(b, kST);
   dim3 grid(static_cast<unsigned>(nt * (nt + 1) / 2), hq);
   const int32_t k = h->cfg.sketch_dim;
-  scores_kernel<<<grid, 256, 0, st>>>(q_sk, k_sk, b, hq, hq / hkv, k, 1.0 / sqrt((double)k), scores);
+  scores_kernel<<<grid, 64, 0, st>>>(q_sk, k_sk, b, hq, hq / hkv, k, 1.0 / sqrt((double)k), scores);
   note_launches(1);
   return cudaGetLastError();
 }
