@@ -345,7 +345,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int kAttnThreads = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 
 // Row u of a staged [B][D] bf16 tile keeps its 16-byte chunks XOR-swizzled by
 // u mod (D/8), so that the column accesses of the mma fragments and of
@@ -368,8 +368,9 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
   constexpr int TILE = BS * D;
   extern __shared__ __align__(16) uint8_t smem[];
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);  // [kStages][2][BS][D]
-  float* sc = reinterpret_cast<float*>(stage + kStages * 2 * TILE);  // [8][BS]
-  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(sc + 8 * BS);  // [8][BS + 8]
+  constexpr int SCS = BS + 4;  // padded score row: the 8 head rows fall in different banks
+  float* sc = reinterpret_cast<float*>(stage + kStages * 2 * TILE);  // [8][SCS]
+  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(sc + 8 * SCS);  // [8][BS + 8]
   float* corr_s = reinterpret_cast<float*>(ps + 8 * (BS + 8));       // [8]
   float* ml_s = corr_s + 8;                                          // [8][2]
 
@@ -464,15 +465,15 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
       if (gq < G) {
         const bool hv = (hm >> gq) & 1u;
         const int u0 = n0 + 2 * tq;
-        sc[gq * BS + u0] = (hv && t0 + u0 < len) ? c[0] * qscale : -INFINITY;
-        sc[gq * BS + u0 + 1] = (hv && t0 + u0 + 1 < len) ? c[1] * qscale : -INFINITY;
+        sc[gq * SCS + u0] = (hv && t0 + u0 < len) ? c[0] * qscale : -INFINITY;
+        sc[gq * SCS + u0 + 1] = (hv && t0 + u0 + 1 < len) ? c[1] * qscale : -INFINITY;
       }
     }
     __syncthreads();
     // online softmax: warp w owns heads w, w + 4
     for (int r = warp; r < G; r += 4) {
       float mx = -INFINITY;
-      for (int u = lane; u < BS; u += 32) mx = fmaxf(mx, sc[r * BS + u]);
+      for (int u = lane; u < BS; u += 32) mx = fmaxf(mx, sc[r * SCS + u]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       const float mr = ml_s[2 * r];
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
       if (mn != -INFINITY) {
         corr = exp2f(mr - mn);
         for (int u = lane; u < BS; u += 32) {
-          const float p = exp2f(sc[r * BS + u] - mn);
+          const float p = exp2f(sc[r * SCS + u] - mn);
           sum += p;
           ps[r * (BS + 8) + u] = __float2bfloat16_rn(p);
         }
@@ -575,7 +576,7 @@ cudaError_t launch_attn3(const __nv_bfloat16* q, const __nv_bfloat16* kc, const 
                          int32_t hkv, int64_t max_len, int64_t max_blocks, const int32_t* lens, const int32_t* sel,
                          const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits, int32_t* err,
                          cudaStream_t st) {
-  const size_t smem = (size_t)kStages * 2 * BS * D * 2 + 8 * BS * 4 + 8 * (BS + 8) * 2 + 8 * 4 + 16 * 4;
+  const size_t smem = (size_t)kStages * 2 * BS * D * 2 + 8 * (BS + 4) * 4 + 8 * (BS + 8) * 2 + 8 * 4 + 16 * 4;
   auto kern = decode_attn_kernel<D, BS, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
