@@ -237,23 +237,34 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
   }
   __syncthreads();
 
-  // 2. z_j = q~ . k~_j / sqrt(k) for every head, one thread per key block
+  // 2. z_j = q~ . k~_j / sqrt(k) for every head on the fp64 tensor path: one
+  //    m16n8k4 product per 8 key blocks and 4 sketch dims, the group's query
+  //    heads as rows 0..group-1 of A; a lane's k~ fragment is 4 consecutive
+  //    doubles of one cached block, so every load uses whole sectors
   double* z = reinterpret_cast<double*>(keys);
   const double inv_sqrt_k = 1.0 / sqrt((double)k);
-  for (int j = tid; j < nb; j += kSelThreads) {
-    const double* kr = ksk + (int64_t)j * k;
-    double acc[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
-    for (int c = 0; c < k; ++c) {
-      const double kv = kr[c];
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < group) acc[r] = fma(qt[r * k + c], kv, acc[r]);
+  {
+    const int g8 = lane >> 2, t4 = lane & 3;
+    for (int n0 = warp * 8; n0 < nb; n0 += kSelWarps * 8) {
+      const int j = n0 + g8;
+      const double* kr = ksk + (int64_t)(j < nb ? j : 0) * k;
+      double c4[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int c0 = 0; c0 < k; c0 += 4) {
+        const int c = c0 + t4;
+        const double a0 = (g8 < group && c < k) ? qt[g8 * k + c] : 0.0;
+        const double b0 = (j < nb && c < k) ? kr[c] : 0.0;
+        asm volatile(
+            "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+            : "+d"(c4[0]), "+d"(c4[1]), "+d"(c4[2]), "+d"(c4[3])
+            : "d"(a0), "d"(0.0), "d"(b0));
+      }
+      // c4[0], c4[1]: head g8, key blocks n0 + 2 t4 and n0 + 2 t4 + 1
+      if (g8 < group) {
+        const int j0 = n0 + 2 * t4;
+        if (j0 < nb) z[g8 * max_blocks + j0] = c4[0] * inv_sqrt_k;
+        if (j0 + 1 < nb) z[g8 * max_blocks + j0 + 1] = c4[1] * inv_sqrt_k;
+      }
     }
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < group) z[r * max_blocks + j] = acc[r] * inv_sqrt_k;
   }
   __syncthreads();
 
