@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--decode-n0", type=int, default=None, help="shorter cached prompt (profiling only)")
     ap.add_argument("--decode-layers", type=int, default=None, help="fewer decode layers (profiling only)")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement (profiling only)")
+    ap.add_argument("--no-variants", action="store_true", help="skip the elementwise-walk and dense-first variants")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -335,6 +336,44 @@ def bench_prefill(args, world, S, W, torch):
     return res
 
 
+def bench_prefill_variants(args, world, S, W, torch, pf):
+    """The pages' own alternatives on the same inputs, timed like the headline
+    step: the entrywise walk power (the other reading of (.)^s) and the
+    dense-first-two-layers policy of §7."""
+    w, inputs = pf["w"], pf["inputs"]
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, 20))
+    out = {}
+    for name, mode, dense in (("elementwise_walk", S.SWS_WALK_ELEMENTWISE, 0),
+                              ("dense_first_2_layers", S.SWS_WALK_MATRIX_POWER, 2)):
+        cfg = S.make_config(w.d, w.B, w.k, w.s, mode, w.density, w.seed)
+        h = S.Handle(cfg)
+        path = S.PrefillPath(h, w.n, w.hq, w.hkv, torch.bfloat16, dense_layers=dense)
+
+        def step():
+            for layer, (Q, K, V) in enumerate(inputs):
+                path.layer(Q, K, V, layer == 0, layer=layer)
+
+        for _ in range(args.warmup):
+            step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        ms = max_over_ranks(a.elapsed_time(b), world) / steps
+        out[name] = {"tokens_per_s": world * w.n / (ms * 1e-3), "ms_per_step": ms, "steps": steps}
+        h.close()
+        if path.h_dense is not None:
+            path.h_dense.close()
+        del path
+    return out
+
+
 def bench_prefill_e2e(args, world, S, torch, pf):
     w, path, inputs = pf["w"], pf["path"], pf["inputs"]
     host_in = [tuple(x.cpu().pin_memory() for x in t) for t in inputs]
@@ -527,6 +566,8 @@ def main():
     line["sketch_roofline"]["frac"] = line["sketch_roofline"]["achieved"] / peaks["hbm_gbs"]
     if not args.no_e2e:
         line["e2e"] = bench_prefill_e2e(args, world, S, torch, pf)
+    if not args.no_variants:
+        line["variants"] = bench_prefill_variants(args, world, S, W, torch, pf)
     pf["h"].close()
     del pf
     torch.cuda.empty_cache()

@@ -13,10 +13,17 @@ from . import _lib as L
 class PrefillPath:
     """Per-layer prefill: sws_sketch -> sws_walk_select -> sws_sparse_attn_prefill.
 
-    The walk state R [hq, b, b] (fp64) is carried from layer to layer."""
+    The walk state R [hq, b, b] (fp64) is carried from layer to layer.
 
-    def __init__(self, handle: L.Handle, n: int, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda"):
+    ``dense_layers`` is the caller policy of "Scout Before You Attend" §7 (the
+    first layers attend densely): layers below it select every causal block,
+    through a second handle with density 1/1 and the same projection, while
+    the walk state still runs through them."""
+
+    def __init__(self, handle: L.Handle, n: int, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda",
+                 dense_layers: int = 0):
         cfg = handle.cfg
+        self.dense_layers = dense_layers
         self.h, self.n, self.hq, self.hkv = handle, n, hq, hkv
         self.b = L.sws_num_blocks(cfg, n)
         self.nnz = L.sws_csr_nnz(cfg, n)
@@ -33,23 +40,43 @@ class PrefillPath:
         wss = L.sws_workspace_size(cfg, L.SWS_OP_SKETCH, n, hq, hkv)
         self.ws_sketch = torch.empty(max(wss, 16), dtype=torch.uint8, device=device)
         self.o = torch.empty(hq, n, d, dtype=dtype, device=device)
+        self.h_dense = None
+        if dense_layers > 0:
+            self.h_dense = L.Handle(L.make_config(cfg.head_dim, cfg.block_size, cfg.sketch_dim, cfg.walk_power,
+                                                  cfg.walk_mode, (1, 1), cfg.seed))
+            nnz_dense = L.sws_csr_nnz(self.h_dense.cfg, n)
+            self.row_ptr_dense = torch.empty(hq, self.b + 1, dtype=torch.int32, device=device)
+            self.col_idx_dense = torch.empty(hq, nnz_dense, dtype=torch.int32, device=device)
+
+    def _dense(self, layer) -> bool:
+        return self.h_dense is not None and layer is not None and layer < self.dense_layers
+
+    def csr(self, layer=None):
+        """(row_ptr, col_idx) that the given layer uses."""
+        if self._dense(layer):
+            return self.row_ptr_dense, self.col_idx_dense
+        return self.row_ptr, self.col_idx
 
     def sketch(self, q, k, stream=None):
         L.sws_sketch(self.h, q, k, self.q_sk, self.k_sk, self.scores, self.ws_sketch, stream)
 
-    def walk_select(self, first_layer: bool, stream=None):
-        L.sws_walk_select(self.h, self.scores, self.n, first_layer, self.walk_state, self.row_ptr, self.col_idx,
-                          self.ws, stream)
+    def walk_select(self, first_layer: bool, stream=None, layer=None):
+        h = self.h_dense if self._dense(layer) else self.h
+        rp, ci = self.csr(layer)
+        L.sws_walk_select(h, self.scores, self.n, first_layer, self.walk_state, rp, ci, self.ws, stream)
 
-    def attention(self, q, k, v, out=None, stream=None):
+    def attention(self, q, k, v, out=None, stream=None, layer=None):
         o = self.o if out is None else out
-        L.sws_sparse_attn_prefill(self.h, q, k, v, self.row_ptr, self.col_idx, o, None, stream)
+        h = self.h_dense if self._dense(layer) else self.h
+        rp, ci = self.csr(layer)
+        L.sws_sparse_attn_prefill(h, q, k, v, rp, ci, o, None, stream)
         return o
 
-    def layer(self, q, k, v, first_layer: bool, out=None, stream=None):
+    def layer(self, q, k, v, first_layer: bool, out=None, stream=None, layer=None):
+        """One layer; ``layer`` (its index) is needed only with dense_layers > 0."""
         self.sketch(q, k, stream)
-        self.walk_select(first_layer, stream)
-        return self.attention(q, k, v, out, stream)
+        self.walk_select(first_layer, stream, layer)
+        return self.attention(q, k, v, out, stream, layer)
 
 
 class DecodePath:

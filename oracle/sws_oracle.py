@@ -36,6 +36,13 @@ reason, in the design notes):
      rho^l = rho^{l-1} + s * (z^l - logsumexp(z^l)).
   R8 the decode token is appended to the cache before it attends.
 No blocking, fusion or reordering is done beyond what those definitions state.
+
+Group-shared selection (an extension the pages do not define; §8 row F1 of
+the build's scope): the query heads of one GQA group share one set of key
+blocks per query block, the top-tau of the sum of the group's walk rows
+(their mean up to a positive factor) in prefill, and of the log-sum-exp over
+the group's log-domain walk rows rho in decode (the same sum, taken of
+exp(rho), in the log domain).
 """
 from __future__ import annotations
 
@@ -50,6 +57,7 @@ __all__ = [
     "walk_matrix", "walk_update", "tau_of_row", "csr_nnz", "top_tau_row", "select_top_tau",
     "sparse_attention_block", "sparse_attention", "prefill_layer", "PrefillState",
     "decode_block_means", "decode_layer_select", "decode_attention",
+    "group_shared_walk_rows", "group_shared_log_rows",
 ]
 
 _M64 = (1 << 64) - 1
@@ -283,13 +291,34 @@ class PrefillState:
         self.R = {}
 
 
+def group_shared_walk_rows(R_heads: Sequence[np.ndarray]) -> np.ndarray:
+    """Selection scores shared by one GQA group: the sum of its heads' walk
+    matrices, added in head order (their mean up to the factor 1/group, which
+    does not change the ranking)."""
+    acc = np.array(R_heads[0], dtype=np.float64, copy=True)
+    for R in R_heads[1:]:
+        acc = acc + R
+    return acc
+
+
+def group_shared_log_rows(rho_heads: np.ndarray) -> np.ndarray:
+    """Decode counterpart: log(sum_h exp(rho_h)) per key block for the rows
+    rho_heads [group, nb], as max + log(sum exp(rho - max))."""
+    m = rho_heads.max(axis=0)
+    return m + np.log(np.exp(rho_heads - m).sum(axis=0))
+
+
 def prefill_layer(Q, K, V, Hd, B: int, s: int, density: Tuple[int, int], state: PrefillState,
-                  heads: Optional[Sequence[int]] = None, attention_blocks="all", mode: str = "matrix_power"):
+                  heads: Optional[Sequence[int]] = None, attention_blocks="all", mode: str = "matrix_power",
+                  select: str = "per_head"):
     """One layer of the prefill path for the listed query heads.
 
     Q [hq, n, d], K and V [hkv, n, d] (any float dtype; widened to fp64).
     Query head h reads KV head h // (hq / hkv). ``attention_blocks``: "all",
     None (skip attention), or a list of query blocks to compute.
+    ``select``: "per_head" (each head its own top-tau) or "group_shared" (the
+    group's heads share the top-tau of ``group_shared_walk_rows``; every head
+    of a listed head's group is then computed, since the choice needs them all).
     Returns per head: q_tilde, k_tilde, S, R (the new walk state), CSR and O.
     """
     hq, hkv = Q.shape[0], K.shape[0]
@@ -297,7 +326,39 @@ def prefill_layer(Q, K, V, Hd, B: int, s: int, density: Tuple[int, int], state: 
     num, den = density
     out = {}
     kbar_cache = {}
-    for h in (range(hq) if heads is None else heads):
+    heads = list(range(hq) if heads is None else heads)
+    if select == "group_shared":
+        heads = sorted({g * group + r for h in heads for g in [h // group] for r in range(group)})
+    shared = {}
+    if select == "group_shared":
+        # the walk of every head of the groups first, then one choice per group
+        for h in heads:
+            g = h // group
+            q64 = np.asarray(Q[h], dtype=np.float64)
+            if g not in kbar_cache:
+                kbar_cache[g] = block_means(np.asarray(K[g], dtype=np.float64), B)
+            qt = sketch_project(block_means(q64, B), Hd)
+            kt = sketch_project(kbar_cache[g], Hd)
+            S = sketch_scores(qt, kt)
+            M = walk_matrix(block_attention(S), s, mode)
+            R = walk_update(state.R.get(h), M)
+            state.R[h] = R
+            out[h] = dict(q_tilde=qt, k_tilde=kt, S=S, R=R)
+        for g in sorted({h // group for h in heads}):
+            shared[g] = select_top_tau(group_shared_walk_rows([out[g * group + r]["R"] for r in range(group)]),
+                                       num, den)
+        for h in heads:
+            g = h // group
+            row_ptr, col_idx = shared[g]
+            O = None
+            if attention_blocks is not None:
+                qb = None if attention_blocks == "all" else attention_blocks
+                O = sparse_attention(np.asarray(Q[h], dtype=np.float64), np.asarray(K[g], dtype=np.float64),
+                                     np.asarray(V[g], dtype=np.float64), row_ptr, col_idx, B, qb)
+            out[h].update(row_ptr=row_ptr, col_idx=col_idx, O=O,
+                          shared_scores=group_shared_walk_rows([out[g * group + r]["R"] for r in range(group)]))
+        return out
+    for h in heads:
         g = h // group
         q64 = np.asarray(Q[h], dtype=np.float64)
         if g not in kbar_cache:
@@ -328,12 +389,15 @@ def decode_block_means(Kcache: np.ndarray, length: int, B: int) -> np.ndarray:
 
 
 def decode_layer_select(q_tok, Kcaches, length: int, Hd, B: int, s: int, density: Tuple[int, int],
-                        rho_prev: Optional[np.ndarray]):
+                        rho_prev: Optional[np.ndarray], select: str = "per_head"):
     """Selection for one decode token in one layer, all query heads.
 
     q_tok [hq, d]; Kcaches [hkv, >=length, d] holds the new token at length-1.
     rho_prev [hq, nb] (None in the first layer). Returns (rho [hq, nb],
     z [hq, nb], sel: list of ascending block-index arrays, one per head).
+    ``select`` = "group_shared": every head of a GQA group gets the top-tau of
+    ``group_shared_log_rows`` of the group's rho rows (the walk state itself
+    stays per head).
     """
     hq, hkv = q_tok.shape[0], Kcaches.shape[0]
     group = hq // hkv
@@ -348,7 +412,11 @@ def decode_layer_select(q_tok, Kcaches, length: int, Hd, B: int, s: int, density
     m = z.max(axis=1, keepdims=True)
     lse = m + np.log(np.exp(z - m).sum(axis=1, keepdims=True))
     rho = s * (z - lse) + (0.0 if rho_prev is None else rho_prev)
-    sel = [top_tau_row(rho[h], tau) for h in range(hq)]
+    if select == "group_shared":
+        gsel = [top_tau_row(group_shared_log_rows(rho[g * group:(g + 1) * group]), tau) for g in range(hkv)]
+        sel = [gsel[h // group] for h in range(hq)]
+    else:
+        sel = [top_tau_row(rho[h], tau) for h in range(hq)]
     return rho, z, sel
 
 

@@ -197,3 +197,35 @@ def test_invalid_arguments_queue_nothing():
         S.sws_walk_select(h, sc, 256, True, sc, torch.zeros(4, 5, dtype=torch.int32, device="cuda"),
                           torch.zeros(4, 8, dtype=torch.int32, device="cuda"), ws)
     assert e.value.status == S.SWS_ERR_WORKSPACE
+
+
+def test_dense_first_layers_policy():
+    """The dense-first-layers policy of §7: layers 0-1 select every causal block
+    (the walk still runs through them), later layers the configured density;
+    compared with the oracle run with density 1/1 for the first two layers."""
+    w = W.PREFILL_16K.scaled(name="dense_first2", n=2000, hq=4, hkv=2, layers=4)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    path = S.PrefillPath(h, w.n, w.hq, w.hkv, dense_layers=2)
+    Hd = oracle.srht_matrix(w.d, w.k, w.seed)
+    st = so.PrefillState()
+    for layer in range(w.layers):
+        Q, K, V = W.prefill_layer_inputs(w, layer, "cuda")
+        o = path.layer(Q, K, V, layer == 0, layer=layer)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        dens = (1, 1) if layer < 2 else w.density
+        ref = so.prefill_layer(LazyHeads(Q), LazyHeads(K), LazyHeads(V), Hd, w.B, w.s, dens, st, heads=range(w.hq),
+                               attention_blocks=None)
+        rp_all, ci_all = (x.cpu().numpy() for x in path.csr(layer))
+        og = o.float().cpu().numpy()
+        for hh in range(w.hq):
+            r = ref[hh]
+            compare_walk(path.walk_state[hh].cpu().numpy(), r["R"])
+            rp, ci = rp_all[hh], ci_all[hh]
+            check_csr_valid(rp, ci, w.b, *dens)
+            compare_csr(rp, ci, r["row_ptr"], r["col_idx"], r["R"])
+            Qh, Kg, Vg = LazyHeads(Q)[hh], LazyHeads(K)[hh // 2], LazyHeads(V)[hh // 2]
+            for i in (0, w.b // 2, w.b - 1):
+                want = so.sparse_attention_block(Qh, Kg, Vg, i, ci[rp[i]:rp[i + 1]], w.B)
+                compare_attention(og[hh, i * w.B:min(w.n, (i + 1) * w.B)], want)

@@ -287,6 +287,80 @@ def pin_decode():
     assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
 
 
+def pin_group_shared_log_rows():
+    """The decode group score is log(sum_h exp(rho_h)): scipy's logsumexp on
+    rows far below exp's range, and shift invariance."""
+    from scipy.special import logsumexp
+    rho = rng.uniform(-1500.0, -900.0, size=(4, 37))
+    got = so.group_shared_log_rows(rho)
+    assert np.all(np.isfinite(got))
+    assert np.allclose(got, logsumexp(rho, axis=0), rtol=1e-13, atol=0)
+    assert np.allclose(so.group_shared_log_rows(rho + 3.5), got + 3.5, rtol=1e-13, atol=0)
+    one = rng.standard_normal((1, 9))
+    assert np.array_equal(so.group_shared_log_rows(one), one[0])
+
+
+def _shared_case(hq, hkv, same_heads=False, perm=None):
+    d, B, n = 8, 4, 29
+    r = np.random.default_rng(77)
+    Q = r.standard_normal((hq, n, d))
+    if same_heads:
+        Q[:] = Q[0]
+    if perm is not None:
+        Q = Q[perm]
+    K, V = r.standard_normal((hkv, n, d)), r.standard_normal((hkv, n, d))
+    Hd = so.srht_matrix(d, 4, 3)
+    return Q, K, V, Hd, B
+
+
+def pin_group_shared_prefill():
+    """Group-shared prefill selection: with one head per group it is the
+    per-head choice; with identical heads it is each head's own choice; it
+    does not depend on the order of the group's heads; every head of a group
+    gets the same CSR rows."""
+    for hq, hkv in ((2, 2), (4, 2)):
+        Q, K, V, Hd, B = _shared_case(hq, hkv, same_heads=(hq != hkv))
+        for layers in (1, 2):
+            sp, ss = so.PrefillState(), so.PrefillState()
+            for _ in range(layers):
+                per = so.prefill_layer(Q, K, V, Hd, B, 2, (2, 5), sp, attention_blocks=None)
+                sh = so.prefill_layer(Q, K, V, Hd, B, 2, (2, 5), ss, attention_blocks=None, select="group_shared")
+            for h in range(hq):
+                assert np.array_equal(per[h]["col_idx"], sh[h]["col_idx"])
+                assert np.array_equal(per[h]["row_ptr"], sh[h]["row_ptr"])
+    Q, K, V, Hd, B = _shared_case(4, 2)
+    a = so.prefill_layer(Q, K, V, Hd, B, 2, (2, 5), so.PrefillState(), attention_blocks=None, select="group_shared")
+    Qp = Q[[1, 0, 3, 2]]
+    b = so.prefill_layer(Qp, K, V, Hd, B, 2, (2, 5), so.PrefillState(), attention_blocks=None, select="group_shared")
+    for h in range(4):
+        assert np.array_equal(a[h]["col_idx"], b[h]["col_idx"])
+        assert np.array_equal(a[h]["col_idx"], a[(h // 2) * 2]["col_idx"])
+    per = so.prefill_layer(Q, K, V, Hd, B, 2, (2, 5), so.PrefillState(), attention_blocks=None)
+    assert any(not np.array_equal(per[h]["col_idx"], a[h]["col_idx"]) for h in range(4))  # the choice is shared
+
+
+def pin_group_shared_decode():
+    """Group-shared decode selection: per-head choice when a group has one
+    head or identical heads, independent of head order, one set per group."""
+    d, B, L = 8, 4, 37
+    r = np.random.default_rng(5)
+    Kc = r.standard_normal((2, 40, d))
+    Hd = so.srht_matrix(d, 4, 2)
+    q = r.standard_normal((2, d))
+    _, _, per = so.decode_layer_select(q, Kc, L, Hd, B, 8, (1, 3), None)
+    _, _, sh = so.decode_layer_select(q, Kc, L, Hd, B, 8, (1, 3), None, select="group_shared")
+    assert all(np.array_equal(x, y) for x, y in zip(per, sh))
+    q4 = np.repeat(q[:1], 4, axis=0)
+    _, _, per = so.decode_layer_select(q4, Kc[:1], L, Hd, B, 8, (1, 3), None)
+    _, _, sh = so.decode_layer_select(q4, Kc[:1], L, Hd, B, 8, (1, 3), None, select="group_shared")
+    assert all(np.array_equal(x, y) for x, y in zip(per, sh))
+    q4 = r.standard_normal((4, d))
+    rho, _, a = so.decode_layer_select(q4, Kc, L, Hd, B, 8, (1, 3), None, select="group_shared")
+    _, _, b = so.decode_layer_select(q4[[1, 0, 3, 2]], Kc, L, Hd, B, 8, (1, 3), None, select="group_shared")
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    assert np.array_equal(a[0], a[1]) and np.array_equal(a[2], a[3])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -322,6 +396,10 @@ PLANTED = {
             Q[i * B:(i + 1) * B] @ K[u].T / math.sqrt(Q.shape[1])))(
             np.concatenate([np.arange(j * B, min(len(Q), (j + 1) * B)) for j in blocks]))),
         pin_attention_dense_limit),
+    "group_shared_first_head_only": ("group_shared_walk_rows", lambda orig: (lambda R_heads: orig(R_heads[:1])),
+                                     pin_group_shared_prefill),
+    "group_shared_lse_without_shift": ("group_shared_log_rows", lambda orig: (
+        lambda rho: np.log(np.exp(rho).sum(axis=0))), pin_group_shared_log_rows),
     "attention_scale_1_over_d": ("sparse_attention_block", lambda orig: (
         lambda Q, K, V, i, blocks, B: orig(np.asarray(Q) / math.sqrt(Q.shape[1]), K, V, i, blocks, B)),
         pin_attention_dense_limit),
