@@ -440,7 +440,7 @@ def bench_decode(args, world, S, W, torch, peaks):
     warm = min(args.warmup, wd.steps - 1)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * wd.layers + 1)] for _ in range(wd.steps)]
 
-    def step(t, rec):
+    def step(t, rec, h=h):
         path.begin_step()
         if rec:
             ev[t][0].record(stream)
@@ -503,6 +503,28 @@ def bench_decode(args, world, S, W, torch, peaks):
                      "frac": attn_bytes / (attn_launch_ms * 1e-3) / 1e9 / hbm,
                      "traffic": profiled_traffic("decode_attn_b16_n131072", "k_decode.cu")},
     }
+    if not args.no_variants:
+        # the group-shared selection variant on the same caches and tokens: the
+        # caches are rebuilt to the prompt and the same steps replayed
+        hs = S.Handle(S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed, select_group=wd.hq // wd.hkv))
+        path.init_cache(torch.full((wd.batch,), wd.n0, dtype=torch.int32, device="cuda"))
+        for t in range(warm):
+            step(t, False, hs)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for t in range(warm, wd.steps):
+            step(t, False, hs)
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(hs) == 0
+        sh_ms = max_over_ranks(a.elapsed_time(b), world) / timed
+        us = union_log[warm:].double()
+        sh_kv = float(us.sum().item()) * wd.B * wd.d * 2 * 2 / timed
+        out["variants"] = {"group_shared_selection": {
+            "step_us": sh_ms * 1e3, "kv_bytes_per_step": sh_kv, "union_blocks_per_unit": float(us.mean().item()),
+            "hbm_gbs": (sh_kv + sk_bytes + tok_bytes) / (sh_ms * 1e-3) / 1e9}}
+        hs.close()
     h.close()
     return out
 

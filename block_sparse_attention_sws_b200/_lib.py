@@ -36,7 +36,7 @@ class SwsConfig(ctypes.Structure):
     _fields_ = [
         ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("sketch_dim", ctypes.c_int32),
         ("walk_power", ctypes.c_int32), ("walk_mode", ctypes.c_int32), ("density_num", ctypes.c_int32),
-        ("density_den", ctypes.c_int32), ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("density_den", ctypes.c_int32), ("select_group", ctypes.c_int32), ("seed", ctypes.c_uint64),
     ]
 
 
@@ -98,8 +98,9 @@ def _check(s: int, where: str) -> None:
 
 
 def make_config(head_dim=128, block_size=64, sketch_dim=32, walk_power=8, walk_mode=SWS_WALK_MATRIX_POWER,
-                density=(1, 5), seed=0) -> SwsConfig:
-    return SwsConfig(head_dim, block_size, sketch_dim, walk_power, walk_mode, density[0], density[1], 0, seed)
+                density=(1, 5), seed=0, select_group=0) -> SwsConfig:
+    return SwsConfig(head_dim, block_size, sketch_dim, walk_power, walk_mode, density[0], density[1], select_group,
+                     seed)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

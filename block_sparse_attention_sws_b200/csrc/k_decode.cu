@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     double* __restrict__ k_psum, double* __restrict__ k_sketch, int first_layer, double* __restrict__ walk_state,
     int32_t* __restrict__ head_sel, int32_t* __restrict__ head_cnt, int32_t* __restrict__ sel,
     uint8_t* __restrict__ sel_mask, int32_t* __restrict__ sel_cnt, const double* __restrict__ hdt, int32_t k,
-    int32_t B, int32_t s_pow, int32_t num, int32_t den, int32_t* err) {
+    int32_t B, int32_t s_pow, int32_t num, int32_t den, int shared, int32_t* err) {
   const int group = hq / hkv;
   extern __shared__ __align__(16) uint8_t smem[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                       // [group][max_blocks] (z, then keys)
@@ -299,14 +299,36 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     for (int j = t; j < nb; j += nthr) {
       const double val = (first_layer ? 0.0 : rho[j]) + s_pow * (zr[j] - lse);
       rho[j] = val;
-      kr[j] = order_key(val);
+      if (shared) zr[j] = val;  // kept for the group's log-sum-exp below
+      else kr[j] = order_key(val);
     }
     named_bar(bar_id, nthr);
-    group_top_tau(kr, nb, tau, hist + r * 256, ctl + r * 4, t, nthr, bar_id,
-                  head_sel + ((int64_t)bi * hq + h) * max_blocks, mark, 1u << r, err);
-    if (t == 0) head_cnt[(int64_t)bi * hq + h] = tau;
+    if (!shared) {
+      group_top_tau(kr, nb, tau, hist + r * 256, ctl + r * 4, t, nthr, bar_id,
+                    head_sel + ((int64_t)bi * hq + h) * max_blocks, mark, 1u << r, err);
+      if (t == 0) head_cnt[(int64_t)bi * hq + h] = tau;
+    }
   }
   __syncthreads();
+  if (shared) {
+    // one selection for the whole group: the top-tau of log(sum_h exp(rho_h)),
+    // by every warp of the CTA; the other heads copy the first head's list
+    for (int j = tid; j < nb; j += kSelThreads) {
+      double m = z[j];
+      for (int q = 1; q < group; ++q) m = fmax(m, z[q * max_blocks + j]);
+      double se = 0.0;
+      for (int q = 0; q < group; ++q) se += exp(z[q * max_blocks + j] - m);
+      keys[j] = order_key(m + log(se));
+    }
+    __syncthreads();
+    int32_t* sel0 = head_sel + ((int64_t)bi * hq + (int64_t)g * group) * max_blocks;
+    group_top_tau(keys, nb, tau, hist, ctl, tid, kSelThreads, 1, sel0, mark, (1u << group) - 1u, err);
+    __syncthreads();
+    for (int q = 1; q < group; ++q)
+      for (int x = tid; x < tau; x += kSelThreads) sel0[(int64_t)q * max_blocks + x] = sel0[x];
+    if (tid < group) head_cnt[(int64_t)bi * hq + g * group + tid] = tau;
+    __syncthreads();
+  }
 
   // 4. ordered compaction of the union
   int base = 0;
@@ -667,7 +689,7 @@ cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok
   kern<<<static_cast<unsigned>((int64_t)batch * hkv), kSelThreads, smem, st>>>(
       q_tok, k_tok, v_tok, hq, hkv, max_len, mb, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
       walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, h->hdt, c.sketch_dim, c.block_size, c.walk_power,
-      c.density_num, c.density_den, h->err);
+      c.density_num, c.density_den, (c.select_group > 1 && hq / hkv > 1) ? 1 : 0, h->err);
   note_launches(1);
   return cudaGetLastError();
 }

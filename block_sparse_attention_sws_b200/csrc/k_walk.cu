@@ -194,8 +194,11 @@ __global__ void __launch_bounds__(kGemmThreads, 8) tri_gemm_kernel(const double*
 
 // One warp per row: copies R's row to the walk state (zeros above the
 // diagonal), writes row_ptr, and emits the row's top-tau blocks ascending.
+// With G > 1 query heads sharing a selection, a warp takes one row of a
+// group: it copies the G heads' rows, selects on their sum (added in head
+// order) and writes the same blocks to the CSR row of every head.
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ R, int64_t b, int64_t rows,
-                                                     int32_t num, int32_t den, int64_t nnz,
+                                                     int32_t G, int32_t num, int32_t den, int64_t nnz,
                                                      double* __restrict__ walk_state, int32_t* __restrict__ row_ptr,
                                                      int32_t* __restrict__ col_idx, int32_t* err) {
   extern __shared__ __align__(16) uint64_t keys_all[];
@@ -204,13 +207,17 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   if (row >= rows) return;
   uint64_t* keys = keys_all + (size_t)warp * b;
   int* hist = reinterpret_cast<int*>(keys_all + (size_t)(blockDim.x >> 5) * b) + warp * 256;
-  const int64_t h = row / b, i = row % b;
-  const double* r = R + row * b;
-  double* ws = walk_state + row * b;
+  const int64_t grp = row / b, i = row % b;
+  const int64_t h0 = grp * G;  // first head of the row's group
   for (int64_t j = lane; j < b; j += 32) {
-    const double x = (j <= i) ? r[j] : 0.0;
-    ws[j] = x;
-    if (j <= i) keys[j] = order_key(x);
+    double sum = 0.0;
+    for (int q = 0; q < G; ++q) {
+      const int64_t off = ((h0 + q) * b + i) * b + j;
+      const double x = (j <= i) ? R[off] : 0.0;
+      walk_state[off] = x;
+      sum = q == 0 ? x : sum + x;
+    }
+    if (j <= i) keys[j] = order_key(sum);
   }
   int64_t rp = 0;
   for (int64_t q = lane; q < i; q += 32) rp += tau_of_row(q, num, den);
@@ -218,11 +225,17 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   for (int off = 16; off > 0; off >>= 1) rp += __shfl_xor_sync(0xffffffffu, rp, off);
   const int tau = tau_of_row(i, num, den);
   if (lane == 0) {
-    row_ptr[h * (b + 1) + i] = static_cast<int32_t>(rp);
-    if (i == b - 1) row_ptr[h * (b + 1) + b] = static_cast<int32_t>(rp + tau);
+    for (int q = 0; q < G; ++q) {
+      row_ptr[(h0 + q) * (b + 1) + i] = static_cast<int32_t>(rp);
+      if (i == b - 1) row_ptr[(h0 + q) * (b + 1) + b] = static_cast<int32_t>(rp + tau);
+    }
   }
   __syncwarp();
-  warp_top_tau8(keys, static_cast<int>(i + 1), tau, col_idx + h * nnz + rp, hist, err);
+  int32_t* out0 = col_idx + h0 * nnz + rp;
+  warp_top_tau8(keys, static_cast<int>(i + 1), tau, out0, hist, err);
+  __syncwarp();  // the first head's row is written: the others copy it
+  for (int q = 1; q < G; ++q)
+    for (int t = lane; t < tau; t += 32) col_idx[(h0 + q) * nnz + rp + t] = out0[t];
 }
 
 }  // namespace
@@ -249,7 +262,8 @@ cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_
 
 cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32_t hq, double* walk_state,
                           int32_t* row_ptr, int32_t* col_idx, cudaStream_t st) {
-  const int64_t rows = (int64_t)hq * b;
+  const int32_t G = h->cfg.select_group > 1 ? h->cfg.select_group : 1;
+  const int64_t rows = (int64_t)(hq / G) * b;
   int warps = static_cast<int>(std::min<int64_t>(8, std::max<int64_t>(1, (160 << 10) / (b * 8))));
   const size_t smem = (size_t)warps * (b * sizeof(uint64_t) + 256 * sizeof(int));
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -257,7 +271,7 @@ cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32
   int64_t nnz = 0;
   for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
   select_kernel<<<static_cast<unsigned>(ceil_div64(rows, warps)), warps * 32, smem, st>>>(
-      R, b, rows, h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
+      R, b, rows, G, h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -83,7 +83,7 @@ const char* sws_status_string(sws_status s) {
 
 sws_status sws_config_check(const sws_config* c) {
   if (!c) return SWS_ERR_INVALID_ARG;
-  if (c->reserved != 0) return SWS_ERR_INVALID_ARG;
+  if (c->select_group < 0 || c->select_group > 8) return SWS_ERR_INVALID_ARG;
   if (c->head_dim != 64 && c->head_dim != 128) return SWS_ERR_UNSUPPORTED;
   if (c->block_size != 64 && c->block_size != 128) return SWS_ERR_UNSUPPORTED;
   if (c->sketch_dim < 1 || c->sketch_dim > c->head_dim) return SWS_ERR_INVALID_ARG;
@@ -267,6 +267,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
                            double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
                            void* stream) {
   if (!h || n < 1 || hq < 1) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.select_group > 1 && hq % h->cfg.select_group != 0) return SWS_ERR_INVALID_ARG;
   if (!aligned16(scores) || !aligned16(walk_state) || !aligned16(row_ptr) || !aligned16(col_idx) || !aligned16(ws))
     return SWS_ERR_INVALID_ARG;
   const int64_t b = ceil_div64(n, h->cfg.block_size);
@@ -369,6 +370,7 @@ sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k
                            uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
   if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (hq / hkv > 8) return SWS_ERR_UNSUPPORTED;
+  if (h->cfg.select_group > 1 && h->cfg.select_group != hq / hkv) return SWS_ERR_INVALID_ARG;
   const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch,
                         walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
   for (const void* p : ptrs)

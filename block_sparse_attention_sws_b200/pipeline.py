@@ -43,7 +43,7 @@ class PrefillPath:
         self.h_dense = None
         if dense_layers > 0:
             self.h_dense = L.Handle(L.make_config(cfg.head_dim, cfg.block_size, cfg.sketch_dim, cfg.walk_power,
-                                                  cfg.walk_mode, (1, 1), cfg.seed))
+                                                  cfg.walk_mode, (1, 1), cfg.seed, cfg.select_group))
             nnz_dense = L.sws_csr_nnz(self.h_dense.cfg, n)
             self.row_ptr_dense = torch.empty(hq, self.b + 1, dtype=torch.int32, device=device)
             self.col_idx_dense = torch.empty(hq, nnz_dense, dtype=torch.int32, device=device)

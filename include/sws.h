@@ -64,7 +64,11 @@ typedef struct {
   int32_t walk_mode;   /* sws_walk_mode */
   int32_t density_num; /* 0 < num <= den; 1/5 = the page's 20% density */
   int32_t density_den;
-  int32_t reserved;    /* must be 0 */
+  int32_t select_group; /* query heads that share one selection: 0 or 1 = each head its own (the
+                        * page's method); G > 1 = the G consecutive query heads of a GQA group
+                        * share the top-tau of their summed walk rows (prefill) or of the
+                        * log-sum-exp of their log-domain walk rows (decode). An extension the
+                        * page does not define. Prefill needs G | hq; decode needs G = hq/hkv. */
   uint64_t seed;       /* seeds the random signs and columns of H_d */
 } sws_config;
 

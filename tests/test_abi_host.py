@@ -57,7 +57,7 @@ def test_status_strings(lib):
     ("sketch_dim", 129, S.SWS_ERR_INVALID_ARG), ("walk_power", 0, S.SWS_ERR_INVALID_ARG),
     ("walk_power", 65, S.SWS_ERR_INVALID_ARG), ("walk_mode", 2, S.SWS_ERR_INVALID_ARG),
     ("density_num", 0, S.SWS_ERR_INVALID_ARG), ("density_num", 6, S.SWS_ERR_INVALID_ARG),
-    ("reserved", 1, S.SWS_ERR_INVALID_ARG),
+    ("select_group", 9, S.SWS_ERR_INVALID_ARG), ("select_group", -1, S.SWS_ERR_INVALID_ARG),
 ])
 def test_config_rejections(lib, field, value, want):
     cfg = S.make_config()

@@ -20,10 +20,10 @@ from parity import compare_attention, compare_selection
 pytestmark = pytest.mark.gpu
 
 
-def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None):
+def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
     dev = "cuda"
     batch = len(n0s)
-    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed, select_group=(w.hq // w.hkv) if shared else 0)
     h = S.Handle(cfg)
     max_len = max(n0s) + steps
     path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev)
@@ -67,7 +67,8 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None):
                 nb = -(-length // w.B)
                 Kh, Vh = host[(s_, layer)]
                 q = Qs[(s_, layer)][:, t].double().cpu().numpy()
-                rho, z, osel = so.decode_layer_select(q, Kh, length, Hd, w.B, w.s, w.density, rho_prev[s_])
+                rho, z, osel = so.decode_layer_select(q, Kh, length, Hd, w.B, w.s, w.density, rho_prev[s_],
+                                                      select="group_shared" if shared else "per_head")
                 rho_prev[s_] = rho
                 assert np.allclose(rho_gpu[s_, :, :nb], rho, rtol=1e-9, atol=1e-9 * np.abs(rho).max())
                 union = {}
@@ -76,7 +77,9 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None):
                     gsel = hs[s_, hh, :tau]
                     assert tau == so.tau_of_row(nb - 1, *w.density)
                     assert np.all(np.diff(gsel) > 0) and gsel.max() < nb
-                    swaps += [(t, layer, s_, hh) + x for x in compare_selection(gsel, osel[hh], rho[hh],
+                    g0 = (hh // group) * group
+                    score = so.group_shared_log_rows(rho[g0:g0 + group]) if shared else rho[hh]
+                    swaps += [(t, layer, s_, hh) + x for x in compare_selection(gsel, osel[hh], score,
                                                                                  log_domain=True)]
                     for j in gsel:
                         union[int(j)] = union.get(int(j), 0) | (1 << (hh % group))
@@ -151,3 +154,13 @@ def test_decode_bad_length_guard():
                       path.k_sketch[0], True, path.walk_state, path.head_sel, path.head_cnt, path.sel, path.sel_mask,
                       path.sel_cnt)
     assert S.sws_sync_check(h) == 4  # GUARD_BAD_LEN
+
+
+def test_decode_group_shared_selection():
+    """Group-shared selection: the group's heads get one set of blocks (the
+    top-tau of the log-sum-exp of their rho rows), the union is that set with
+    every head's bit, and attention matches the oracle on it."""
+    w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
+    swaps = run_decode(w, [1000, 1500, 638], steps=4, shared=True)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)

@@ -20,9 +20,11 @@ pytestmark = pytest.mark.gpu
 MODES = {S.SWS_WALK_MATRIX_POWER: "matrix_power", S.SWS_WALK_ELEMENTWISE: "elementwise"}
 
 
-def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATRIX_POWER, report=None):
+def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATRIX_POWER, report=None,
+             shared=False):
     dev = "cuda"
-    cfg = S.make_config(w.d, w.B, w.k, w.s, mode, w.density, w.seed)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, mode, w.density, w.seed,
+                        select_group=(w.hq // w.hkv) if shared else 0)
     h = S.Handle(cfg)
     dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
     path = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, dev)
@@ -37,7 +39,8 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
         torch.cuda.synchronize()
         assert S.sws_sync_check(h) == 0
         ref = so.prefill_layer(LazyHeads(Q), LazyHeads(K), LazyHeads(V), Hd, w.B, w.s, w.density, st, heads=heads,
-                               attention_blocks=None, mode=MODES[mode])
+                               attention_blocks=None, mode=MODES[mode],
+                               select="group_shared" if shared else "per_head")
         rp_all = path.row_ptr.cpu().numpy()
         ci_all = path.col_idx.cpu().numpy()
         for hh in heads:
@@ -51,7 +54,8 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
             compare_walk(path.walk_state[hh].cpu().numpy(), r["R"])
             rp, ci = rp_all[hh], ci_all[hh]
             check_csr_valid(rp, ci, w.b, *w.density)
-            swaps += [(layer, hh) + s for s in compare_csr(rp, ci, r["row_ptr"], r["col_idx"], r["R"])]
+            swaps += [(layer, hh) + s for s in compare_csr(rp, ci, r["row_ptr"], r["col_idx"],
+                                                          r["shared_scores"] if shared else r["R"])]
             qb = range(w.b) if blocks is None else [i for i in blocks if 0 <= i < w.b]
             Qh, Kg, Vg = LazyHeads(Q)[hh], LazyHeads(K)[g], LazyHeads(V)[g]
             o_gpu = path.o[hh].float().cpu().numpy()
@@ -229,3 +233,15 @@ def test_dense_first_layers_policy():
             for i in (0, w.b // 2, w.b - 1):
                 want = so.sparse_attention_block(Qh, Kg, Vg, i, ci[rp[i]:rp[i + 1]], w.B)
                 compare_attention(og[hh, i * w.B:min(w.n, (i + 1) * w.B)], want)
+
+
+@pytest.mark.parametrize("w", [
+    W.PREFILL_16K.scaled(name="shared_p16k", hq=8, hkv=2, n=2000, layers=3),
+    W.PREFILL_64K.scaled(name="shared_p64k", hq=4, hkv=1, n=4200, layers=2),
+], ids=lambda w: w.name)
+def test_group_shared_selection(w):
+    """Group-shared selection: every head of a GQA group gets the top-tau of
+    the sum of the group's walk rows; the walk state stays per head."""
+    swaps = run_case(w, shared=True)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
