@@ -82,16 +82,30 @@ __global__ void __launch_bounds__(256) block_softmax_wide_kernel(const double* _
 }
 
 // C = A * Bm for lower-triangular b x b matrices on the fp64 tensor path
-// (mma.sync m16n8k4 f64). One 32 x 32 output tile per CTA of two warps (on or
-// below the diagonal, heaviest first; many small CTAs keep every SM busy and
-// waste less of the triangle than large tiles), each warp a 16 x 32 slice;
-// k staged 16 at a time through padded shared memory (row strides of 20 and
-// 36 doubles make the fragment loads conflict-free) with the next chunk
-// prefetched into registers. Entries above the diagonal of A and Bm are
-// treated as zero whatever the buffers hold.
-constexpr int kTT = 32, kTK = 16, kGemmThreads = 64;
-constexpr int kApad = kTK + 4;   // A tile row stride (doubles)
-constexpr int kBpad = kTT + 4;   // B tile row stride (doubles)
+// (mma.sync m16n8k4 f64). On this part each SM sub-partition completes one
+// such product about every 32 cycles, and one warp with one accumulator chain
+// already keeps it busy, so what matters is that every sub-partition always
+// has a product to issue and that the loads feeding it stay cheap.
+//
+// One 32 x 32 output tile (on or below the diagonal) per CTA of four warps.
+// The tile's k range, key blocks J..I of the walk, is cut into chunks of 8
+// and warp w takes chunks w, w+4, ...: a long tile and a short one alike keep
+// all four sub-partitions of their SM equally busy. Each warp reads its
+// fragments from L2 straight into registers (every operand element is used by
+// exactly one warp, so shared-memory staging would only add traffic), with the
+// next chunk's loads in flight while the current chunk's sixteen products
+// issue. The loads are 16 bytes wide: a lane takes two neighbouring k of an A
+// row and two neighbouring columns of a Bm row, and the k order inside a chunk
+// and the column order inside the tile are permuted to match (a sum over k
+// does not care about its order up to rounding; the columns are put back when
+// the tile is written). The four partial tiles are summed in warp order
+// through shared memory, so the result does not depend on scheduling. Tiles
+// go out heaviest first across all heads. Entries above the diagonal of A and
+// Bm are treated as zero whatever the buffers hold. An odd b (rows not 16-byte
+// aligned) and the tiles of the last tile row of a ragged b take a checked
+// path with 8-byte loads.
+constexpr int kTT = 32, kGemmWarps = 4, kGemmThreads = 32 * kGemmWarps;
+constexpr int kPartLd = kTT + 2;  // partial-tile row stride (doubles): 16-B rows, spread banks
 
 __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int64_t& tj) {
   // heaviest tiles (largest ti - tj) first
@@ -104,90 +118,162 @@ __device__ __forceinline__ void tile_of(int64_t t, int64_t nt, int64_t& ti, int6
 }
 
 __device__ __forceinline__ void dmma_16x8x4(double (&c)[4], double a0, double a1, double b0) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
       : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
       : "d"(a0), "d"(a1), "d"(b0));
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 8) tri_gemm_kernel(const double* __restrict__ A,
+// One warp's share of a tile: chunks warp, warp + 4, ... of [j0, kend), chunk
+// c covering k = j0 + 8c .. j0 + 8c + 7. Lane (g, t4) holds, for the chunk's
+// two mma k-steps q = 0, 1, the k = j0 + 8c + 2 t4 + q: A at rows
+// i0 + g + 8m (m = 0..3, the two m16 halves), Bm at columns j0 + 16p + 2g + e
+// (p, e = 0, 1), which form the n8 block n = 2p + e. So the accumulator
+// element v of (h, n) is C[16h + g + 8(v >> 1)][16p + 4 t4 + 2(v & 1) + e].
+template <bool kChecked>
+__device__ __forceinline__ void tile_products(const double* __restrict__ Ah, const double* __restrict__ Bh, int64_t b,
+                                              int64_t i0, int64_t j0, int64_t kend, int warp, int lane,
+                                              double (&acc)[2][4][4]) {
+  const int g = lane >> 2, t4 = lane & 3;
+  const int nchunks = static_cast<int>((kend - j0 + 7) >> 3);
+  // coordinates relative to j0 (all fit in 32 bits: b <= 8192)
+  const int di = static_cast<int>(i0 - j0), rb = static_cast<int>(b - j0), re = static_cast<int>(kend - j0);
+  const double* pa = Ah + (i0 + g) * b + j0 + 2 * t4;    // row i0 + g, column j0 + 2 t4
+  const double* pb = Bh + (j0 + 2 * t4) * b + j0 + 2 * g;  // row j0 + 2 t4, column j0 + 2g
+  double2 fa[2][4], fb[2][4];  // fb[.][2q + p]
+  // raw loads; the masks are applied where the products use the values, so
+  // that nothing waits on a load before the previous chunk's products issue
+  auto load = [&](int c, double2(&xa)[4], double2(&xb)[4]) {
+    const double* a = pa + 8 * c;
+    const double* bp = pb + (int64_t)(8 * c) * b;
+    const int kr = 8 * c + 2 * t4;  // k - j0 of q = 0
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const double* src = a + (int64_t)(8 * m) * b;
+      if (!kChecked) {
+        xa[m] = __ldg(reinterpret_cast<const double2*>(src));
+      } else {
+        const bool row_ok = di + g + 8 * m < rb;
+        xa[m].x = (row_ok && kr < re) ? __ldg(src) : 0.0;
+        xa[m].y = (row_ok && kr + 1 < re) ? __ldg(src + 1) : 0.0;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const double* src = bp + q * b + 16 * p;
+        if (!kChecked) {
+          xb[2 * q + p] = __ldg(reinterpret_cast<const double2*>(src));
+        } else {
+          const bool k_ok = kr + q < re;
+          const int cr = 16 * p + 2 * g;  // column - j0
+          xb[2 * q + p].x = (k_ok && cr < rb) ? __ldg(src) : 0.0;
+          xb[2 * q + p].y = (k_ok && cr + 1 < rb) ? __ldg(src + 1) : 0.0;
+        }
+      }
+  };
+  auto mma = [&](int c, const double2(&xa)[4], const double2(&xb)[4]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int kr = 8 * c + 2 * t4 + q;
+      double ma[4], mb[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const double x = q ? xa[m].y : xa[m].x;
+        ma[m] = kr <= di + g + 8 * m ? x : 0.0;  // A above its diagonal
+      }
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const double x = e ? xb[2 * q + p].y : xb[2 * q + p].x;
+          mb[2 * p + e] = 16 * p + 2 * g + e <= kr ? x : 0.0;  // Bm above its diagonal
+        }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) dmma_16x8x4(acc[h][n], ma[2 * h], ma[2 * h + 1], mb[n]);
+    }
+  };
+  int c = warp;
+  if (c >= nchunks) return;
+  load(c, fa[0], fb[0]);
+  // two chunks per trip, the loads of the next one in flight under the products of this one
+  while (true) {
+    const bool more1 = c + kGemmWarps < nchunks;
+    if (more1) load(c + kGemmWarps, fa[1], fb[1]);
+    mma(c, fa[0], fb[0]);
+    if (!more1) break;
+    c += kGemmWarps;
+    const bool more0 = c + kGemmWarps < nchunks;
+    if (more0) load(c + kGemmWarps, fa[0], fb[0]);
+    mma(c, fa[1], fb[1]);
+    if (!more0) break;
+    c += kGemmWarps;
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 3) tri_gemm_kernel(const double* __restrict__ A,
                                                                 const double* __restrict__ Bm,
-                                                                double* __restrict__ C, int64_t b) {
-  constexpr int PER = kTT * kTK / kGemmThreads;  // 8 elements of each operand chunk per thread
-  __shared__ __align__(16) double As[2][kTT][kApad];
-  __shared__ __align__(16) double Bs[2][kTK][kBpad];
+                                                                double* __restrict__ C, int64_t b, int32_t hq) {
+  __shared__ __align__(16) double part[kGemmWarps][kTT][kPartLd];
   const int64_t nt = ceil_div64(b, kTT);
+  const int64_t head = blockIdx.x % hq;  // tile-major: every head's heaviest tile first
   int64_t ti, tj;
-  tile_of(blockIdx.x, nt, ti, tj);
-  const size_t hoff = (size_t)blockIdx.y * b * b;
-  const double* Ah = A + hoff;
-  const double* Bh = Bm + hoff;
-  double* Ch = C + hoff;
+  tile_of(blockIdx.x / hq, nt, ti, tj);
+  const size_t hoff = (size_t)head * b * b;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
   const int64_t i0 = ti * kTT, j0 = tj * kTT;
-  const int64_t kbeg = j0, kend = std::min<int64_t>(b, i0 + kTT);
+  const int64_t kend = std::min<int64_t>(b, i0 + kTT);
+  const bool pairs = (b & 1) == 0;  // 16-B aligned row starts
 
-  double ra[PER], rb[PER];
-  auto load = [&](int64_t k0) {
+  double acc[2][4][4];
 #pragma unroll
-    for (int q = 0; q < PER; ++q) {
-      const int e = tid + q * kGemmThreads;
-      // A: element (row e / KC, k e % KC): 16 consecutive threads read one row
-      const int64_t ar = i0 + e / kTK, ak = k0 + e % kTK;
-      ra[q] = (ar < b && ak < kend && ak <= ar) ? Ah[ar * b + ak] : 0.0;
-      // B: element (k e / T, column e % T): a warp reads one row
-      const int64_t bk = k0 + e / kTT, bc = j0 + e % kTT;
-      rb[q] = (bk < kend && bc < b && bc <= bk) ? Bh[bk * b + bc] : 0.0;
-    }
-  };
-  auto store = [&](int buf) {
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int q = 0; q < PER; ++q) {
-      const int e = tid + q * kGemmThreads;
-      As[buf][e / kTK][e % kTK] = ra[q];
-      Bs[buf][e / kTT][e % kTT] = rb[q];
-    }
-  };
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[h][n][v] = 0.0;
+  if (i0 + kTT <= b && pairs)
+    tile_products<false>(A + hoff, Bm + hoff, b, i0, j0, kend, warp, lane, acc);
+  else
+    tile_products<true>(A + hoff, Bm + hoff, b, i0, j0, kend, warp, lane, acc);
 
-  double acc[4][4];
+  // accumulator element v of (h, n = 2p + e): row 16h + g + 8(v >> 1),
+  // column 16p + 4 t4 + 2(v & 1) + e; a lane's four columns of one row are contiguous
 #pragma unroll
-  for (int n8 = 0; n8 < 4; ++n8)
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc[n8][v] = 0.0;
-
-  int buf = 0;
-  load(kbeg);
-  store(0);
+    for (int p = 0; p < 2; ++p)
+#pragma unroll
+      for (int hv = 0; hv < 2; ++hv) {
+        double* dst = &part[warp][16 * h + g + 8 * hv][16 * p + 4 * t4];
+        *reinterpret_cast<double2*>(dst) = make_double2(acc[h][2 * p][2 * hv], acc[h][2 * p + 1][2 * hv]);
+        *reinterpret_cast<double2*>(dst + 2) =
+            make_double2(acc[h][2 * p][2 * hv + 1], acc[h][2 * p + 1][2 * hv + 1]);
+      }
   __syncthreads();
-  for (int64_t k0 = kbeg; k0 < kend; k0 += kTK) {
-    const bool more = k0 + kTK < kend;
-    if (more) load(k0 + kTK);
+  double* Ch = C + hoff;
 #pragma unroll
-    for (int ks = 0; ks < kTK / 4; ++ks) {
-      const double a0 = As[buf][warp * 16 + g][ks * 4 + t4];
-      const double a1 = As[buf][warp * 16 + g + 8][ks * 4 + t4];
-      double bf[4];
-#pragma unroll
-      for (int n8 = 0; n8 < 4; ++n8) bf[n8] = Bs[buf][ks * 4 + t4][n8 * 8 + g];
-#pragma unroll
-      for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4(acc[n8], a0, a1, bf[n8]);
-    }
-    if (more) {
-      store(buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int64_t i = i0 + warp * 16 + g + 8 * hh;
+  for (int q = 0; q < kTT * kTT / 2 / kGemmThreads; ++q) {
+    const int e2 = tid + q * kGemmThreads;
+    const int r = e2 >> 4, c = 2 * (e2 & 15);
+    const int64_t i = i0 + r, j = j0 + c;
     if (i >= b) continue;
+    double2 sum = *reinterpret_cast<const double2*>(&part[0][r][c]);
 #pragma unroll
-    for (int n8 = 0; n8 < 4; ++n8) {
-      const int64_t j = j0 + n8 * 8 + 2 * t4;
-      if (j < b) Ch[i * b + j] = acc[n8][2 * hh];
-      if (j + 1 < b) Ch[i * b + j + 1] = acc[n8][2 * hh + 1];
+    for (int w = 1; w < kGemmWarps; ++w) {
+      const double2 pw = *reinterpret_cast<const double2*>(&part[w][r][c]);
+      sum.x += pw.x;
+      sum.y += pw.y;
+    }
+    if (pairs && j + 1 < b) {
+      *reinterpret_cast<double2*>(Ch + i * b + j) = sum;
+    } else {
+      if (j < b) Ch[i * b + j] = sum.x;
+      if (j + 1 < b) Ch[i * b + j + 1] = sum.y;
     }
   }
 }
@@ -244,18 +330,20 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
                                  cudaStream_t st) {
   const int64_t rows = (int64_t)hq * b;
   const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
+  const unsigned grid = static_cast<unsigned>(ceil_div64(rows, 8));
   if (b <= 32 * kSoftmaxPerLane)
-    block_softmax_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
+    block_softmax_kernel<<<grid, 256, 0, st>>>(scores, b, rows, temp, A);
   else
-    block_softmax_wide_kernel<<<static_cast<unsigned>(ceil_div64(rows, 8)), 256, 0, st>>>(scores, b, rows, temp, A);
+    block_softmax_wide_kernel<<<grid, 256, 0, st>>>(scores, b, rows, temp, A);
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st) {
   const int64_t nt = ceil_div64(b, kTT);
-  dim3 grid(static_cast<unsigned>(nt * (nt + 1) / 2), hq);
-  tri_gemm_kernel<<<grid, kGemmThreads, 0, st>>>(A, Bm, C, b);
+  const int64_t ctas = nt * (nt + 1) / 2 * hq;  // one CTA per tile
+  if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+  tri_gemm_kernel<<<static_cast<unsigned>(ctas), kGemmThreads, 0, st>>>(A, Bm, C, b, hq);
   note_launches(1);
   return cudaGetLastError();
 }
