@@ -472,14 +472,25 @@ def bench_decode(args, world, S, W, torch, peaks):
             ev[t][0].record(stream)
         for layer in range(wd.layers):
             L = S
-            L.sws_decode_step(h, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer], path.seq_lens,
-                              path.k_cache[layer], path.v_cache[layer], path.k_psum[layer], path.k_sketch[layer],
-                              layer == 0, path.walk_state, path.head_sel, path.head_cnt, path.sel, path.sel_mask,
-                              path.sel_cnt)
+            if path.paged:
+                L.sws_decode_step_paged(h, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer], path.k_cache[layer],
+                                        path.v_cache[layer], path.block_table, path.seq_lens, path.k_psum[layer],
+                                        path.k_sketch[layer], layer == 0, path.walk_state, path.head_sel,
+                                        path.head_cnt, path.sel, path.sel_mask, path.sel_cnt)
+            else:
+                L.sws_decode_step(h, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer], path.seq_lens,
+                                  path.k_cache[layer], path.v_cache[layer], path.k_psum[layer], path.k_sketch[layer],
+                                  layer == 0, path.walk_state, path.head_sel, path.head_cnt, path.sel, path.sel_mask,
+                                  path.sel_cnt)
             if rec:
                 ev[t][1 + 2 * layer].record(stream)
-            L.sws_sparse_attn_decode(h, toks_q[t, layer], path.k_cache[layer], path.v_cache[layer], path.seq_lens,
-                                     path.sel, path.sel_mask, path.sel_cnt, path.o, path.ws)
+            if path.paged:
+                L.sws_sparse_attn_decode_paged(h, toks_q[t, layer], path.k_cache[layer], path.v_cache[layer],
+                                               path.block_table, path.seq_lens, path.sel, path.sel_mask, path.sel_cnt,
+                                               path.o, path.ws)
+            else:
+                L.sws_sparse_attn_decode(h, toks_q[t, layer], path.k_cache[layer], path.v_cache[layer],
+                                         path.seq_lens, path.sel, path.sel_mask, path.sel_cnt, path.o, path.ws)
             if rec:
                 ev[t][2 + 2 * layer].record(stream)
             union_log[t, layer].copy_(path.sel_cnt, non_blocking=True)
@@ -551,6 +562,28 @@ def bench_decode(args, world, S, W, torch, peaks):
             "step_us": sh_ms * 1e3, "kv_bytes_per_step": sh_kv, "union_blocks_per_unit": float(us.mean().item()),
             "hbm_gbs": (sh_kv + sk_bytes + tok_bytes) / (sh_ms * 1e-3) / 1e9}}
         hs.close()
+        # the paged cache: the same caches moved to a pool whose pages hold the
+        # blocks in a seeded random order, the same steps replayed
+        perm = torch.randperm(wd.batch * path.mb, generator=torch.Generator().manual_seed(wd.seed))
+        path.to_paged(perm.to(torch.int32).reshape(wd.batch, path.mb).cuda(), wd.batch * path.mb)
+        path.init_cache(torch.full((wd.batch,), wd.n0, dtype=torch.int32, device="cuda"))
+        for t in range(warm):
+            step(t, False)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for t in range(warm, wd.steps):
+            step(t, False)
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        pg_ms = max_over_ranks(a.elapsed_time(b), world) / timed
+        up = union_log[warm:].double()
+        pg_kv = float(up.sum().item()) * wd.B * wd.d * 2 * 2 / timed
+        out["variants"]["paged_kv"] = {
+            "step_us": pg_ms * 1e3, "kv_bytes_per_step": pg_kv, "union_blocks_per_unit": float(up.mean().item()),
+            "hbm_gbs": (pg_kv + sk_bytes + tok_bytes) / (pg_ms * 1e-3) / 1e9,
+            "same_selection_as_contiguous": bool(torch.equal(up, u))}
     h.close()
     return out
 

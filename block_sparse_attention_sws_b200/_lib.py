@@ -27,7 +27,8 @@ EXPORTS = [
     "sws_workspace_size", "sws_create", "sws_destroy", "sws_projection_device", "sws_launch_count",
     "sws_sync_check", "sws_sketch",
     "sws_walk_select", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
-    "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc",
+    "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc", "sws_decode_init_cache_paged", "sws_decode_step_paged",
+    "sws_sparse_attn_decode_paged",
 ]
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SWS_NOALLOC_SCRATCH_BYTES
 
@@ -79,6 +80,11 @@ def load() -> ctypes.CDLL:
                                            P, P, P]),
         "sws_sparse_attn_decode": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, SZ, P]),
         "sws_sparse_attn_decode_noalloc": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P]),
+        "sws_decode_init_cache_paged": (ctypes.c_int, [P, P, I64, P, I64, I32, I32, P, P, P, P]),
+        "sws_decode_step_paged": (ctypes.c_int, [P, P, P, P, I32, I32, I32, P, P, I64, P, I64, P, P, P, ctypes.c_int,
+                                                 P, P, P, P, P, P, P]),
+        "sws_sparse_attn_decode_paged": (ctypes.c_int, [P, P, P, P, I64, P, I64, I32, I32, I32, P, P, P, P, P, P, SZ,
+                                                        P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -266,3 +272,39 @@ def sws_sparse_attn_decode_noalloc(h: Handle, q_tok, k_cache, v_cache, seq_lens,
     _check(load().sws_sparse_attn_decode_noalloc(h.ptr, _ptr(q_tok), _ptr(k_cache), _ptr(v_cache), batch, hq, hkv,
                                                  max_len, _ptr(seq_lens), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
                                                  _ptr(o), _stream(stream)), "sws_sparse_attn_decode_noalloc")
+
+
+# ------------------------------------------------------ paged KV cache ----
+
+def sws_decode_init_cache_paged(h: Handle, k_pages, block_table, seq_lens, k_psum, k_sketch, stream=None) -> None:
+    """k_pages [num_pages, hkv, B, d]; block_table [batch, max_blocks] int32."""
+    num_pages, hkv = k_pages.shape[0], k_pages.shape[1]
+    batch, max_blocks = block_table.shape
+    _check(load().sws_decode_init_cache_paged(h.ptr, _ptr(k_pages), num_pages, _ptr(block_table), max_blocks, batch,
+                                              hkv, _ptr(seq_lens), _ptr(k_psum), _ptr(k_sketch), _stream(stream)),
+           "sws_decode_init_cache_paged")
+
+
+def sws_decode_step_paged(h: Handle, q_tok, k_tok, v_tok, k_pages, v_pages, block_table, seq_lens, k_psum, k_sketch,
+                          first_layer: bool, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                          stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    num_pages, hkv = k_pages.shape[0], k_pages.shape[1]
+    max_blocks = block_table.shape[1]
+    _check(load().sws_decode_step_paged(h.ptr, _ptr(q_tok), _ptr(k_tok), _ptr(v_tok), batch, hq, hkv, _ptr(k_pages),
+                                        _ptr(v_pages), num_pages, _ptr(block_table), max_blocks, _ptr(seq_lens),
+                                        _ptr(k_psum), _ptr(k_sketch), int(bool(first_layer)), _ptr(walk_state),
+                                        _ptr(head_sel), _ptr(head_cnt), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
+                                        _stream(stream)), "sws_decode_step_paged")
+
+
+def sws_sparse_attn_decode_paged(h: Handle, q_tok, k_pages, v_pages, block_table, seq_lens, sel, sel_mask, sel_cnt, o,
+                                 ws, stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    num_pages, hkv = k_pages.shape[0], k_pages.shape[1]
+    max_blocks = block_table.shape[1]
+    _check(load().sws_sparse_attn_decode_paged(h.ptr, _ptr(q_tok), _ptr(k_pages), _ptr(v_pages), num_pages,
+                                               _ptr(block_table), max_blocks, batch, hq, hkv, _ptr(seq_lens),
+                                               _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt), _ptr(o), _ptr(ws),
+                                               ws.numel() * ws.element_size(), _stream(stream)),
+           "sws_sparse_attn_decode_paged")

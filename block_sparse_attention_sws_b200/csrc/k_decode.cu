@@ -30,34 +30,38 @@ namespace {
 // ---------------------------------------------------------------- init ------
 // k_sketch for every cached block and k_psum (sum of the last block's keys).
 template <int D>
-__global__ void __launch_bounds__(D) init_cache_kernel(const __nv_bfloat16* __restrict__ kc, int32_t hkv,
-                                                       int64_t max_len, int32_t B, int64_t max_blocks,
+__global__ void __launch_bounds__(D) init_cache_kernel(const __nv_bfloat16* __restrict__ kc, KvLayout kv,
                                                        const int32_t* __restrict__ seq_lens,
                                                        const double* __restrict__ hdt, int32_t k,
                                                        double* __restrict__ k_psum, double* __restrict__ k_sketch,
                                                        int32_t* err) {
   __shared__ double mean[D];
   const int64_t unit = blockIdx.y;  // sequence * hkv + kv head
-  const int bi = static_cast<int>(unit / hkv);
+  const int64_t bi = unit / kv.hkv, g = unit % kv.hkv;
   const int32_t len = seq_lens[bi];
-  if (len < 1 || len > max_len) {
+  if (len < 1 || len > kv.max_len) {
     if (threadIdx.x == 0) record_error(err, GUARD_BAD_LEN);
     return;
   }
-  const int64_t nb = ceil_div64(len, B);
+  const int64_t nb = ceil_div64(len, kv.B);
   const int64_t j = blockIdx.x;
   if (j >= nb) return;
-  const int64_t r0 = j * B, r1 = std::min<int64_t>(len, r0 + B);
-  const __nv_bfloat16* base = kc + unit * max_len * D;
+  const int64_t off = kv_block_offset(kv, bi, g, j);
+  if (off < 0) {
+    if (threadIdx.x == 0) record_error(err, GUARD_BAD_PAGE);
+    return;
+  }
+  const int64_t rows = std::min<int64_t>(len - j * kv.B, kv.B);
+  const __nv_bfloat16* base = kc + off;
   double s = 0.0;
-  for (int64_t r = r0; r < r1; ++r) s += static_cast<double>(__bfloat162float(base[r * D + threadIdx.x]));
+  for (int64_t r = 0; r < rows; ++r) s += static_cast<double>(__bfloat162float(base[r * D + threadIdx.x]));
   if (j == nb - 1) k_psum[unit * D + threadIdx.x] = s;
-  mean[threadIdx.x] = s / static_cast<double>(r1 - r0);
+  mean[threadIdx.x] = s / static_cast<double>(rows);
   __syncthreads();
   for (int c = threadIdx.x; c < k; c += D) {
     double acc = 0.0;
     for (int t = 0; t < D; ++t) acc += mean[t] * hdt[(size_t)c * D + t];
-    k_sketch[(unit * max_blocks + j) * k + c] = acc;
+    k_sketch[(unit * kv.max_blocks + j) * k + c] = acc;
   }
 }
 
@@ -179,12 +183,14 @@ __device__ void group_top_tau(const uint64_t* keys, int m, int tau, int* hist, i
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_tok,
-    const __nv_bfloat16* __restrict__ v_tok, int32_t hq, int32_t hkv, int64_t max_len, int64_t max_blocks,
-    const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache,
-    double* __restrict__ k_psum, double* __restrict__ k_sketch, int first_layer, double* __restrict__ walk_state,
+    const __nv_bfloat16* __restrict__ v_tok, int32_t hq, KvLayout kv, const int32_t* __restrict__ seq_lens,
+    __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, double* __restrict__ k_psum,
+    double* __restrict__ k_sketch, int first_layer, double* __restrict__ walk_state,
     int32_t* __restrict__ head_sel, int32_t* __restrict__ head_cnt, int32_t* __restrict__ sel,
     uint8_t* __restrict__ sel_mask, int32_t* __restrict__ sel_cnt, const double* __restrict__ hdt, int32_t k,
     int32_t B, int32_t s_pow, int32_t num, int32_t den, int shared, int32_t* err) {
+  const int32_t hkv = kv.hkv;
+  const int64_t max_blocks = kv.max_blocks;
   const int group = hq / hkv;
   extern __shared__ __align__(16) uint8_t smem[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem);                       // [group][max_blocks] (z, then keys)
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
   const int64_t unit = blockIdx.x;
   const int bi = static_cast<int>(unit / hkv), g = static_cast<int>(unit % hkv);
   const int32_t len = seq_lens[bi];
-  if (len < 1 || len > max_len) {
+  if (len < 1 || len > kv.max_len) {
     if (tid == 0) record_error(err, GUARD_BAD_LEN);
     return;
   }
@@ -209,14 +215,19 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
   const int64_t blk = pos / B;
   const int cnt = static_cast<int>(pos % B) + 1;
   const int nb = static_cast<int>(blk + 1);
+  const int64_t tok_off = kv_block_offset(kv, bi, g, blk);  // the same for every thread
+  if (tok_off < 0) {
+    if (tid == 0) record_error(err, GUARD_BAD_PAGE);
+    return;
+  }
   for (int j = tid; j < nb; j += kSelThreads) mark[j] = 0u;
 
   // 1. append the token, update the last block's running key sum; stage the
   //    block mean and the group's query rows
   if (tid < D) {
     const __nv_bfloat16 kt = k_tok[unit * D + tid];
-    k_cache[(unit * max_len + pos) * D + tid] = kt;
-    v_cache[(unit * max_len + pos) * D + tid] = v_tok[unit * D + tid];
+    k_cache[tok_off + (pos % B) * D + tid] = kt;
+    v_cache[tok_off + (pos % B) * D + tid] = v_tok[unit * D + tid];
     double ps = (cnt == 1) ? 0.0 : k_psum[unit * D + tid];
     ps += static_cast<double>(__bfloat162float(kt));
     k_psum[unit * D + tid] = ps;
@@ -389,12 +400,14 @@ __device__ __forceinline__ int swz(int u, int d) {
   return u * D + (((d >> 3) ^ (u & (CPR - 1))) << 3) + (d & 7);
 }
 
-template <int D, int BS, int G>
+// kPaged: the cache is a page pool (a block-table lookup per block); otherwise
+// contiguous [batch, hkv, max_len, D].
+template <int D, int BS, int G, bool kPaged>
 __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_cache,
-    const __nv_bfloat16* __restrict__ v_cache, int32_t hkv, int64_t max_len, int64_t max_blocks,
-    const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ sel, const uint8_t* __restrict__ sel_mask,
-    const int32_t* __restrict__ sel_cnt, float* __restrict__ partial, int32_t splits, int32_t* err) {
+    const __nv_bfloat16* __restrict__ v_cache, KvLayout kv, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ sel, const uint8_t* __restrict__ sel_mask, const int32_t* __restrict__ sel_cnt,
+    float* __restrict__ partial, int32_t splits, int32_t* err) {
   static_assert(G >= 1 && G <= 8, "GQA group of 1..8 query heads");
   constexpr int NT_QK = BS / 8 / 4;  // score n-tiles (8 tokens) per warp
   constexpr int NT_PV = D / 8 / 4;   // output n-tiles (8 dims) per warp
@@ -409,12 +422,14 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;
+  const int32_t hkv = kv.hkv;
+  const int64_t max_blocks = kv.max_blocks;
   const int64_t unit = blockIdx.y;
   const int bi = static_cast<int>(unit / hkv);
   const int split = blockIdx.x;
   int32_t len = seq_lens[bi];
   int64_t U = sel_cnt[unit];
-  if (len < 1 || len > max_len || U < 0 || U > ceil_div64(len, BS)) {  // stale or corrupt state: no work
+  if (len < 1 || len > kv.max_len || U < 0 || U > ceil_div64(len, BS)) {  // stale or corrupt state: no work
     if (tid == 0) record_error(err, GUARD_BAD_LEN);
     len = 0;
     U = 0;
@@ -422,8 +437,6 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
   const int64_t lo = U * split / splits, hi = U * (split + 1) / splits;
   const int32_t* blist = sel + unit * max_blocks;
   const uint8_t* mlist = sel_mask + unit * max_blocks;
-  const __nv_bfloat16* kbase = k_cache + unit * max_len * D;
-  const __nv_bfloat16* vbase = v_cache + unit * max_len * D;
 
   // Q fragments (rows = heads of the group, pre-scaled later in fp32)
   uint32_t qa[D / 16][2];
@@ -448,17 +461,43 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
   for (int nt = 0; nt < NT_PV; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
 
   auto block_ok = [&](int64_t j) { return j >= 0 && j * BS < len; };
+  // contiguous: the unit's rows; paged: looked up per block. A row that is
+  // not loaded (src-size 0) still gets an address inside the cache.
+  const __nv_bfloat16* kbase = k_cache + (kPaged ? 0 : unit * kv.max_len * D);
+  const __nv_bfloat16* vbase = v_cache + (kPaged ? 0 : unit * kv.max_len * D);
   auto issue = [&](int64_t idx, int st) {
-    const int64_t j = block_ok(blist[idx]) ? blist[idx] : -1;
+    int64_t j = block_ok(blist[idx]) ? blist[idx] : -1;
+    const __nv_bfloat16* kblk = kbase;
+    const __nv_bfloat16* vblk = vbase;
+    if constexpr (kPaged) {
+      const int64_t off = j < 0 ? -1 : kv_block_offset(kv, bi, unit % hkv, j);
+      if (j >= 0 && off < 0) {
+        if (tid == 0) record_error(err, GUARD_BAD_PAGE);
+        j = -1;
+      }
+      if (j >= 0) {
+        kblk += off;
+        vblk += off;
+      }
+    }
     const int64_t t0 = j < 0 ? (int64_t)len : j * BS;  // an invalid block stages zeros
     __nv_bfloat16* ksm = stage + (st * 2) * TILE;
     __nv_bfloat16* vsm = ksm + TILE;
     for (int x = tid; x < TILE / 8; x += kAttnThreads) {
       const int u = x / (D / 8), c = x % (D / 8);
       const bool valid = t0 + u < len;
-      const int64_t row = valid ? (t0 + u) : 0;
-      cp_async16(ksm + swz<D>(u, c * 8), kbase + row * D + c * 8, valid);
-      cp_async16(vsm + swz<D>(u, c * 8), vbase + row * D + c * 8, valid);
+      const __nv_bfloat16* ks;
+      const __nv_bfloat16* vs;
+      if constexpr (kPaged) {
+        ks = valid ? kblk + u * D : kbase;
+        vs = valid ? vblk + u * D : vbase;
+      } else {
+        const int64_t row = valid ? (t0 + u) : 0;
+        ks = kbase + row * D;
+        vs = vbase + row * D;
+      }
+      cp_async16(ksm + swz<D>(u, c * 8), ks + c * 8, valid);
+      cp_async16(vsm + swz<D>(u, c * 8), vs + c * 8, valid);
     }
   };
 
@@ -606,29 +645,26 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restri
 
 template <int D, int BS, int G>
 cudaError_t launch_attn3(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc, int32_t batch,
-                         int32_t hkv, int64_t max_len, int64_t max_blocks, const int32_t* lens, const int32_t* sel,
-                         const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits, int32_t* err,
-                         cudaStream_t st) {
+                         const KvLayout& kv, const int32_t* lens, const int32_t* sel, const uint8_t* mask,
+                         const int32_t* cnt, float* partial, int32_t splits, int32_t* err, cudaStream_t st) {
   const size_t smem = (size_t)kStages * 2 * BS * D * 2 + 8 * (BS + 4) * 4 + 8 * (BS + 8) * 2 + 8 * 4 + 16 * 4;
-  auto kern = decode_attn_kernel<D, BS, G>;
+  auto kern = kv.block_table ? decode_attn_kernel<D, BS, G, true> : decode_attn_kernel<D, BS, G, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(splits, static_cast<unsigned>((int64_t)batch * hkv));
-  kern<<<grid, kAttnThreads, smem, st>>>(q, kc, vc, hkv, max_len, max_blocks, lens, sel, mask, cnt, partial, splits,
-                                         err);
+  dim3 grid(splits, static_cast<unsigned>((int64_t)batch * kv.hkv));
+  kern<<<grid, kAttnThreads, smem, st>>>(q, kc, vc, kv, lens, sel, mask, cnt, partial, splits, err);
   note_launches(1);
   return cudaGetLastError();
 }
 
 template <int D, int BS>
 cudaError_t launch_attn2(int32_t group, const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vc,
-                         int32_t batch, int32_t hkv, int64_t max_len, int64_t max_blocks, const int32_t* lens,
-                         const int32_t* sel, const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits,
-                         int32_t* err, cudaStream_t st) {
-#define SWS_G(GG)                                                                                                  \
-  case GG:                                                                                                         \
-    return launch_attn3<D, BS, GG>(q, kc, vc, batch, hkv, max_len, max_blocks, lens, sel, mask, cnt, partial, \
-                                   splits, err, st);
+                         int32_t batch, const KvLayout& kv, const int32_t* lens, const int32_t* sel,
+                         const uint8_t* mask, const int32_t* cnt, float* partial, int32_t splits, int32_t* err,
+                         cudaStream_t st) {
+#define SWS_G(GG) \
+  case GG:        \
+    return launch_attn3<D, BS, GG>(q, kc, vc, batch, kv, lens, sel, mask, cnt, partial, splits, err, st);
   switch (group) {
     SWS_G(1) SWS_G(2) SWS_G(4) SWS_G(8)
     default:
@@ -652,18 +688,16 @@ int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group)
   return static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(256, ceil_div64(umax, 16))));
 }
 
-cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, int32_t batch, int32_t hkv,
-                                     int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, const KvLayout& kv,
+                                     int32_t batch, const int32_t* seq_lens, double* k_psum, double* k_sketch,
                                      cudaStream_t st) {
-  const int32_t B = h->cfg.block_size;
-  const int64_t mb = ceil_div64(max_len, B);
-  dim3 grid(static_cast<unsigned>(mb), static_cast<unsigned>((int64_t)batch * hkv));
+  dim3 grid(static_cast<unsigned>(kv.max_blocks), static_cast<unsigned>((int64_t)batch * kv.hkv));
   if (h->cfg.head_dim == 128)
-    init_cache_kernel<128><<<grid, 128, 0, st>>>(k_cache, hkv, max_len, B, mb, seq_lens, h->hdt, h->cfg.sketch_dim,
-                                                 k_psum, k_sketch, h->err);
+    init_cache_kernel<128><<<grid, 128, 0, st>>>(k_cache, kv, seq_lens, h->hdt, h->cfg.sketch_dim, k_psum, k_sketch,
+                                                 h->err);
   else
-    init_cache_kernel<64><<<grid, 64, 0, st>>>(k_cache, hkv, max_len, B, mb, seq_lens, h->hdt, h->cfg.sketch_dim,
-                                               k_psum, k_sketch, h->err);
+    init_cache_kernel<64><<<grid, 64, 0, st>>>(k_cache, kv, seq_lens, h->hdt, h->cfg.sketch_dim, k_psum, k_sketch,
+                                               h->err);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -675,19 +709,19 @@ cudaError_t launch_decode_advance(int32_t* seq_lens, int32_t batch, cudaStream_t
 }
 
 cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
-                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, const KvLayout& kv,
                                  const int32_t* seq_lens, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
                                  double* k_psum, double* k_sketch, int first_layer, double* walk_state,
                                  int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
                                  int32_t* sel_cnt, cudaStream_t st) {
   const sws_config& c = h->cfg;
-  const int64_t mb = ceil_div64(max_len, c.block_size);
-  const size_t smem = decode_select_smem_bytes(c, mb, hq / hkv);
+  const int32_t hkv = kv.hkv;
+  const size_t smem = decode_select_smem_bytes(c, kv.max_blocks, hq / hkv);
   auto kern = c.head_dim == 128 ? decode_select_kernel<128> : decode_select_kernel<64>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<static_cast<unsigned>((int64_t)batch * hkv), kSelThreads, smem, st>>>(
-      q_tok, k_tok, v_tok, hq, hkv, max_len, mb, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
+      q_tok, k_tok, v_tok, hq, kv, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
       walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, h->hdt, c.sketch_dim, c.block_size, c.walk_power,
       c.density_num, c.density_den, (c.select_group > 1 && hq / hkv > 1) ? 1 : 0, h->err);
   note_launches(1);
@@ -695,24 +729,24 @@ cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok
 }
 
 cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,
-                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, const KvLayout& kv,
                                const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
                                const int32_t* sel_cnt, __nv_bfloat16* o, float* partial, int32_t splits,
                                cudaStream_t st) {
   const sws_config& c = h->cfg;
-  const int64_t mb = ceil_div64(max_len, c.block_size);
+  const int32_t hkv = kv.hkv;
   const int32_t group = hq / hkv;
   cudaError_t e;
   if (c.head_dim == 128)
-    e = c.block_size == 64 ? launch_attn2<128, 64>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
-                                                    sel, sel_mask, sel_cnt, partial, splits, h->err, st)
-                           : launch_attn2<128, 128>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb,
-                                                     seq_lens, sel, sel_mask, sel_cnt, partial, splits, h->err, st);
+    e = c.block_size == 64 ? launch_attn2<128, 64>(group, q_tok, k_cache, v_cache, batch, kv, seq_lens, sel, sel_mask,
+                                                    sel_cnt, partial, splits, h->err, st)
+                           : launch_attn2<128, 128>(group, q_tok, k_cache, v_cache, batch, kv, seq_lens, sel,
+                                                     sel_mask, sel_cnt, partial, splits, h->err, st);
   else
-    e = c.block_size == 64 ? launch_attn2<64, 64>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
-                                                   sel, sel_mask, sel_cnt, partial, splits, h->err, st)
-                           : launch_attn2<64, 128>(group, q_tok, k_cache, v_cache, batch, hkv, max_len, mb, seq_lens,
-                                                    sel, sel_mask, sel_cnt, partial, splits, h->err, st);
+    e = c.block_size == 64 ? launch_attn2<64, 64>(group, q_tok, k_cache, v_cache, batch, kv, seq_lens, sel, sel_mask,
+                                                   sel_cnt, partial, splits, h->err, st)
+                           : launch_attn2<64, 128>(group, q_tok, k_cache, v_cache, batch, kv, seq_lens, sel, sel_mask,
+                                                    sel_cnt, partial, splits, h->err, st);
   if (e != cudaSuccess) return e;
   if (c.head_dim == 128)
     decode_combine_kernel<128><<<static_cast<unsigned>((int64_t)batch * hq), 128, 0, st>>>(partial, hq, hkv, splits,
@@ -783,7 +817,8 @@ extern "C" sws_status sws_sparse_attn_decode_noalloc(const sws_handle* h, const 
   if (noalloc_scratch(device, &scratch) != cudaSuccess) return SWS_ERR_CUDA;
   const cudaError_t e = sws::launch_decode_attn(
       h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_cache),
-      static_cast<const __nv_bfloat16*>(v_cache), batch, hq, hkv, max_len, seq_lens, sel, sel_mask, sel_cnt,
-      static_cast<__nv_bfloat16*>(o), static_cast<float*>(scratch), splits, static_cast<cudaStream_t>(stream));
+      static_cast<const __nv_bfloat16*>(v_cache), batch, hq, sws::contiguous_kv(h->cfg, hkv, max_len), seq_lens, sel,
+      sel_mask, sel_cnt, static_cast<__nv_bfloat16*>(o), static_cast<float*>(scratch), splits,
+      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWS_OK : SWS_ERR_CUDA;
 }

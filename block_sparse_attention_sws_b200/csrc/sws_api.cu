@@ -67,6 +67,68 @@ constexpr int64_t kMaxPrefillBlocks = 8192;  // top-tau counters and row staging
 
 }  // namespace
 
+namespace {
+
+sws_status decode_init_cache(const sws_handle* h, const void* k_cache, const KvLayout& kv, int32_t batch,
+                             const int32_t* seq_lens, double* k_psum, double* k_sketch, void* stream) {
+  if (!aligned16(k_cache) || !aligned16(seq_lens) || !aligned16(k_psum) || !aligned16(k_sketch))
+    return SWS_ERR_INVALID_ARG;
+  return cuda_status(launch_decode_init_cache(h, static_cast<const __nv_bfloat16*>(k_cache), kv, batch, seq_lens,
+                                              k_psum, k_sketch, static_cast<cudaStream_t>(stream)),
+                     "decode init cache");
+}
+
+sws_status decode_step(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok, int32_t batch,
+                       int32_t hq, const KvLayout& kv, const int32_t* seq_lens, void* k_cache, void* v_cache,
+                       double* k_psum, double* k_sketch, int first_layer, double* walk_state, int32_t* head_sel,
+                       int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
+  if (!h || batch < 1 || check_heads(hq, kv.hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (hq / kv.hkv > 8) return SWS_ERR_UNSUPPORTED;
+  if (h->cfg.select_group > 1 && h->cfg.select_group != hq / kv.hkv) return SWS_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch,
+                        walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  if (decode_select_smem_bytes(h->cfg, kv.max_blocks, hq / kv.hkv) > (200u << 10)) return SWS_ERR_UNSUPPORTED;
+  return cuda_status(
+      launch_decode_select(h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_tok),
+                           static_cast<const __nv_bfloat16*>(v_tok), batch, hq, kv, seq_lens,
+                           static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), k_psum,
+                           k_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                           static_cast<cudaStream_t>(stream)),
+      "decode step");
+}
+
+sws_status sparse_attn_decode(const sws_handle* h, const void* q_tok, const void* k_cache, const void* v_cache,
+                              int32_t batch, int32_t hq, const KvLayout& kv, const int32_t* seq_lens,
+                              const int32_t* sel, const uint8_t* sel_mask, const int32_t* sel_cnt, void* o, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (!h || batch < 1 || check_heads(hq, kv.hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  const int32_t group = hq / kv.hkv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o, ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  size_t need = 0;
+  sws_workspace_size(&h->cfg, SWS_OP_DECODE_ATTN, kv.max_len, hq, kv.hkv, batch, &need);
+  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
+  const int32_t splits = decode_num_splits(h->cfg, kv.max_len, group);
+  return cuda_status(launch_decode_attn(h, static_cast<const __nv_bfloat16*>(q_tok),
+                                        static_cast<const __nv_bfloat16*>(k_cache),
+                                        static_cast<const __nv_bfloat16*>(v_cache), batch, hq, kv, seq_lens, sel,
+                                        sel_mask, sel_cnt, static_cast<__nv_bfloat16*>(o), static_cast<float*>(ws),
+                                        splits, static_cast<cudaStream_t>(stream)),
+                     "decode attention");
+}
+
+// a paged pool: [num_pages, hkv, B, d] pages and a [batch, max_blocks] table
+bool paged_args_ok(int32_t hkv, int64_t num_pages, const int32_t* block_table, int64_t max_blocks) {
+  return hkv >= 1 && num_pages >= 1 && num_pages <= INT32_MAX && max_blocks >= 1 && max_blocks <= (INT32_MAX / 4096) &&
+         aligned16(block_table);
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* sws_status_string(sws_status s) {
@@ -351,11 +413,16 @@ sws_status sws_decode_init_cache(const sws_handle* h, const void* k_cache, int32
                                  int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
                                  void* stream) {
   if (!h || batch < 1 || hkv < 1 || max_len < 1) return SWS_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(seq_lens) || !aligned16(k_psum) || !aligned16(k_sketch))
-    return SWS_ERR_INVALID_ARG;
-  return cuda_status(launch_decode_init_cache(h, static_cast<const __nv_bfloat16*>(k_cache), batch, hkv, max_len,
-                                              seq_lens, k_psum, k_sketch, static_cast<cudaStream_t>(stream)),
-                     "decode init cache");
+  return decode_init_cache(h, k_cache, contiguous_kv(h->cfg, hkv, max_len), batch, seq_lens, k_psum, k_sketch,
+                           stream);
+}
+
+sws_status sws_decode_init_cache_paged(const sws_handle* h, const void* k_pages, int64_t num_pages,
+                                       const int32_t* block_table, int64_t max_blocks, int32_t batch, int32_t hkv,
+                                       const int32_t* seq_lens, double* k_psum, double* k_sketch, void* stream) {
+  if (!h || batch < 1 || !paged_args_ok(hkv, num_pages, block_table, max_blocks)) return SWS_ERR_INVALID_ARG;
+  return decode_init_cache(h, k_pages, paged_kv(h->cfg, hkv, block_table, max_blocks, num_pages), batch, seq_lens,
+                           k_psum, k_sketch, stream);
 }
 
 sws_status sws_decode_advance(const sws_handle* h, int32_t* seq_lens, int32_t batch, void* stream) {
@@ -368,44 +435,42 @@ sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k
                            void* k_cache, void* v_cache, double* k_psum, double* k_sketch, int first_layer,
                            double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
                            uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
-  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
-  if (hq / hkv > 8) return SWS_ERR_UNSUPPORTED;
-  if (h->cfg.select_group > 1 && h->cfg.select_group != hq / hkv) return SWS_ERR_INVALID_ARG;
-  const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch,
-                        walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
-  const int64_t mb = ceil_div64(max_len, h->cfg.block_size);
-  if (decode_select_smem_bytes(h->cfg, mb, hq / hkv) > (200u << 10)) return SWS_ERR_UNSUPPORTED;
-  return cuda_status(
-      launch_decode_select(h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_tok),
-                           static_cast<const __nv_bfloat16*>(v_tok), batch, hq, hkv, max_len, seq_lens,
-                           static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), k_psum,
-                           k_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
-                           static_cast<cudaStream_t>(stream)),
-      "decode step");
+  if (!h || max_len < 1 || hkv < 1) return SWS_ERR_INVALID_ARG;
+  return decode_step(h, q_tok, k_tok, v_tok, batch, hq, contiguous_kv(h->cfg, hkv, max_len), seq_lens, k_cache,
+                     v_cache, k_psum, k_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                     stream);
+}
+
+sws_status sws_decode_step_paged(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                 int32_t batch, int32_t hq, int32_t hkv, void* k_pages, void* v_pages,
+                                 int64_t num_pages, const int32_t* block_table, int64_t max_blocks,
+                                 const int32_t* seq_lens, double* k_psum, double* k_sketch, int first_layer,
+                                 double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
+                                 uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
+  if (!h || !paged_args_ok(hkv, num_pages, block_table, max_blocks)) return SWS_ERR_INVALID_ARG;
+  return decode_step(h, q_tok, k_tok, v_tok, batch, hq, paged_kv(h->cfg, hkv, block_table, max_blocks, num_pages),
+                     seq_lens, k_pages, v_pages, k_psum, k_sketch, first_layer, walk_state, head_sel, head_cnt, sel,
+                     sel_mask, sel_cnt, stream);
 }
 
 sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const void* k_cache, const void* v_cache,
                                   int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
                                   const int32_t* sel, const uint8_t* sel_mask, const int32_t* sel_cnt, void* o,
                                   void* ws, size_t ws_bytes, void* stream) {
-  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
-  const int32_t group = hq / hkv;
-  if (group != 1 && group != 2 && group != 4 && group != 8) return SWS_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q_tok, k_cache, v_cache, seq_lens, sel, sel_mask, sel_cnt, o, ws};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
-  size_t need = 0;
-  sws_workspace_size(&h->cfg, SWS_OP_DECODE_ATTN, max_len, hq, hkv, batch, &need);
-  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
-  const int32_t splits = decode_num_splits(h->cfg, max_len, group);
-  return cuda_status(launch_decode_attn(h, static_cast<const __nv_bfloat16*>(q_tok),
-                                        static_cast<const __nv_bfloat16*>(k_cache),
-                                        static_cast<const __nv_bfloat16*>(v_cache), batch, hq, hkv, max_len,
-                                        seq_lens, sel, sel_mask, sel_cnt, static_cast<__nv_bfloat16*>(o),
-                                        static_cast<float*>(ws), splits, static_cast<cudaStream_t>(stream)),
-                     "decode attention");
+  if (!h || max_len < 1 || hkv < 1) return SWS_ERR_INVALID_ARG;
+  return sparse_attn_decode(h, q_tok, k_cache, v_cache, batch, hq, contiguous_kv(h->cfg, hkv, max_len), seq_lens,
+                            sel, sel_mask, sel_cnt, o, ws, ws_bytes, stream);
+}
+
+sws_status sws_sparse_attn_decode_paged(const sws_handle* h, const void* q_tok, const void* k_pages,
+                                        const void* v_pages, int64_t num_pages, const int32_t* block_table,
+                                        int64_t max_blocks, int32_t batch, int32_t hq, int32_t hkv,
+                                        const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
+                                        const int32_t* sel_cnt, void* o, void* ws, size_t ws_bytes, void* stream) {
+  if (!h || !paged_args_ok(hkv, num_pages, block_table, max_blocks)) return SWS_ERR_INVALID_ARG;
+  return sparse_attn_decode(h, q_tok, k_pages, v_pages, batch, hq,
+                            paged_kv(h->cfg, hkv, block_table, max_blocks, num_pages), seq_lens, sel, sel_mask,
+                            sel_cnt, o, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -28,7 +28,8 @@ enum Guard : int32_t {
   GUARD_BAD_CSR = 2,       // a CSR entry outside [0, i] or a non-ascending row
   GUARD_BAD_SELECT = 3,    // top-tau bookkeeping inconsistent
   GUARD_BAD_LEN = 4,       // a sequence length outside [1, max_len]
-  GUARD_TMEM = 5           // tensor memory allocation failed
+  GUARD_TMEM = 5,          // tensor memory allocation failed
+  GUARD_BAD_PAGE = 6       // a block table entry outside [0, num_pages)
 };
 
 __device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
@@ -162,12 +163,44 @@ cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const voi
                                    int32_t hq, int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o,
                                    cudaStream_t st);
 
-cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, int32_t batch, int32_t hkv,
-                                     int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
+// Where the cached keys (or values) of one (sequence, KV head) live.
+//  contiguous (block_table null): [batch, hkv, max_len, D]; token t of the unit
+//    (sequence i, KV head g) is row (i * hkv + g) * max_len + t.
+//  paged: a pool of pages [num_pages, hkv, B, D], one page per key block of a
+//    sequence (all its KV heads); block_table[i * max_blocks + j] is the page of
+//    logical block j of sequence i, so token t is row t % B of page
+//    block_table[i * max_blocks + t / B]. max_len = max_blocks * B.
+struct KvLayout {
+  const int32_t* block_table;
+  int64_t max_len;     // tokens a sequence can hold
+  int64_t max_blocks;  // ceil(max_len / B)
+  int64_t num_pages;
+  int32_t hkv, B, D;
+};
+
+inline KvLayout contiguous_kv(const sws_config& c, int32_t hkv, int64_t max_len) {
+  return KvLayout{nullptr, max_len, ceil_div64(max_len, c.block_size), 0, hkv, c.block_size, c.head_dim};
+}
+inline KvLayout paged_kv(const sws_config& c, int32_t hkv, const int32_t* block_table, int64_t max_blocks,
+                         int64_t num_pages) {
+  return KvLayout{block_table, max_blocks * c.block_size, max_blocks, num_pages, hkv, c.block_size, c.head_dim};
+}
+
+// Element offset of the first row of logical block j of (sequence bi, KV
+// head g), or -1 when the block table points outside the pool.
+__device__ __forceinline__ int64_t kv_block_offset(const KvLayout& L, int64_t bi, int64_t g, int64_t j) {
+  if (!L.block_table) return ((bi * L.hkv + g) * L.max_len + j * L.B) * L.D;
+  const int64_t p = L.block_table[bi * L.max_blocks + j];
+  if (p < 0 || p >= L.num_pages) return -1;
+  return ((p * L.hkv + g) * L.B) * L.D;
+}
+
+cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k_cache, const KvLayout& kv,
+                                     int32_t batch, const int32_t* seq_lens, double* k_psum, double* k_sketch,
                                      cudaStream_t st);
 cudaError_t launch_decode_advance(int32_t* seq_lens, int32_t batch, cudaStream_t st);
 cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
-                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                 const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, const KvLayout& kv,
                                  const int32_t* seq_lens, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
                                  double* k_psum, double* k_sketch, int first_layer, double* walk_state,
                                  int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
@@ -175,7 +208,7 @@ cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok
 int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group);
 size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
 cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,
-                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                               const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, const KvLayout& kv,
                                const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
                                const int32_t* sel_cnt, __nv_bfloat16* o, float* partial, int32_t splits,
                                cudaStream_t st);

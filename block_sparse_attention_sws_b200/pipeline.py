@@ -82,18 +82,34 @@ class PrefillPath:
 class DecodePath:
     """Per-layer decode state and the per-step call order:
     sws_decode_step -> sws_sparse_attn_decode for each layer, then
-    sws_decode_advance once the step's layers are done."""
+    sws_decode_advance once the step's layers are done.
 
-    def __init__(self, handle: L.Handle, batch: int, hq: int, hkv: int, max_len: int, layers: int, device="cuda"):
+    paged=True keeps each layer's keys and values in a pool of pages
+    [num_pages, hkv, B, d] addressed through block_table [batch, max_blocks]
+    (shared by the layers) and calls the *_paged entry points. The default
+    table gives sequence i the pages i * max_blocks .. (i + 1) * max_blocks - 1;
+    a caller may overwrite self.block_table with any assignment of distinct
+    pages before writing the caches."""
+
+    def __init__(self, handle: L.Handle, batch: int, hq: int, hkv: int, max_len: int, layers: int, device="cuda",
+                 paged=False, num_pages=None):
         cfg = handle.cfg
         self.h, self.batch, self.hq, self.hkv, self.max_len, self.layers = handle, batch, hq, hkv, max_len, layers
-        d, k = cfg.head_dim, cfg.sketch_dim
+        d, k, B = cfg.head_dim, cfg.sketch_dim, cfg.block_size
         self.mb = L.sws_num_blocks(cfg, max_len)
+        self.paged = paged
         bf = dict(dtype=torch.bfloat16, device=device)
         f64 = dict(dtype=torch.float64, device=device)
         i32 = dict(dtype=torch.int32, device=device)
-        self.k_cache = [torch.empty(batch, hkv, max_len, d, **bf) for _ in range(layers)]
-        self.v_cache = [torch.empty(batch, hkv, max_len, d, **bf) for _ in range(layers)]
+        if paged:
+            self.num_pages = batch * self.mb if num_pages is None else num_pages
+            self.block_table = torch.arange(batch * self.mb, **i32).reshape(batch, self.mb) % self.num_pages
+            self.k_cache = [torch.empty(self.num_pages, hkv, B, d, **bf) for _ in range(layers)]
+            self.v_cache = [torch.empty(self.num_pages, hkv, B, d, **bf) for _ in range(layers)]
+            self.max_len = self.mb * B
+        else:
+            self.k_cache = [torch.empty(batch, hkv, max_len, d, **bf) for _ in range(layers)]
+            self.v_cache = [torch.empty(batch, hkv, max_len, d, **bf) for _ in range(layers)]
         self.k_psum = [torch.zeros(batch, hkv, d, **f64) for _ in range(layers)]
         self.k_sketch = [torch.zeros(batch, hkv, self.mb, k, **f64) for _ in range(layers)]
         self.seq_lens = torch.zeros(batch, **i32)
@@ -103,25 +119,76 @@ class DecodePath:
         self.sel = torch.zeros(batch, hkv, self.mb, **i32)
         self.sel_mask = torch.zeros(batch, hkv, self.mb, dtype=torch.uint8, device=device)
         self.sel_cnt = torch.zeros(batch, hkv, **i32)
-        ws = L.sws_workspace_size(cfg, L.SWS_OP_DECODE_ATTN, max_len, hq, hkv, batch)
+        ws = L.sws_workspace_size(cfg, L.SWS_OP_DECODE_ATTN, self.max_len, hq, hkv, batch)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.o = torch.empty(batch, hq, d, **bf)
+
+    @staticmethod
+    def _scatter_pages(pool, pages, src, n: int, B: int):
+        # tokens [0, n) of src [hkv, >= n, d] to the pages of their blocks
+        nf, r = divmod(n, B)
+        if nf:
+            pool[pages[:nf]] = src[:, :nf * B].reshape(src.shape[0], nf, B, -1).transpose(0, 1)
+        if r:
+            pool[pages[nf], :, :r] = src[:, nf * B:n]
+
+    def write_cache(self, layer: int, seq: int, k, v, n: int):
+        """Store the first n tokens of k, v [hkv, >= n, d] as sequence seq's cache."""
+        if not self.paged:
+            self.k_cache[layer][seq, :, :n] = k[:, :n]
+            self.v_cache[layer][seq, :, :n] = v[:, :n]
+            return
+        pages = self.block_table[seq].long()
+        B = self.h.cfg.block_size
+        self._scatter_pages(self.k_cache[layer], pages, k, n, B)
+        self._scatter_pages(self.v_cache[layer], pages, v, n, B)
+
+    def to_paged(self, block_table: torch.Tensor, num_pages: int):
+        """Move contiguous caches into page pools (every token slot, one layer
+        and one of K, V at a time, so that about one layer's cache is the extra
+        memory); block_table [batch, max_blocks] int32 on the device, distinct
+        pages in [0, num_pages). Sketches and lengths are kept."""
+        assert not self.paged and tuple(block_table.shape) == (self.batch, self.mb)
+        B, d = self.h.cfg.block_size, self.h.cfg.head_dim
+        pages = block_table.long()
+        for caches in (self.k_cache, self.v_cache):
+            for layer in range(self.layers):
+                src = caches[layer]
+                pool = torch.empty(num_pages, self.hkv, B, d, dtype=src.dtype, device=src.device)
+                for i in range(self.batch):
+                    self._scatter_pages(pool, pages[i], src[i], self.max_len, B)
+                caches[layer] = pool
+                del src
+        self.paged, self.block_table, self.num_pages = True, block_table, num_pages
+        self.max_len = self.mb * B
 
     def init_cache(self, lens: torch.Tensor, stream=None):
         """Caches already hold lens[i] tokens per sequence: build their sketches."""
         self.seq_lens.copy_(lens)
         for layer in range(self.layers):
-            L.sws_decode_init_cache(self.h, self.k_cache[layer], self.seq_lens, self.k_psum[layer],
-                                    self.k_sketch[layer], stream)
+            if self.paged:
+                L.sws_decode_init_cache_paged(self.h, self.k_cache[layer], self.block_table, self.seq_lens,
+                                              self.k_psum[layer], self.k_sketch[layer], stream)
+            else:
+                L.sws_decode_init_cache(self.h, self.k_cache[layer], self.seq_lens, self.k_psum[layer],
+                                        self.k_sketch[layer], stream)
 
     def begin_step(self, stream=None):
         L.sws_decode_advance(self.h, self.seq_lens, stream)
 
     def layer(self, layer: int, q_tok, k_tok, v_tok, out=None, stream=None):
+        o = self.o if out is None else out
+        if self.paged:
+            L.sws_decode_step_paged(self.h, q_tok, k_tok, v_tok, self.k_cache[layer], self.v_cache[layer],
+                                    self.block_table, self.seq_lens, self.k_psum[layer], self.k_sketch[layer],
+                                    layer == 0, self.walk_state, self.head_sel, self.head_cnt, self.sel,
+                                    self.sel_mask, self.sel_cnt, stream)
+            L.sws_sparse_attn_decode_paged(self.h, q_tok, self.k_cache[layer], self.v_cache[layer], self.block_table,
+                                           self.seq_lens, self.sel, self.sel_mask, self.sel_cnt, o, self.ws, stream)
+            return o
         L.sws_decode_step(self.h, q_tok, k_tok, v_tok, self.seq_lens, self.k_cache[layer], self.v_cache[layer],
                           self.k_psum[layer], self.k_sketch[layer], layer == 0, self.walk_state, self.head_sel,
                           self.head_cnt, self.sel, self.sel_mask, self.sel_cnt, stream)
-        o = self.o if out is None else out
         L.sws_sparse_attn_decode(self.h, q_tok, self.k_cache[layer], self.v_cache[layer], self.seq_lens, self.sel,
                                  self.sel_mask, self.sel_cnt, o, self.ws, stream)
         return o

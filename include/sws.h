@@ -210,6 +210,38 @@ sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const 
                                   const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
                                   const int32_t* sel_cnt, void* o, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------ paged KV cache --- */
+/* The same three decode calls over a paged cache: a pool of pages shared by all the
+ * sequences of a batch, each page holding one key block (B tokens) of one sequence for
+ * all of its KV heads, and a block table that maps each sequence's logical blocks to
+ * pages. The pages have no counterpart in "Scout Before You Attend"; they let a
+ * serving loop grow, share and free sequence storage block by block. Selection and
+ * attention are the same as with the contiguous cache: the same pool content gives
+ * the same result, bit for bit.
+ *   k_pages, v_pages [num_pages, hkv, B, d] bf16 (device)
+ *   block_table      [batch, max_blocks] int32 (device): the page of logical block j of
+ *                    sequence i; entries past ceil(seq_lens[i] / B) are not read
+ * A sequence holds at most max_blocks * B tokens (the max_len of the contiguous calls;
+ * size k_sketch and walk_state with max_blocks, and query sws_workspace_size with
+ * n = max_blocks * B). The step call writes the new token into its block's page, so
+ * that page must be assigned before the call. A table entry outside [0, num_pages)
+ * is not dereferenced: the block reads as empty (init, attention) or the token is not
+ * appended, and guard code 6 is recorded for sws_sync_check. */
+sws_status sws_decode_init_cache_paged(const sws_handle* h, const void* k_pages, int64_t num_pages,
+                                       const int32_t* block_table, int64_t max_blocks, int32_t batch, int32_t hkv,
+                                       const int32_t* seq_lens, double* k_psum, double* k_sketch, void* stream);
+sws_status sws_decode_step_paged(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                 int32_t batch, int32_t hq, int32_t hkv, void* k_pages, void* v_pages,
+                                 int64_t num_pages, const int32_t* block_table, int64_t max_blocks,
+                                 const int32_t* seq_lens, double* k_psum, double* k_sketch, int first_layer,
+                                 double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
+                                 uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
+sws_status sws_sparse_attn_decode_paged(const sws_handle* h, const void* q_tok, const void* k_pages,
+                                        const void* v_pages, int64_t num_pages, const int32_t* block_table,
+                                        int64_t max_blocks, int32_t batch, int32_t hq, int32_t hkv,
+                                        const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
+                                        const int32_t* sel_cnt, void* o, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------- no-allocation variant --- */
 /* The paper has no counterpart to this call; it serves callers that cannot allocate
  * device memory on the decode path (a plug-in whose host framework owns every device

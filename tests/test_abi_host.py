@@ -116,6 +116,12 @@ def test_null_handle_rejected_without_launch(lib):
                                        None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_destroy(None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_projection_device(None) is None
+    assert lib.sws_decode_init_cache_paged(None, P(16), 4, P(16), 4, 1, 1, P(16), P(16), P(16),
+                                           None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_decode_step_paged(None, P(16), P(16), P(16), 1, 4, 1, P(16), P(16), 4, P(16), 4, P(16), P(16),
+                                     P(16), 1, P(16), P(16), P(16), P(16), P(16), P(16), None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_sparse_attn_decode_paged(None, P(16), P(16), P(16), 4, P(16), 4, 1, 4, 1, P(16), P(16), P(16),
+                                            P(16), P(16), P(16), 1 << 20, None) == S.SWS_ERR_INVALID_ARG
 
 
 def test_create_reports_error_without_gpu(lib):

@@ -20,13 +20,25 @@ from parity import compare_attention, compare_selection
 pytestmark = pytest.mark.gpu
 
 
-def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
+def make_path(h, w, batch, max_len, paged, dev="cuda"):
+    """A decode path; paged: the pool has a few spare pages and each sequence's
+    blocks sit on pages in a seeded random order."""
+    if not paged:
+        return S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev)
+    mb = -(-max_len // w.B)
+    path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev, paged=True, num_pages=batch * mb + 5)
+    perm = torch.randperm(batch * mb + 5, generator=torch.Generator().manual_seed(w.seed + 77))[:batch * mb]
+    path.block_table.copy_(perm.reshape(batch, mb).to(torch.int32))
+    return path
+
+
+def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False, paged=False, path_out=None):
     dev = "cuda"
     batch = len(n0s)
     cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed, select_group=(w.hq // w.hkv) if shared else 0)
     h = S.Handle(cfg)
     max_len = max(n0s) + steps
-    path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev)
+    path = make_path(h, w, batch, max_len, paged, dev)
     group = w.hq // w.hkv
     check_seqs = list(range(batch)) if check_seqs is None else list(check_seqs)
     KV, Qs = {}, {}
@@ -36,8 +48,7 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
         for s_, n0 in enumerate(n0s):
             ws_ = w.scaled(n0=n0, steps=steps)
             K, V = W.decode_cache_inputs(ws_, s_, layer, dev)
-            path.k_cache[layer][s_, :, :n0] = K[:, :n0]
-            path.v_cache[layer][s_, :, :n0] = V[:, :n0]
+            path.write_cache(layer, s_, K, V, n0)
             KV[(s_, layer)] = (K, V)
             Qs[(s_, layer)] = W.decode_queries(ws_, s_, layer, dev)
     path.init_cache(torch.tensor(n0s, dtype=torch.int32, device=dev))
@@ -45,6 +56,7 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
     host = {key: (K.double().cpu().numpy(), V.double().cpu().numpy()) for key, (K, V) in KV.items()
             if key[0] in check_seqs}
     swaps = []
+    outputs = []
     for t in range(steps):
         path.begin_step()
         rho_prev = {s_: None for s_ in check_seqs}
@@ -62,6 +74,8 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
             msk = path.sel_mask.cpu().numpy()
             cnt = path.sel_cnt.cpu().numpy()
             og = o.float().cpu().numpy()
+            outputs.append((hs.copy(), hc.copy(), rho_gpu.copy(), sel.copy(), msk.copy(), cnt.copy(),
+                            o.view(torch.int16).cpu().numpy()))
             for s_ in check_seqs:
                 length = n0s[s_] + t + 1
                 nb = -(-length // w.B)
@@ -97,6 +111,8 @@ def run_decode(w: W.DecodeWorkload, n0s, steps, check_seqs=None, shared=False):
                     assert n == len(ug)
                     assert list(sel[s_, g, :n]) == sorted(ug)
                     assert [int(m) for m in msk[s_, g, :n]] == [ug[j] for j in sorted(ug)]
+    if path_out is not None:
+        path_out.extend(outputs)
     h.close()
     return swaps
 
@@ -164,3 +180,65 @@ def test_decode_group_shared_selection():
     swaps = run_decode(w, [1000, 1500, 638], steps=4, shared=True)
     for s in swaps:
         print("tolerated near-tie swap:", s)
+
+
+def test_decode_paged_cache():
+    """The paged pool (blocks on shuffled pages, spare pages, NaN in every
+    unwritten slot) against the oracle, ragged lengths crossing block ends."""
+    w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
+    swaps = run_decode(w, [1000, 1500, 638], steps=5, paged=True)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
+def test_decode_paged_equals_contiguous_bitwise():
+    """The same caches and tokens through the contiguous and the paged calls:
+    every selection, walk state and attention output is bit-identical."""
+    w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=4)
+    outs = {}
+    for paged in (False, True):
+        outs[paged] = []
+        run_decode(w, [900, 1300, 64], steps=3, check_seqs=[], paged=paged, path_out=outs[paged])
+    assert len(outs[False]) == len(outs[True]) == 6
+    for a, b in zip(outs[False], outs[True]):
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+def test_decode_paged_bad_page_guard():
+    """A block table entry outside the pool is not dereferenced: the kernels
+    record guard code 6 and the context stays usable."""
+    w = W.DECODE_128K.scaled(layers=1, hq=4, hkv=1)
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    path = S.DecodePath(h, 1, 4, 1, 256, 1, paged=True)
+    path.k_cache[0].zero_()
+    path.v_cache[0].zero_()
+    path.init_cache(torch.tensor([100], dtype=torch.int32, device="cuda"))
+    assert S.sws_sync_check(h) == 0
+    path.block_table[0, 1] = path.num_pages  # one past the pool
+    path.init_cache(torch.tensor([100], dtype=torch.int32, device="cuda"))
+    assert S.sws_sync_check(h) == 6  # GUARD_BAD_PAGE
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, 1, 128, dtype=torch.bfloat16, device="cuda")
+    path.begin_step()
+    path.layer(0, q, kv, kv)  # the token goes to block 1: not appended
+    assert S.sws_sync_check(h) == 6
+    path.block_table[0, 1] = -3
+    path.sel[0, 0, 0] = 1
+    path.sel_mask[0, 0, 0] = 1
+    path.sel_cnt[0, 0] = 1
+    S.sws_sparse_attn_decode_paged(h, q, path.k_cache[0], path.v_cache[0], path.block_table, path.seq_lens,
+                                   path.sel, path.sel_mask, path.sel_cnt, path.o, path.ws)
+    assert S.sws_sync_check(h) == 6
+    path.block_table[0, 1] = 1
+    path.init_cache(torch.tensor([100], dtype=torch.int32, device="cuda"))
+    assert S.sws_sync_check(h) == 0  # usable again
+    # host validation: an empty pool, an empty table, a misaligned table queue nothing
+    lib, P = S.load(), S._lib._ptr
+    for num_pages, bt, mb in ((0, P(path.block_table), 4), (4, P(path.block_table), 0),
+                              (4, P(path.block_table) + 4, 4)):
+        assert lib.sws_decode_init_cache_paged(h.ptr, P(path.k_cache[0]), num_pages, bt, mb, 1, 1,
+                                               P(path.seq_lens), P(path.k_psum[0]), P(path.k_sketch[0]),
+                                               None) == S.SWS_ERR_INVALID_ARG
+    h.close()
