@@ -465,20 +465,33 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
   // not loaded (src-size 0) still gets an address inside the cache.
   const __nv_bfloat16* kbase = k_cache + (kPaged ? 0 : unit * kv.max_len * D);
   const __nv_bfloat16* vbase = v_cache + (kPaged ? 0 : unit * kv.max_len * D);
+  // Paged: issue() is called for idx = lo, lo + 1, ... in order. The list
+  // entry of idx + 2 and the page of idx + 1 are loaded while idx is issued,
+  // and only used (the page checked and turned into an offset) one call
+  // later, so the copies of a block never wait on the two dependent lookups.
+  int64_t pf_raw = lo < hi ? blist[lo] : -1;  // list entry of the next idx to issue
+  int64_t pf_page = (kPaged && block_ok(pf_raw)) ? kv.block_table[(int64_t)bi * kv.max_blocks + pf_raw] : -1;
+  int64_t pf_raw2 = lo + 1 < hi ? blist[lo + 1] : -1;  // list entry after it
   auto issue = [&](int64_t idx, int st) {
-    int64_t j = block_ok(blist[idx]) ? blist[idx] : -1;
+    int64_t j;
     const __nv_bfloat16* kblk = kbase;
     const __nv_bfloat16* vblk = vbase;
     if constexpr (kPaged) {
-      const int64_t off = j < 0 ? -1 : kv_block_offset(kv, bi, unit % hkv, j);
-      if (j >= 0 && off < 0) {
+      j = block_ok(pf_raw) ? pf_raw : -1;
+      if (j >= 0 && (pf_page < 0 || pf_page >= kv.num_pages)) {
         if (tid == 0) record_error(err, GUARD_BAD_PAGE);
         j = -1;
       }
       if (j >= 0) {
+        const int64_t off = ((pf_page * hkv + unit % hkv) * BS) * D;
         kblk += off;
         vblk += off;
       }
+      pf_raw = pf_raw2;
+      pf_page = (idx + 1 < hi && block_ok(pf_raw)) ? kv.block_table[(int64_t)bi * kv.max_blocks + pf_raw] : -1;
+      pf_raw2 = idx + 2 < hi ? blist[idx + 2] : -1;
+    } else {
+      j = block_ok(blist[idx]) ? blist[idx] : -1;
     }
     const int64_t t0 = j < 0 ? (int64_t)len : j * BS;  // an invalid block stages zeros
     __nv_bfloat16* ksm = stage + (st * 2) * TILE;
