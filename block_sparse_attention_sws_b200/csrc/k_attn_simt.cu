@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
                                                           const int32_t* __restrict__ row_ptr,
                                                           const int32_t* __restrict__ col_idx, int64_t nnz,
                                                           T* __restrict__ o, float qscale, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   constexpr int HD = D / 2;
   constexpr int VE = 16 / sizeof(T);
   extern __shared__ __align__(16) uint8_t smem[];
@@ -122,8 +124,12 @@ cudaError_t launch_t(const sws_handle* h, const void* q, const void* k, const vo
   for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
   const float qscale = static_cast<float>(1.4426950408889634 / sqrt((double)D));  // log2(e) / sqrt(d)
   dim3 grid(static_cast<unsigned>(b), hq);
-  kern<<<grid, 2 * B, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), n,
-                                  hq / hkv, row_ptr, col_idx, nnz, static_cast<T*>(o), qscale, h->err);
+  {
+    const cudaError_t le = launch_k(kern, grid, 2 * B, smem, st, static_cast<const T*>(q), static_cast<const T*>(k),
+                                    static_cast<const T*>(v), n, hq / hkv, row_ptr, col_idx, nnz, static_cast<T*>(o),
+                                    qscale, h->err);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }

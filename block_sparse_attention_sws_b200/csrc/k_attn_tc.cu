@@ -347,6 +347,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
     const __grid_constant__ CUtensorMap tmv, int64_t n, int32_t hq, int32_t group, const int32_t* __restrict__ row_ptr,
     const int32_t* __restrict__ col_idx, int64_t nnz, __nv_bfloat16* __restrict__ o, float qscale, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   using L = Smem<D>;
   constexpr int QB = 256 / BLK;  // query blocks per item
   extern __shared__ uint8_t smem_raw[];
@@ -735,8 +737,11 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
   const int64_t items = ceil_div64(n, 2 * kTileM) * hq;
   const int grid = static_cast<int>(std::min<int64_t>(items, h->num_sms));
   const float qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
-  kern<<<grid, kTcThreads, smem, st>>>(mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx, nnz,
-                                       static_cast<__nv_bfloat16*>(o), qscale, h->err);
+  {
+    const cudaError_t le = launch_k(kern, grid, kTcThreads, smem, st, mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx,
+                                    nnz, static_cast<__nv_bfloat16*>(o), qscale, h->err);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }

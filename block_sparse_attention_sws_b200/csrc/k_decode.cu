@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(D) init_cache_kernel(const __nv_bfloat16* __re
                                                        const double* __restrict__ hdt, int32_t k,
                                                        double* __restrict__ k_psum, double* __restrict__ k_sketch,
                                                        int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   __shared__ double mean[D];
   const int64_t unit = blockIdx.y;  // sequence * hkv + kv head
   const int64_t bi = unit / kv.hkv, g = unit % kv.hkv;
@@ -66,6 +68,8 @@ __global__ void __launch_bounds__(D) init_cache_kernel(const __nv_bfloat16* __re
 }
 
 __global__ void advance_kernel(int32_t* seq_lens, int32_t batch) {
+  grid_dependency_wait();
+  allow_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < batch) seq_lens[i] += 1;
 }
@@ -189,6 +193,8 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     int32_t* __restrict__ head_sel, int32_t* __restrict__ head_cnt, int32_t* __restrict__ sel,
     uint8_t* __restrict__ sel_mask, int32_t* __restrict__ sel_cnt, const double* __restrict__ hdt, int32_t k,
     int32_t B, int32_t s_pow, int32_t num, int32_t den, int shared, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   const int32_t hkv = kv.hkv;
   const int64_t max_blocks = kv.max_blocks;
   const int group = hq / hkv;
@@ -408,6 +414,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ v_cache, KvLayout kv, const int32_t* __restrict__ seq_lens,
     const int32_t* __restrict__ sel, const uint8_t* __restrict__ sel_mask, const int32_t* __restrict__ sel_cnt,
     float* __restrict__ partial, int32_t splits, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   static_assert(G >= 1 && G <= 8, "GQA group of 1..8 query heads");
   constexpr int NT_QK = BS / 8 / 4;  // score n-tiles (8 tokens) per warp
   constexpr int NT_PV = D / 8 / 4;   // output n-tiles (8 dims) per warp
@@ -637,6 +645,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ partial, int32_t hq, int32_t hkv,
                                                            int32_t splits, __nv_bfloat16* __restrict__ o) {
+  grid_dependency_wait();
+  allow_dependents();
   const int64_t bh = blockIdx.x;  // sequence * hq + head
   const int group = hq / hkv;
   const int64_t bi = bh / hq;
@@ -665,7 +675,11 @@ cudaError_t launch_attn3(const __nv_bfloat16* q, const __nv_bfloat16* kc, const 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(splits, static_cast<unsigned>((int64_t)batch * kv.hkv));
-  kern<<<grid, kAttnThreads, smem, st>>>(q, kc, vc, kv, lens, sel, mask, cnt, partial, splits, err);
+  {
+    const cudaError_t le = launch_k(kern, grid, kAttnThreads, smem, st, q, kc, vc, kv, lens, sel, mask, cnt, partial,
+                                    splits, err);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -706,17 +720,27 @@ cudaError_t launch_decode_init_cache(const sws_handle* h, const __nv_bfloat16* k
                                      cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(kv.max_blocks), static_cast<unsigned>((int64_t)batch * kv.hkv));
   if (h->cfg.head_dim == 128)
-    init_cache_kernel<128><<<grid, 128, 0, st>>>(k_cache, kv, seq_lens, h->hdt, h->cfg.sketch_dim, k_psum, k_sketch,
-                                                 h->err);
+    {
+      const cudaError_t le = launch_k(init_cache_kernel<128>, grid, 128, 0, st, k_cache, kv, seq_lens,
+                                      h->hdt, h->cfg.sketch_dim, k_psum, k_sketch, h->err);
+      if (le != cudaSuccess) return le;
+    }
   else
-    init_cache_kernel<64><<<grid, 64, 0, st>>>(k_cache, kv, seq_lens, h->hdt, h->cfg.sketch_dim, k_psum, k_sketch,
-                                               h->err);
+    {
+      const cudaError_t le = launch_k(init_cache_kernel<64>, grid, 64, 0, st, k_cache, kv, seq_lens,
+                                      h->hdt, h->cfg.sketch_dim, k_psum, k_sketch, h->err);
+      if (le != cudaSuccess) return le;
+    }
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_advance(int32_t* seq_lens, int32_t batch, cudaStream_t st) {
-  advance_kernel<<<static_cast<unsigned>(ceil_div64(batch, 128)), 128, 0, st>>>(seq_lens, batch);
+  {
+    const cudaError_t le = launch_k(advance_kernel, static_cast<unsigned>(ceil_div64(batch, 128)), 128, 0, st, seq_lens,
+                                    batch);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -733,10 +757,14 @@ cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok
   auto kern = c.head_dim == 128 ? decode_select_kernel<128> : decode_select_kernel<64>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>((int64_t)batch * hkv), kSelThreads, smem, st>>>(
-      q_tok, k_tok, v_tok, hq, kv, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
-      walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, h->hdt, c.sketch_dim, c.block_size, c.walk_power,
-      c.density_num, c.density_den, (c.select_group > 1 && hq / hkv > 1) ? 1 : 0, h->err);
+  {
+    const cudaError_t le = launch_k(kern, static_cast<unsigned>((int64_t)batch * hkv), kSelThreads, smem, st, q_tok,
+                                    k_tok, v_tok, hq, kv, seq_lens, k_cache, v_cache, k_psum, k_sketch, first_layer,
+                                    walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt, h->hdt, c.sketch_dim,
+                                    c.block_size, c.walk_power, c.density_num, c.density_den,
+                                    (c.select_group > 1 && hq / hkv > 1) ? 1 : 0, h->err);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -762,10 +790,17 @@ cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, 
                                                     sel_cnt, partial, splits, h->err, st);
   if (e != cudaSuccess) return e;
   if (c.head_dim == 128)
-    decode_combine_kernel<128><<<static_cast<unsigned>((int64_t)batch * hq), 128, 0, st>>>(partial, hq, hkv, splits,
-                                                                                          o);
+    {
+      const cudaError_t le = launch_k(decode_combine_kernel<128>, static_cast<unsigned>((int64_t)batch * hq), 128, 0,
+                                      st, partial, hq, hkv, splits, o);
+      if (le != cudaSuccess) return le;
+    }
   else
-    decode_combine_kernel<64><<<static_cast<unsigned>((int64_t)batch * hq), 64, 0, st>>>(partial, hq, hkv, splits, o);
+    {
+      const cudaError_t le = launch_k(decode_combine_kernel<64>, static_cast<unsigned>((int64_t)batch * hq), 64, 0, st,
+                                      partial, hq, hkv, splits, o);
+      if (le != cudaSuccess) return le;
+    }
   note_launches(1);
   return cudaGetLastError();
 }

@@ -49,6 +49,8 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
     pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
                         int32_t B, int64_t nblk, const double* __restrict__ sign, const int32_t* __restrict__ col,
                         double scale, int32_t ksk, double* __restrict__ q_sk, double* __restrict__ k_sk) {
+  grid_dependency_wait();
+  allow_dependents();
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte vector
   constexpr int VR = D / VE;          // vectors per row
   static_assert(VR <= 32 && 32 % VR == 0, "row must map onto a whole number of lanes");
@@ -172,6 +174,8 @@ __device__ __forceinline__ void dmma_16x8x4_s(double (&c)[4], double a0, double 
 __global__ void __launch_bounds__(64) scores_kernel(const double* __restrict__ q_sk, const double* __restrict__ k_sk,
                                                     int64_t b, int32_t hq, int32_t group, int32_t k,
                                                     double inv_sqrt_k, double* __restrict__ S) {
+  grid_dependency_wait();
+  allow_dependents();
   __shared__ __align__(16) double qs[kST][kSC + 4];  // [query block][sketch dim]
   __shared__ __align__(16) double ks[kSC][kST + 4];  // [sketch dim][key block]
   const int64_t t = blockIdx.x;
@@ -238,8 +242,11 @@ cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int
   const int64_t nblk = ceil_div64(n, B);
   const int64_t total = (int64_t)(hq + hkv) * nblk;
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 2 * (int64_t)h->num_sms));
-  pool_project_kernel<T, D><<<grid, kPoolWarps * 32, 0, st>>>(q, k, n, hq, hkv, B, nblk, h->sign, h->col, h->scale,
-                                                              h->cfg.sketch_dim, q_sk, k_sk);
+  {
+    const cudaError_t le = launch_k(pool_project_kernel<T, D>, grid, kPoolWarps * 32, 0, st, q, k, n, hq, hkv, B, nblk,
+                                    h->sign, h->col, h->scale, h->cfg.sketch_dim, q_sk, k_sk);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -268,7 +275,11 @@ cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const 
   const int64_t nt = ceil_div64(b, kST);
   dim3 grid(static_cast<unsigned>(nt * (nt + 1) / 2), hq);
   const int32_t k = h->cfg.sketch_dim;
-  scores_kernel<<<grid, 64, 0, st>>>(q_sk, k_sk, b, hq, hq / hkv, k, 1.0 / sqrt((double)k), scores);
+  {
+    const cudaError_t le = launch_k(scores_kernel, grid, 64, 0, st, q_sk, k_sk, b, hq, hq / hkv, k,
+                                    1.0 / sqrt((double)k), scores);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }

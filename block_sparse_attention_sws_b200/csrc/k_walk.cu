@@ -26,6 +26,8 @@ constexpr int kSoftmaxPerLane = 32;  // rows up to 1024 blocks wide
 
 __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __restrict__ S, int64_t b, int64_t rows,
                                                             double temp, double* __restrict__ A) {
+  grid_dependency_wait();
+  allow_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -63,6 +65,8 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
 // the row, the exponentials recomputed for the normalisation.
 __global__ void __launch_bounds__(256) block_softmax_wide_kernel(const double* __restrict__ S, int64_t b,
                                                                  int64_t rows, double temp, double* __restrict__ A) {
+  grid_dependency_wait();
+  allow_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -217,6 +221,8 @@ __device__ __forceinline__ void tile_products(const double* __restrict__ Ah, con
 __global__ void __launch_bounds__(kGemmThreads, 3) tri_gemm_kernel(const double* __restrict__ A,
                                                                 const double* __restrict__ Bm,
                                                                 double* __restrict__ C, int64_t b, int32_t hq) {
+  grid_dependency_wait();
+  allow_dependents();
   __shared__ __align__(16) double part[kGemmWarps][kTT][kPartLd];
   const int64_t nt = ceil_div64(b, kTT);
   const int64_t head = blockIdx.x % hq;  // tile-major: every head's heaviest tile first
@@ -287,6 +293,8 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
                                                      int32_t G, int32_t num, int32_t den, int64_t nnz,
                                                      double* __restrict__ walk_state, int32_t* __restrict__ row_ptr,
                                                      int32_t* __restrict__ col_idx, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
   extern __shared__ __align__(16) uint64_t keys_all[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
@@ -332,9 +340,15 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
   const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
   const unsigned grid = static_cast<unsigned>(ceil_div64(rows, 8));
   if (b <= 32 * kSoftmaxPerLane)
-    block_softmax_kernel<<<grid, 256, 0, st>>>(scores, b, rows, temp, A);
+    {
+      const cudaError_t le = launch_k(block_softmax_kernel, grid, 256, 0, st, scores, b, rows, temp, A);
+      if (le != cudaSuccess) return le;
+    }
   else
-    block_softmax_wide_kernel<<<grid, 256, 0, st>>>(scores, b, rows, temp, A);
+    {
+      const cudaError_t le = launch_k(block_softmax_wide_kernel, grid, 256, 0, st, scores, b, rows, temp, A);
+      if (le != cudaSuccess) return le;
+    }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -343,7 +357,10 @@ cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_
   const int64_t nt = ceil_div64(b, kTT);
   const int64_t ctas = nt * (nt + 1) / 2 * hq;  // one CTA per tile
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-  tri_gemm_kernel<<<static_cast<unsigned>(ctas), kGemmThreads, 0, st>>>(A, Bm, C, b, hq);
+  {
+    const cudaError_t le = launch_k(tri_gemm_kernel, static_cast<unsigned>(ctas), kGemmThreads, 0, st, A, Bm, C, b, hq);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -358,8 +375,12 @@ cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32
   if (e != cudaSuccess) return e;
   int64_t nnz = 0;
   for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
-  select_kernel<<<static_cast<unsigned>(ceil_div64(rows, warps)), warps * 32, smem, st>>>(
-      R, b, rows, G, h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
+  {
+    const cudaError_t le = launch_k(select_kernel, static_cast<unsigned>(ceil_div64(rows, warps)), warps * 32, smem, st,
+                                    R, b, rows, G,
+                                    h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "sws.h"
 
 struct sws_handle {
@@ -35,6 +37,18 @@ enum Guard : int32_t {
 __device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
+
+// ---- programmatic dependent launch ------------------------------------------
+// Every kernel of the library is launched with programmatic stream
+// serialisation (launch_k below), so that it can be scheduled while the
+// previous kernel of the stream drains. Each kernel therefore calls
+// grid_dependency_wait() before its first access to global memory (the wait
+// returns once the previous grid has completed and its writes are visible; it
+// is a no-op when there is no such grid), and allow_dependents() once it has
+// started, which lets the next kernel be scheduled when every CTA of this one
+// has issued it or exited.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- mbarrier / bulk-copy helpers (sm_90+ PTX, used on sm_100a) -------------
 
@@ -142,6 +156,23 @@ __host__ __device__ __forceinline__ int32_t tau_of_row(int64_t i, int32_t num, i
 
 // Counts queued kernels (sws_launch_count); every launcher calls it per launch.
 void note_launches(int count);
+
+// Launches kern<<<grid, block, smem, st>>>(args...) with programmatic stream
+// serialisation allowed (see grid_dependency_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
 
 size_t sketch_workspace_bytes(const sws_config& c, int64_t n, int32_t hq, int32_t hkv);
 cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
