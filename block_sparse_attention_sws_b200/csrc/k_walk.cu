@@ -24,6 +24,7 @@ namespace {
 // sum and the normalisation, so every entry takes one exponential.
 constexpr int kSoftmaxPerLane = 32;  // rows up to 1024 blocks wide
 
+template <int PL>  // entries per lane: rows up to 32 PL blocks wide
 __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __restrict__ S, int64_t b, int64_t rows,
                                                             double temp, double* __restrict__ A) {
   grid_dependency_wait();
@@ -34,10 +35,10 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   const int64_t i = row % b;
   const double* s = S + row * b;
   double* a = A + row * b;
-  double x[kSoftmaxPerLane];
+  double x[PL];
   double mx = -INFINITY;
 #pragma unroll
-  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+  for (int u = 0; u < PL; ++u) {
     const int64_t j = lane + 32 * u;
     x[u] = j <= i ? temp * s[j] : -INFINITY;
     mx = fmax(mx, x[u]);
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   double sum = 0.0;
 #pragma unroll
-  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+  for (int u = 0; u < PL; ++u) {
     if (32 * u > i) break;  // warp-uniform: no entry j <= i left for any lane
     x[u] = exp(x[u] - mx);  // exp(-inf) = 0 for j > i
     sum += x[u];
@@ -55,7 +56,7 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const double* __rest
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   const double inv = 1.0 / sum;
 #pragma unroll
-  for (int u = 0; u < kSoftmaxPerLane; ++u) {
+  for (int u = 0; u < PL; ++u) {
     const int64_t j = lane + 32 * u;
     if (j < b) a[j] = j <= i ? x[u] * inv : 0.0;
   }
@@ -332,6 +333,74 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
     for (int t = lane; t < tau; t += 32) col_idx[(h0 + q) * nnz + rp + t] = out0[t];
 }
 
+// select_kernel for rows of at most 32 PL blocks: the row is loaded into
+// registers with all its loads in flight before its keys go to shared memory
+// for the radix select, and the row's CSR offset is summed in 32-bit
+// arithmetic when it fits.
+template <int PL>
+__global__ void __launch_bounds__(256) select_reg_kernel(const double* __restrict__ R, int64_t b, int64_t rows,
+                                                         int32_t G, int32_t num, int32_t den, int64_t nnz, int tau32,
+                                                         double* __restrict__ walk_state, int32_t* __restrict__ row_ptr,
+                                                         int32_t* __restrict__ col_idx, int32_t* err) {
+  grid_dependency_wait();
+  allow_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const int64_t grp = row / b, i = row % b;
+  const int64_t h0 = grp * G;  // first head of the row's group
+  extern __shared__ __align__(16) uint64_t keys_all[];
+  uint64_t* keys = keys_all + (size_t)warp * b;
+  int* hist = reinterpret_cast<int*>(keys_all + (size_t)(blockDim.x >> 5) * b) + warp * 256;
+  double sum[PL];
+  for (int q = 0; q < G; ++q) {
+    const int64_t off = ((h0 + q) * b + i) * b;
+    double x[PL];
+#pragma unroll
+    for (int u = 0; u < PL; ++u) {
+      const int64_t j = lane + 32 * u;
+      x[u] = j <= i ? R[off + j] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < PL; ++u) {
+      const int64_t j = lane + 32 * u;
+      if (j < b) walk_state[off + j] = x[u];
+      sum[u] = q == 0 ? x[u] : sum[u] + x[u];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < PL; ++u) {
+    const int64_t j = lane + 32 * u;
+    if (j <= i) keys[j] = order_key(sum[u]);
+  }
+  // the CSR offset of row i: the sum of tau over the rows before it, in
+  // 32-bit arithmetic when b * num + den fits (the launcher checks)
+  int64_t rp = 0;
+  if (tau32) {
+    uint32_t r32 = 0;
+    for (uint32_t q = lane; q < static_cast<uint32_t>(i); q += 32)
+      r32 += ((q + 1u) * static_cast<uint32_t>(num) + static_cast<uint32_t>(den) - 1u) / static_cast<uint32_t>(den);
+    rp = __reduce_add_sync(0xffffffffu, r32);
+  } else {
+    for (int64_t q = lane; q < i; q += 32) rp += tau_of_row(q, num, den);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) rp += __shfl_xor_sync(0xffffffffu, rp, off);
+  }
+  const int tau = tau_of_row(i, num, den);
+  if (lane == 0) {
+    for (int q = 0; q < G; ++q) {
+      row_ptr[(h0 + q) * (b + 1) + i] = static_cast<int32_t>(rp);
+      if (i == b - 1) row_ptr[(h0 + q) * (b + 1) + b] = static_cast<int32_t>(rp + tau);
+    }
+  }
+  __syncwarp();
+  int32_t* out0 = col_idx + h0 * nnz + rp;
+  warp_top_tau8(keys, static_cast<int>(i + 1), tau, out0, hist, err);
+  __syncwarp();  // the first head's row is written: the others copy it
+  for (int q = 1; q < G; ++q)
+    for (int t = lane; t < tau; t += 32) col_idx[(h0 + q) * nnz + rp + t] = out0[t];
+}
+
 }  // namespace
 
 cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int64_t b, int32_t hq, double* A,
@@ -339,16 +408,15 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
   const int64_t rows = (int64_t)hq * b;
   const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
   const unsigned grid = static_cast<unsigned>(ceil_div64(rows, 8));
-  if (b <= 32 * kSoftmaxPerLane)
-    {
-      const cudaError_t le = launch_k(block_softmax_kernel, grid, 256, 0, st, scores, b, rows, temp, A);
-      if (le != cudaSuccess) return le;
-    }
-  else
-    {
-      const cudaError_t le = launch_k(block_softmax_wide_kernel, grid, 256, 0, st, scores, b, rows, temp, A);
-      if (le != cudaSuccess) return le;
-    }
+  // the fewest registers per lane that hold a row: more warps per SM
+  auto kern = b <= 256 ? block_softmax_kernel<8>
+              : b <= 512 ? block_softmax_kernel<16>
+              : b <= 32 * kSoftmaxPerLane ? block_softmax_kernel<kSoftmaxPerLane>
+                                          : block_softmax_wide_kernel;
+  {
+    const cudaError_t le = launch_k(kern, grid, 256, 0, st, scores, b, rows, temp, A);
+    if (le != cudaSuccess) return le;
+  }
   note_launches(1);
   return cudaGetLastError();
 }
@@ -369,16 +437,33 @@ cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32
                           int32_t* row_ptr, int32_t* col_idx, cudaStream_t st) {
   const int32_t G = h->cfg.select_group > 1 ? h->cfg.select_group : 1;
   const int64_t rows = (int64_t)(hq / G) * b;
+  int64_t nnz = 0;
+  for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
+  if (b <= 1024) {  // the row fits in registers
+    auto kern = b <= 256 ? select_reg_kernel<8> : b <= 512 ? select_reg_kernel<16> : select_reg_kernel<32>;
+    const size_t smem = 8 * (b * sizeof(uint64_t) + 256 * sizeof(int));
+    const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (ea != cudaSuccess) return ea;
+    // every tau and the row sums fit in 32 bits: (b + 1) num + den and nnz below 2^32
+    const int tau32 = ((b + 1) * (int64_t)h->cfg.density_num + h->cfg.density_den < (int64_t(1) << 32) &&
+                       nnz < (int64_t(1) << 32))
+                          ? 1
+                          : 0;
+    const cudaError_t le = launch_k(kern, static_cast<unsigned>(ceil_div64(rows, 8)), 256, smem, st, R, b, rows, G,
+                                    h->cfg.density_num, h->cfg.density_den, nnz, tau32, walk_state, row_ptr, col_idx,
+                                    h->err);
+    if (le != cudaSuccess) return le;
+    note_launches(1);
+    return cudaGetLastError();
+  }
   int warps = static_cast<int>(std::min<int64_t>(8, std::max<int64_t>(1, (160 << 10) / (b * 8))));
   const size_t smem = (size_t)warps * (b * sizeof(uint64_t) + 256 * sizeof(int));
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int64_t nnz = 0;
-  for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
   {
     const cudaError_t le = launch_k(select_kernel, static_cast<unsigned>(ceil_div64(rows, warps)), warps * 32, smem, st,
-                                    R, b, rows, G,
-                                    h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr, col_idx, h->err);
+                                    R, b, rows, G, h->cfg.density_num, h->cfg.density_den, nnz, walk_state, row_ptr,
+                                    col_idx, h->err);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);
