@@ -28,7 +28,7 @@ EXPORTS = [
     "sws_sync_check", "sws_sketch",
     "sws_walk_select", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
     "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc", "sws_decode_init_cache_paged", "sws_decode_step_paged",
-    "sws_sparse_attn_decode_paged",
+    "sws_sparse_attn_decode_paged", "sws_decode_step_exact",
 ]
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SWS_NOALLOC_SCRATCH_BYTES
 
@@ -81,6 +81,8 @@ def load() -> ctypes.CDLL:
         "sws_sparse_attn_decode": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, SZ, P]),
         "sws_sparse_attn_decode_noalloc": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P]),
         "sws_decode_init_cache_paged": (ctypes.c_int, [P, P, I64, P, I64, I32, I32, P, P, P, P]),
+        "sws_decode_step_exact": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, P, ctypes.c_int,
+                                                 P, P, P, P, P, P, P]),
         "sws_decode_step_paged": (ctypes.c_int, [P, P, P, P, I32, I32, I32, P, P, I64, P, I64, P, P, P, ctypes.c_int,
                                                  P, P, P, P, P, P, P]),
         "sws_sparse_attn_decode_paged": (ctypes.c_int, [P, P, P, P, I64, P, I64, I32, I32, I32, P, P, P, P, P, P, SZ,
@@ -308,3 +310,17 @@ def sws_sparse_attn_decode_paged(h: Handle, q_tok, k_pages, v_pages, block_table
                                                _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt), _ptr(o), _ptr(ws),
                                                ws.numel() * ws.element_size(), _stream(stream)),
            "sws_sparse_attn_decode_paged")
+
+
+# ------------------------------------------------------ exact decode walk ----
+
+def sws_decode_step_exact(h: Handle, q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch, q_psum,
+                          q_sketch, first_layer: bool, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                          stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    hkv, max_len = k_cache.shape[1], k_cache.shape[2]
+    _check(load().sws_decode_step_exact(h.ptr, _ptr(q_tok), _ptr(k_tok), _ptr(v_tok), batch, hq, hkv, max_len,
+                                        _ptr(seq_lens), _ptr(k_cache), _ptr(v_cache), _ptr(k_psum), _ptr(k_sketch),
+                                        _ptr(q_psum), _ptr(q_sketch), int(bool(first_layer)), _ptr(walk_state),
+                                        _ptr(head_sel), _ptr(head_cnt), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
+                                        _stream(stream)), "sws_decode_step_exact")

@@ -166,4 +166,110 @@ __device__ __forceinline__ void warp_top_tau8(const uint64_t* keys, int m, int t
   if (lane == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
 }
 
+// ---- helpers shared by the decode-side kernels ------------------------------
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Output o of a length-D row times H_d, computed by one warp: lane l sums the
+// terms t = l, l + 32, ..., then a shuffle tree adds the lanes.
+template <int D>
+__device__ __forceinline__ double warp_dot_hdt(const double* row_smem, const double* __restrict__ hdt_row, int lane) {
+  double a = 0.0;
+#pragma unroll
+  for (int t = lane; t < D; t += 32) a = fma(row_smem[t], __ldg(hdt_row + t), a);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+  return a;
+}
+
+// Exact top-tau of keys[0, m) (ties to the lower index) by nthr threads (whole
+// warps, the first of them warp `w0`) that share named barrier `bar_id`:
+// eight passes of an 8-bit radix select on the 64-bit keys (a 256-bin shared
+// histogram of the keys that still match the prefix found so far), then an
+// ordered compaction by the first warp that writes the chosen indices
+// ascending to out[] and ORs `bit` into mark[j].
+__device__ inline void group_top_tau(const uint64_t* keys, int m, int tau, int* hist, int* ctl, int t, int nthr,
+                                     int bar_id, int32_t* out, uint32_t* mark, uint32_t bit, int32_t* err) {
+  uint64_t prefix = 0, pm = 0;
+  int need = tau;
+  bool all_cands = false;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int x = t; x < 256; x += nthr) hist[x] = 0;
+    if (t == 0) ctl[0] = ctl[1] = ctl[2] = 0;
+    named_bar(bar_id, nthr);
+    for (int j = t; j < m; j += nthr) {
+      const uint64_t key = keys[j];
+      if ((key & pm) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    named_bar(bar_id, nthr);
+    if (t < 32) {
+      // lane l owns bins 255 - 8l - u, u = 0..7 (descending key order)
+      int c[8], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        c[u] = hist[255 - 8 * t - u];
+        sum += c[u];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (t >= off) incl += y;
+      }
+      const int excl = incl - sum;
+      if (excl < need && need <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (run + c[u] >= need) {
+            ctl[0] = 255 - 8 * t - u;
+            ctl[1] = need - run;
+            ctl[2] = c[u];
+            break;
+          }
+          run += c[u];
+        }
+      }
+    }
+    named_bar(bar_id, nthr);
+    const int digit = ctl[0];
+    need = ctl[1];
+    const int cnt = ctl[2];
+    prefix |= static_cast<uint64_t>(digit) << shift;
+    pm |= 255ull << shift;
+    named_bar(bar_id, nthr);  // ctl and hist are rewritten by the next pass
+    if (cnt == need) {
+      all_cands = true;
+      break;
+    }
+  }
+  if (t >= 32) return;
+  const unsigned lt = lanemask_lt();
+  int base = 0, ties = 0;
+  for (int j0 = 0; j0 < m; j0 += 32) {
+    const int j = j0 + t;
+    const bool valid = j < m;
+    const uint64_t km = valid ? (keys[j] & pm) : 0;
+    const bool above = valid && km > prefix;
+    const bool cand = valid && km == prefix;
+    const unsigned cb = __ballot_sync(0xffffffffu, cand);
+    bool take = cand;
+    if (!all_cands) {
+      take = cand && (ties + __popc(cb & lt)) < need;
+      ties += __popc(cb);
+    }
+    const bool sel = above || take;
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = base + __popc(sb & lt);
+      if (pos < tau) out[pos] = j;
+      atomicOr(&mark[j], bit);
+    }
+    base += __popc(sb);
+  }
+  if (t == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
+}
+
 }  // namespace sws

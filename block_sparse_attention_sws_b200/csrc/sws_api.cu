@@ -441,6 +441,28 @@ sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k
                      stream);
 }
 
+sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                 int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
+                                 void* k_cache, void* v_cache, double* k_psum, double* k_sketch, double* q_psum,
+                                 double* q_sketch, int first_layer, double* walk_state, int32_t* head_sel,
+                                 int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
+  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.select_group > 1 && h->cfg.select_group != hq / hkv) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.walk_mode != SWS_WALK_MATRIX_POWER) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch, q_psum, q_sketch,
+                        walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  if (!decode_exact_supported(h->cfg, ceil_div64(max_len, h->cfg.block_size), hq / hkv)) return SWS_ERR_UNSUPPORTED;
+  return cuda_status(
+      launch_decode_exact(h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_tok),
+                          static_cast<const __nv_bfloat16*>(v_tok), batch, hq, hkv, max_len, seq_lens,
+                          static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), k_psum, k_sketch,
+                          q_psum, q_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
+                          static_cast<cudaStream_t>(stream)),
+      "decode step (exact walk)");
+}
+
 sws_status sws_decode_step_paged(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
                                  int32_t batch, int32_t hq, int32_t hkv, void* k_pages, void* v_pages,
                                  int64_t num_pages, const int32_t* block_table, int64_t max_blocks,

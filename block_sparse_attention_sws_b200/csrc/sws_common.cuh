@@ -236,6 +236,14 @@ cudaError_t launch_decode_select(const sws_handle* h, const __nv_bfloat16* q_tok
                                  double* k_psum, double* k_sketch, int first_layer, double* walk_state,
                                  int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
                                  int32_t* sel_cnt, cudaStream_t st);
+cudaError_t launch_decode_exact(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
+                                const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                const int32_t* seq_lens, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
+                                double* k_psum, double* k_sketch, double* q_psum, double* q_sketch, int first_layer,
+                                double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
+                                uint8_t* sel_mask, int32_t* sel_cnt, cudaStream_t st);
+size_t decode_exact_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
+bool decode_exact_supported(const sws_config& cfg, int64_t max_blocks, int32_t group);
 int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group);
 size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
 cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,

@@ -84,6 +84,10 @@ class DecodePath:
     sws_decode_step -> sws_sparse_attn_decode for each layer, then
     sws_decode_advance once the step's layers are done.
 
+    exact=True selects with the exact decode walk (sws_decode_step_exact): the
+    row of the new token's block in the prefill recurrence, which needs the
+    prompt's query sketches (init_queries) next to the key sketches.
+
     paged=True keeps each layer's keys and values in a pool of pages
     [num_pages, hkv, B, d] addressed through block_table [batch, max_blocks]
     (shared by the layers) and calls the *_paged entry points. The default
@@ -92,7 +96,7 @@ class DecodePath:
     pages before writing the caches."""
 
     def __init__(self, handle: L.Handle, batch: int, hq: int, hkv: int, max_len: int, layers: int, device="cuda",
-                 paged=False, num_pages=None):
+                 paged=False, num_pages=None, exact=False):
         cfg = handle.cfg
         self.h, self.batch, self.hq, self.hkv, self.max_len, self.layers = handle, batch, hq, hkv, max_len, layers
         d, k, B = cfg.head_dim, cfg.sketch_dim, cfg.block_size
@@ -112,6 +116,11 @@ class DecodePath:
             self.v_cache = [torch.empty(batch, hkv, max_len, d, **bf) for _ in range(layers)]
         self.k_psum = [torch.zeros(batch, hkv, d, **f64) for _ in range(layers)]
         self.k_sketch = [torch.zeros(batch, hkv, self.mb, k, **f64) for _ in range(layers)]
+        self.exact = exact
+        if exact:  # the exact walk's cached query sketches (see init_queries)
+            assert not paged, "the exact walk runs on the contiguous cache"
+            self.q_psum = [torch.zeros(batch, hq, d, **f64) for _ in range(layers)]
+            self.q_sketch = [torch.zeros(batch, hq, self.mb, k, **f64) for _ in range(layers)]
         self.seq_lens = torch.zeros(batch, **i32)
         self.walk_state = torch.zeros(batch, hq, self.mb, **f64)
         self.head_sel = torch.zeros(batch, hq, self.mb, **i32)
@@ -173,11 +182,26 @@ class DecodePath:
                 L.sws_decode_init_cache(self.h, self.k_cache[layer], self.seq_lens, self.k_psum[layer],
                                         self.k_sketch[layer], stream)
 
+    def init_queries(self, layer: int, q_prompt, stream=None):
+        """Exact walk: the prompt's queries q_prompt [batch, hq, max_len, d] bf16
+        (rows below the lengths given to init_cache are read) give every cached
+        block's q~ and the last block's query sum, as a prefill would."""
+        assert self.exact and tuple(q_prompt.shape[:3]) == (self.batch, self.hq, self.max_len)
+        L.sws_decode_init_cache(self.h, q_prompt, self.seq_lens, self.q_psum[layer], self.q_sketch[layer], stream)
+
     def begin_step(self, stream=None):
         L.sws_decode_advance(self.h, self.seq_lens, stream)
 
     def layer(self, layer: int, q_tok, k_tok, v_tok, out=None, stream=None):
         o = self.o if out is None else out
+        if self.exact:
+            L.sws_decode_step_exact(self.h, q_tok, k_tok, v_tok, self.seq_lens, self.k_cache[layer],
+                                    self.v_cache[layer], self.k_psum[layer], self.k_sketch[layer], self.q_psum[layer],
+                                    self.q_sketch[layer], layer == 0, self.walk_state, self.head_sel, self.head_cnt,
+                                    self.sel, self.sel_mask, self.sel_cnt, stream)
+            L.sws_sparse_attn_decode(self.h, q_tok, self.k_cache[layer], self.v_cache[layer], self.seq_lens,
+                                     self.sel, self.sel_mask, self.sel_cnt, o, self.ws, stream)
+            return o
         if self.paged:
             L.sws_decode_step_paged(self.h, q_tok, k_tok, v_tok, self.k_cache[layer], self.v_cache[layer],
                                     self.block_table, self.seq_lens, self.k_psum[layer], self.k_sketch[layer],

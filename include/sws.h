@@ -200,6 +200,28 @@ sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k
                            double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
                            uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
 
+/* The decode selection without the log-domain reduction: the row of the new token's
+ * query block in the prefill recurrence of §4, R^l[i] = R^{l-1}[i] (A^l)^s, on the
+ * sequence as it stands (prompt and decoded tokens). Over the layers of a step the row
+ * is carried in walk_state (a probability row, not logarithms; do not mix with
+ * sws_decode_step within a step) and advanced by s vector-matrix products with A^l,
+ * the causal row softmax of q~_m . k~_j / sqrt(k) over every cached query and key block.
+ * The selection then equals that of sws_walk_select for the last query block of a
+ * prefill of the same tokens. It costs O(s b^2) per head and layer.
+ *   q_psum   [batch, hq, d] double: sum of the queries of the last block
+ *   q_sketch [batch, hq, max_blocks, k] double: q~ of every block (the prefill's q_sk)
+ * Initialise both by calling sws_decode_init_cache on the prompt's queries, laid out
+ * [batch, hq, max_len, d] with hkv = hq, next to the same call on the key cache. Other
+ * arguments as sws_decode_step. Requires sketch_dim <= 32, max_blocks <= 1024 and the
+ * per-CTA shared memory (a float triangle of max_blocks rows) to fit in 227 KB, which
+ * holds to about max_blocks = 280 at a GQA group of 4; otherwise SWS_ERR_UNSUPPORTED.
+ * Matrix-power walks only (SWS_ERR_UNSUPPORTED for SWS_WALK_ELEMENTWISE). */
+sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                 int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
+                                 void* k_cache, void* v_cache, double* k_psum, double* k_sketch, double* q_psum,
+                                 double* q_sketch, int first_layer, double* walk_state, int32_t* head_sel,
+                                 int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
+
 /* sw_sparse_attn_decode: one query token per (sequence, head) over the tokens
  * (< seq_lens[i]) of the blocks its head selected. Each KV block of the group's union is
  * read once for all the group's heads (split over the union, then combined).

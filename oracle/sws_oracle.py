@@ -420,6 +420,31 @@ def decode_layer_select(q_tok, Kcaches, length: int, Hd, B: int, s: int, density
     return rho, z, sel
 
 
+def decode_exact_layer(Q, K, Hd, B: int, s: int, density: Tuple[int, int], state: PrefillState,
+                       heads: Optional[Sequence[int]] = None, select: str = "per_head"):
+    """Exact decode walk, one layer (an extension of §5, the "next" row that
+    replaces reading R7's log-domain reduction): the newest token's selection
+    is the row of its query block i = ceil(n/B) - 1 in the walk state R^l of
+    §4, computed by the prefill recurrence on the sequence as it stands.
+
+    Q [hq, n, d] holds the queries of every position so far (prompt and
+    decoded tokens), K [hkv, n, d] the keys. ``state`` carries R over the
+    layers of one decode step (a fresh PrefillState per step: the query block
+    i changes from step to step). Returns per head: ``row`` = R^l[i, :i+1],
+    ``blocks`` = the chosen blocks (ascending) and ``score`` = what they were
+    chosen on (R^l[i], or the group's summed rows for a group-shared choice).
+    """
+    res = prefill_layer(Q, K, K, Hd, B, s, density, state, heads=heads, attention_blocks=None, select=select)
+    out = {}
+    for h, r in res.items():
+        R = r["R"]
+        i = R.shape[0] - 1
+        rp, ci = r["row_ptr"], r["col_idx"]
+        score = r["shared_scores"][i] if select == "group_shared" else R[i]
+        out[h] = dict(row=R[i, :i + 1].copy(), blocks=ci[rp[i]:rp[i + 1]].copy(), score=score[:i + 1].copy())
+    return out
+
+
 def decode_attention(q_tok, Kcache, Vcache, length: int, blocks: Sequence[int], B: int) -> np.ndarray:
     """One query row (the token at position length-1) over the tokens of the
     selected blocks that lie below ``length``; textbook two-pass softmax."""

@@ -34,7 +34,7 @@ import torch
 
 _M64 = (1 << 64) - 1
 
-KIND_Q, KIND_K, KIND_V, KIND_HUB_POS, KIND_HUB_OFF, KIND_QDEC = range(6)
+KIND_Q, KIND_K, KIND_V, KIND_HUB_POS, KIND_HUB_OFF, KIND_QDEC, KIND_QSEQ = range(7)
 
 
 def _mix64(x: int) -> int:
@@ -239,4 +239,24 @@ def decode_queries(w: DecodeWorkload, seq: int, layer: int, device="cpu"):
     Q = torch.empty(w.hq, w.steps, w.d, dtype=out_dt, device=device)
     for h in range(w.hq):
         Q[h] = ar1(w.steps, w.d, w.rho, _gen(device, stream_seed(w.seed, layer, KIND_QDEC, h, seq)), device).to(out_dt)
+    return Q
+
+
+def decode_sequence_queries(w: DecodeWorkload, seq: int, layer: int, device="cpu"):
+    """Q [hq, n0 + steps, d]: the queries of every position of one sequence and
+    layer, prompt and decoded tokens alike (for a decode that needs the prompt's
+    queries too); the same AR(1), sink and hub structure as the keys of the
+    query head's group."""
+    out_dt = _dtype(w.dtype)
+    L = w.max_len
+    b0 = -(-w.n0 // w.B)
+    group = w.hq // w.hkv
+    Q = torch.empty(w.hq, L, w.d, dtype=out_dt, device=device)
+    for g in range(w.hkv):
+        pos, off = hub_layout(b0, w.hubs, w.d, w.seed, layer, g, device, seq)
+        for h in range(g * group, (g + 1) * group):
+            qx = ar1(L, w.d, w.rho, _gen(device, stream_seed(w.seed, layer, KIND_QSEQ, h, seq)), device)
+            _add_structure(qx, w.B, pos, off)
+            Q[h] = qx.to(out_dt)
+            del qx
     return Q

@@ -361,6 +361,38 @@ def pin_group_shared_decode():
     assert np.array_equal(a[0], a[1]) and np.array_equal(a[2], a[3])
 
 
+def pin_exact_decode():
+    """Exact decode walk: the newest block's row of the prefill recurrence.
+    (1) With s = 1 and one layer, when the newest block holds only the new
+    token, the row is the softmax of the row logits: exp of the log-domain
+    decode's rho (a separate route, from the token's own query). (2) Over
+    layers the row stays a probability row. (3) Brute force: e_i times
+    numpy's matrix_power of each layer's block attention, multiplied out."""
+    hq, hkv, d, B, k = 2, 1, 8, 4, 4
+    n = 17  # block 4 holds position 16 only
+    Hd = so.srht_matrix(d, k, 5)
+    Qs = [rng.standard_normal((hq, n, d)) for _ in range(3)]
+    Ks = [rng.standard_normal((hkv, n, d)) for _ in range(3)]
+    one = so.decode_exact_layer(Qs[0], Ks[0], Hd, B, 1, (2, 5), so.PrefillState())
+    rho1, _, sel1 = so.decode_layer_select(Qs[0][:, n - 1], Ks[0], n, Hd, B, 1, (2, 5), None)
+    for h in range(hq):
+        assert np.allclose(one[h]["row"], np.exp(rho1[h]), rtol=1e-12, atol=1e-15)
+        assert np.array_equal(one[h]["blocks"], sel1[h])
+    st = so.PrefillState()
+    rows = [so.decode_exact_layer(Qs[l], Ks[l], Hd, B, 3, (2, 5), st) for l in range(3)]
+    nb = -(-n // B)
+    for h in range(hq):
+        u = np.eye(nb)[nb - 1]
+        for l in range(3):
+            A = so.block_attention(so.sketch_scores(so.sketch_project(so.block_means(Qs[l][h], B), Hd),
+                                                    so.sketch_project(so.block_means(Ks[l][0], B), Hd)))
+            u = u @ np.linalg.matrix_power(A, 3)
+            got = rows[l][h]["row"]
+            assert np.all(got >= 0) and abs(got.sum() - 1.0) < 1e-12
+            assert np.allclose(got, u, rtol=1e-12, atol=1e-15)
+            assert np.array_equal(rows[l][h]["blocks"], so.top_tau_row(u, so.tau_of_row(nb - 1, 2, 5)))
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -404,6 +436,13 @@ PLANTED = {
         lambda Q, K, V, i, blocks, B: orig(np.asarray(Q) / math.sqrt(Q.shape[1]), K, V, i, blocks, B)),
         pin_attention_dense_limit),
 }
+
+
+PLANTED["exact_decode_previous_block_row"] = (
+    "decode_exact_layer", lambda orig: (lambda Q, K, Hd, B, s, density, state, heads=None, select="per_head": {
+        h: dict(r, row=np.append(state.R[h][-2, :-1], 0.0)) for h, r in orig(Q, K, Hd, B, s, density, state, heads,
+                                                                             select).items()}),
+    pin_exact_decode)
 
 
 @pytest.mark.parametrize("name", sorted(PLANTED))
