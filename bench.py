@@ -588,6 +588,60 @@ def bench_decode(args, world, S, W, torch, peaks):
     return out
 
 
+def bench_decode_exact(args, world, S, W, torch):
+    """The exact decode walk (sws_decode_step_exact) against the log-domain walk
+    (sws_decode_step) on one workload its shared-memory triangle holds: the
+    decode workload's shape at a 16K-token prompt. Same caches, tokens and
+    step count for both; each step is all layers' selection and attention."""
+    wd = W.DECODE_128K.scaled(n0=16384, steps=max(4, min(16, args.decode_steps or 16)))
+    cfg = S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed)
+    h = S.Handle(cfg)
+    path = S.DecodePath(h, wd.batch, wd.hq, wd.hkv, wd.max_len, wd.layers, exact=True)
+    toks_k = torch.empty(wd.steps, wd.layers, wd.batch, wd.hkv, wd.d, dtype=torch.bfloat16, device="cuda")
+    toks_v = torch.empty_like(toks_k)
+    toks_q = torch.empty(wd.steps, wd.layers, wd.batch, wd.hq, wd.d, dtype=torch.bfloat16, device="cuda")
+    lens = torch.full((wd.batch,), wd.n0, dtype=torch.int32, device="cuda")
+    path.seq_lens.copy_(lens)
+    for layer in range(wd.layers):
+        qp = torch.empty(wd.batch, wd.hq, wd.max_len, wd.d, dtype=torch.bfloat16, device="cuda")
+        for s_ in range(wd.batch):
+            K, V = W.decode_cache_inputs(wd, s_, layer, "cuda")
+            Q = W.decode_sequence_queries(wd, s_, layer, "cuda")
+            path.write_cache(layer, s_, K, V, wd.n0)
+            qp[s_] = Q
+            toks_k[:, layer, s_] = K[:, wd.n0:].transpose(0, 1)
+            toks_v[:, layer, s_] = V[:, wd.n0:].transpose(0, 1)
+            toks_q[:, layer, s_] = Q[:, wd.n0:].transpose(0, 1)
+            del K, V, Q
+        path.init_queries(layer, qp)
+        del qp
+    stream = torch.cuda.current_stream()
+    warm = min(3, wd.steps - 1)
+    timed = wd.steps - warm
+    out = {"workload": wd.name.replace("n131072", "n16384"), "steps_timed": timed}
+    for mode in ("exact_walk", "log_walk"):
+        path.exact = mode == "exact_walk"
+        path.init_cache(lens)  # back to the prompt: the same steps replayed
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        unions = torch.zeros(wd.steps, wd.layers, wd.batch, wd.hkv, dtype=torch.int32, device="cuda")
+        for t in range(wd.steps):
+            if t == warm:
+                barrier(world)
+                torch.cuda.synchronize()
+                a.record(stream)
+            path.begin_step()
+            for layer in range(wd.layers):
+                path.layer(layer, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer])
+                unions[t, layer].copy_(path.sel_cnt, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        ms = max_over_ranks(a.elapsed_time(b), world) / timed
+        out[mode] = {"step_us": ms * 1e3, "union_blocks_per_unit": float(unions[warm:].double().mean().item())}
+    h.close()
+    return out
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
@@ -654,6 +708,10 @@ def main():
     torch.cuda.empty_cache()
     if not args.no_decode:
         line["decode"] = bench_decode(args, world, S, W, torch, peaks)
+        if not args.no_variants:
+            torch.cuda.empty_cache()
+            line["decode"].setdefault("variants", {})["exact_walk_n16384"] = bench_decode_exact(args, world, S, W,
+                                                                                                 torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W.PREFILL_16K)
     if rank == 0:

@@ -12,16 +12,23 @@
 // queries so far, like its key sketch. The row costs O(s b^2) per head and
 // layer, against O(b) for the log-domain walk of sws_decode_step.
 //
-// One CTA of 1024 threads per (sequence, KV head), as in decode_select_kernel:
+// One CTA of 512 threads per (sequence, KV head), as in decode_select_kernel:
 //  1. append the token's K/V, update the key and query block sums and the last
 //     block's k~ and (per query head of the group) q~;
-//  2. stage k~ of every block in shared memory (fp32, rows padded to k + 1);
-//  3. per query head: A as fp32 in shared memory (one warp per row: the scores
-//     on fp32 FMA, the row maximum, exponentials, the row sum in fp64), then
-//     the s products u <- u A in fp64, each column's sum cut into slices of
-//     rows that are added in a fixed order;
-//  4. per head (or per group, for group-shared selection) the top-tau of u,
+//  2. stage k~ of every block in shared memory (fp32); per query head: the
+//     scores S on fp32 FMA (32-column tiles with k~ in registers and q~
+//     broadcast from shared memory) into a triangle of 4-byte slots; per row
+//     the maximum, exponentials, the row sum and the normalisation in fp64,
+//     each entry of A stored back as the rounded high word of its fp64 value;
+//     then the s products u <- u A in fp64, balanced over the triangle by
+//     pairing column j with column nb - 1 - j;
+//  3. per head (or per group, for group-shared selection) the top-tau of u,
 //     then the union over the group with its head mask.
+//
+// Measured at a 16K-token prompt (257 blocks, group of 4): about 38 us of
+// scores and softmax and 33 us of products per head and layer; the products
+// issue about 500 instructions a lane at ~30% issue efficiency with four
+// warps per sub-partition, which the 224 KB of shared memory allows.
 #include <algorithm>
 
 #include "select.cuh"
@@ -30,23 +37,34 @@
 namespace sws {
 namespace {
 
-constexpr int kExThreads = 1024;
+constexpr int kExThreads = 512;  // 16 warps: up to 128 registers a thread
 constexpr int kExWarps = kExThreads / 32;
 constexpr int kExMaxK = 32;     // sketch dims held in registers per lane
-constexpr int kExSlices = 4;    // row slices of one product's column sums
 
 __host__ __device__ constexpr int64_t tri_count(int64_t nb) { return nb * (nb + 1) / 2; }
+__device__ __forceinline__ int tri32(int m) { return (m * (m + 1)) >> 1; }  // m < 2^15
+
+// The normalised block attention is kept as the high 32 bits of its fp64 value
+// (sign, 11-bit exponent, 20-bit mantissa, rounded to nearest): the same 4
+// bytes as an fp32, the fp64 exponent range, a relative precision of 2^-21,
+// and an fp64 operand for the products from a register move, no conversion.
+__device__ __forceinline__ uint32_t to_hi20(double x) {
+  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x)) + 0x80000000ull;
+  return static_cast<uint32_t>(b >> 32);
+}
+__device__ __forceinline__ double from_hi20(uint32_t h) { return __hiloint2double(static_cast<int>(h), 0); }
 
 // Shared-memory carve-up for max_blocks blocks; every part 16-byte aligned.
 struct ExactSmem {
-  int64_t a, ks, u, part, keys, mark, mean, qrow, hist, ctl, wsum, total;
+  int64_t a, qs, ks, u, part, keys, mark, mean, qrow, hist, ctl, wsum, total;
   __host__ __device__ ExactSmem(int64_t mb, int group, int k, int D) {
     auto up = [](int64_t x) { return (x + 15) & ~int64_t(15); };
     a = 0;                                                  // float [tri(mb)]
-    ks = up(a + tri_count(mb) * 4);                         // float [mb][k + 1]
+    qs = up(a + tri_count(mb) * 4);                         // float [mb][k]: one head's q~
+    ks = up(qs + mb * k * 4);                               // float [mb][k + 1]: the KV head's k~
     u = up(ks + mb * (k + 1) * 4);                          // double [2][mb]
-    part = up(u + 2 * mb * 8);                              // double [kExSlices][mb]
-    keys = up(part + kExSlices * mb * 8);                   // uint64 [group][mb] (u rows for a shared choice)
+    part = up(u + 2 * mb * 8);                              // double [mb]
+    keys = up(part + mb * 8);                               // uint64 [group][mb] (u rows for a shared choice)
     mark = up(keys + (int64_t)group * mb * 8);              // uint32 [mb]
     mean = up(mark + mb * 4);                               // double [D]
     qrow = up(mean + D * 8);                                // double [group][D]
@@ -56,6 +74,21 @@ struct ExactSmem {
     total = up(wsum + (kExWarps + 1) * 4);
   }
 };
+
+// sum over m = m0, m0 + step, ... < nb of u[m] A[m][j], in four interleaved
+// chains added in a fixed order (fp64; A from the triangle of high words)
+__device__ __forceinline__ double column_dot(const double* u, const uint32_t* A, int m0, int step, int nb, int j) {
+  double c0 = 0.0, c1 = 0.0, c2 = 0.0, c3 = 0.0;
+  int m = m0;
+  for (; m + 3 * step < nb; m += 4 * step) {
+    c0 = fma(u[m], from_hi20(A[tri32(m) + j]), c0);
+    c1 = fma(u[m + step], from_hi20(A[tri32(m + step) + j]), c1);
+    c2 = fma(u[m + 2 * step], from_hi20(A[tri32(m + 2 * step) + j]), c2);
+    c3 = fma(u[m + 3 * step], from_hi20(A[tri32(m + 3 * step) + j]), c3);
+  }
+  for (; m < nb; m += step) c0 = fma(u[m], from_hi20(A[tri32(m) + j]), c0);
+  return (c0 + c1) + (c2 + c3);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
@@ -72,8 +105,11 @@ __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
   const int group = hq / hkv;
   extern __shared__ __align__(16) uint8_t smem[];
   const ExactSmem L(max_blocks, group, k, D);
-  float* A = reinterpret_cast<float*>(smem + L.a);
+  float* A = reinterpret_cast<float*>(smem + L.a);  // scores, then (as Ah) the attention's high words
+  const uint32_t* Ah = reinterpret_cast<const uint32_t*>(smem + L.a);
+  float* qs = reinterpret_cast<float*>(smem + L.qs);
   float* ks = reinterpret_cast<float*>(smem + L.ks);
+  const int ksp = k + 1;  // padded k~ rows: lanes on consecutive rows read consecutive banks
   double* ubuf = reinterpret_cast<double*>(smem + L.u);
   double* part = reinterpret_cast<double*>(smem + L.part);
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem + L.keys);
@@ -83,7 +119,6 @@ __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
   int* hist = reinterpret_cast<int*>(smem + L.hist);
   int* ctl = reinterpret_cast<int*>(smem + L.ctl);
   int* wsum = reinterpret_cast<int*>(smem + L.wsum);
-  const int ksp = k + 1;  // padded k~ row (floats): lanes on consecutive rows hit consecutive banks
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t unit = blockIdx.x;
@@ -131,33 +166,62 @@ __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
     }
   }
   __syncthreads();  // the CTA's global writes above are visible to it after the barrier
-
-  // 2. k~ of every block, fp32, padded rows
+  // 2. k~ of every block, fp32, in shared memory (coalesced reads; shared by the group's heads)
   for (int x = tid; x < nb * k; x += kExThreads) ks[(x / k) * ksp + x % k] = static_cast<float>(ksk[x]);
-  __syncthreads();
 
   const float inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(k)));
-  const int ntiles = (nb + 31) / 32;
   for (int r = 0; r < group; ++r) {
     const int64_t h = (int64_t)g * group + r;
     const double* qsk = q_sketch + ((int64_t)bi * hq + h) * max_blocks * k;
-    // 3a. A = row softmax of S over j <= m, fp32, row m at offset m (m + 1) / 2
-    for (int m = warp; m < nb; m += kExWarps) {
-      float qv[kExMaxK];
+    // 3a. the scores S_mj, fp32, into the triangle (row m at offset m (m + 1) / 2).
+    //     A warp works down one 32-column tile at a time with its lane's k~_j
+    //     in registers, reading each row's q~ as 16-byte broadcasts from shared
+    //     memory: four FMAs per shared load. The (tile, row) items, rows
+    //     m >= 32 J of tile J, are dealt to the warps in order.
+    for (int x = tid; x < nb * k; x += kExThreads) qs[x] = static_cast<float>(qsk[x]);
+    __syncthreads();
+    {
+      const int ntiles = (nb + 31) / 32;
+      int tile = -1, tile_first = 0;  // the tile of the registers and its first item index
+      float kreg[kExMaxK];
+      int jt = 0, start = 0;          // walking the tiles: tile jt covers items [start, start + nb - 32 jt)
+      for (int x = warp; ; x += kExWarps) {
+        while (jt < ntiles && x >= start + (nb - 32 * jt)) {
+          start += nb - 32 * jt;
+          ++jt;
+        }
+        if (jt >= ntiles) break;
+        if (jt != tile) {
+          tile = jt;
+          tile_first = start;
+          const int j = 32 * tile + lane;
 #pragma unroll
-      for (int c = 0; c < kExMaxK; ++c) qv[c] = c < k ? static_cast<float>(qsk[(int64_t)m * k + c]) : 0.f;
-      float* arow = A + tri_count(m);
-      float mx = -INFINITY;
-      for (int j = lane; j <= m; j += 32) {
-        const float* kr = ks + j * ksp;
+          for (int c = 0; c < kExMaxK; ++c) kreg[c] = (c < k && j < nb) ? ks[j * ksp + c] : 0.f;
+        }
+        const int m = 32 * tile + (x - tile_first);
+        const int j = 32 * tile + lane;
+        const float4* q4 = reinterpret_cast<const float4*>(qs + m * k);
         float sdot = 0.f;
 #pragma unroll
-        for (int c = 0; c < kExMaxK; ++c)
-          if (c < k) sdot = fmaf(qv[c], kr[c], sdot);
-        sdot *= inv_sqrt_k;
-        arow[j] = sdot;
-        mx = fmaxf(mx, sdot);
+        for (int c4 = 0; c4 < kExMaxK / 4; ++c4) {
+          if (4 * c4 < k) {
+            const float4 qv = q4[c4];
+            sdot = fmaf(qv.x, kreg[4 * c4], sdot);
+            sdot = fmaf(qv.y, kreg[4 * c4 + 1], sdot);
+            sdot = fmaf(qv.z, kreg[4 * c4 + 2], sdot);
+            sdot = fmaf(qv.w, kreg[4 * c4 + 3], sdot);
+          }
+        }
+        if (j <= m) A[tri32(m) + j] = sdot * inv_sqrt_k;
       }
+    }
+    __syncthreads();
+    // 3a'. row softmax over j <= m, one warp per row: maximum, exponentials
+    //      (the sum in fp64), normalisation in fp64, stored as high words
+    for (int m = warp; m < nb; m += kExWarps) {
+      float* arow = A + tri32(m);
+      float mx = -INFINITY;
+      for (int j = lane; j <= m; j += 32) mx = fmaxf(mx, arow[j]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       double se = 0.0;
@@ -168,8 +232,9 @@ __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
-      const float inv = static_cast<float>(1.0 / se);
-      for (int j = lane; j <= m; j += 32) arow[j] *= inv;
+      const double inv = 1.0 / se;
+      uint32_t* hrow = reinterpret_cast<uint32_t*>(arow);
+      for (int j = lane; j <= m; j += 32) hrow[j] = to_hi20(static_cast<double>(arow[j]) * inv);
     }
     // 3b. u: e_i on the first layer, else the previous layer's row
     double* u0 = ubuf;
@@ -177,26 +242,30 @@ __global__ void __launch_bounds__(kExThreads) decode_exact_kernel(
     double* wrow = walk_state + ((int64_t)bi * hq + h) * max_blocks;
     for (int j = tid; j < nb; j += kExThreads) u0[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
     __syncthreads();
-    // 3c. s products u <- u A: column j sums u_m A_mj over m >= j; warp w
-    //     takes column tile w % ntiles and the rows of slice w / ntiles
-    const int fit = kExWarps / ntiles;  // >= 1 since nb <= kExThreads
-    const int slices = fit < kExSlices ? (fit < 1 ? 1 : fit) : kExSlices;
-    const int rows_per = (nb + slices - 1) / slices;
+    // 3c. s products u <- u A. Column j sums u_m A_mj over m >= j; columns j
+    //     and nb - 1 - j together have nb + 1 terms, so a group of 4 lanes
+    //     takes such a pair (128 pairs at a time), its lanes striding over the
+    //     rows of both columns in eight chains, and adds its lanes with a fixed
+    //     shuffle tree (the same order on every run).
+    const int npairs = (nb + 1) / 2;
     for (int p = 0; p < s_pow; ++p) {
-      if (warp < ntiles * slices) {
-        const int j = (warp % ntiles) * 32 + lane;
-        const int sl = warp / ntiles;
-        const int m0 = std::max(j, sl * rows_per), m1 = std::min(nb, (sl + 1) * rows_per);
-        double acc = 0.0;
-        if (j < nb)
-          for (int m = m0; m < m1; ++m) acc = fma(u0[m], static_cast<double>(A[tri_count(m) + j]), acc);
-        if (j < nb) part[sl * max_blocks + j] = acc;
-      }
-      __syncthreads();
-      for (int j = tid; j < nb; j += kExThreads) {
-        double acc = part[j];
-        for (int sl = 1; sl < slices; ++sl) acc += part[sl * max_blocks + j];
-        u1[j] = acc;
+      for (int base = warp * 8; base < npairs; base += kExThreads / 4) {  // warp-uniform trip count
+        const int pr = base + (lane >> 2), sub = lane & 3;
+        const int ja = pr, jb = nb - 1 - pr;
+        double acc_a = 0.0, acc_b = 0.0;
+        if (pr < npairs) {
+          acc_a = column_dot(u0, Ah, ja + sub, 4, nb, ja);
+          if (jb != ja) acc_b = column_dot(u0, Ah, jb + sub, 4, nb, jb);
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+          acc_a += __shfl_xor_sync(0xffffffffu, acc_a, off);
+          acc_b += __shfl_xor_sync(0xffffffffu, acc_b, off);
+        }
+        if (pr < npairs && sub == 0) {
+          u1[ja] = acc_a;
+          if (jb != ja) u1[jb] = acc_b;
+        }
       }
       __syncthreads();
       double* t = u0;
@@ -276,7 +345,8 @@ size_t decode_exact_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_
 }
 
 bool decode_exact_supported(const sws_config& cfg, int64_t max_blocks, int32_t group) {
-  return cfg.sketch_dim <= kExMaxK && max_blocks <= kExThreads && group >= 1 && group <= 8 &&
+  return cfg.sketch_dim <= kExMaxK && cfg.sketch_dim % 4 == 0 && max_blocks <= kExThreads && group >= 1 &&
+         group <= 8 &&
          decode_exact_smem_bytes(cfg, max_blocks, group) <= (227u << 10);
 }
 

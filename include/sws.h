@@ -212,9 +212,12 @@ sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k
  *   q_sketch [batch, hq, max_blocks, k] double: q~ of every block (the prefill's q_sk)
  * Initialise both by calling sws_decode_init_cache on the prompt's queries, laid out
  * [batch, hq, max_len, d] with hkv = hq, next to the same call on the key cache. Other
- * arguments as sws_decode_step. Requires sketch_dim <= 32, max_blocks <= 1024 and the
- * per-CTA shared memory (a float triangle of max_blocks rows) to fit in 227 KB, which
- * holds to about max_blocks = 280 at a GQA group of 4; otherwise SWS_ERR_UNSUPPORTED.
+ * arguments as sws_decode_step. Requires sketch_dim <= 32 and a multiple of 4, and the
+ * per-CTA shared memory (a 4-byte triangle of max_blocks rows, one head's q~ and the
+ * KV head's k~) to fit in 227 KB, which holds to about max_blocks = 260 at a GQA group
+ * of 4 and d = 128; otherwise SWS_ERR_UNSUPPORTED. The block attention is held to a
+ * relative 2^-21 (scores in fp32, each entry rounded to a 20-bit mantissa with the
+ * fp64 exponent range); the products accumulate in fp64.
  * Matrix-power walks only (SWS_ERR_UNSUPPORTED for SWS_WALK_ELEMENTWISE). */
 sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
                                  int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
