@@ -159,10 +159,13 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
 
 // S[h, i, j] = q~_i . k~_j / sqrt(k) for j <= i, fp64, on the fp64 tensor path
 // (mma.sync m16n8k4 f64): one 32 x 32 tile on or below the block diagonal per
-// CTA of two warps (each a 16 x 32 slice), the sketch dimension staged 16 at a
-// time through padded shared memory (conflict-free fragment loads, as in the
-// walk's GEMM). Query head h reads the sketches of KV head h / group.
-constexpr int kST = 32, kSC = 16;
+// CTA of two warps (each a 16 x 32 slice). The sketch dimension is staged 32
+// at a time (all of it at k = 32: one round of loads) by cp.async straight
+// into shared memory, both operands row-major with a row stride of 36
+// doubles, which puts every fragment load at the minimum of two wavefronts.
+// Eight CTAs fit per SM, so a layer's tiles run in one wave. Query head h
+// reads the sketches of KV head h / group.
+constexpr int kST = 32, kSC = 32, kSLd = kSC + 4;
 
 __device__ __forceinline__ void dmma_16x8x4_s(double (&c)[4], double a0, double a1, double b0) {
   asm volatile(
@@ -171,13 +174,19 @@ __device__ __forceinline__ void dmma_16x8x4_s(double (&c)[4], double a0, double 
       : "d"(a0), "d"(a1), "d"(b0));
 }
 
-__global__ void __launch_bounds__(64) scores_kernel(const double* __restrict__ q_sk, const double* __restrict__ k_sk,
-                                                    int64_t b, int32_t hq, int32_t group, int32_t k,
-                                                    double inv_sqrt_k, double* __restrict__ S) {
+// 8 bytes global -> shared, asynchronously; zero-filled when !valid
+__device__ __forceinline__ void cp_async8(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 8 : 0)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(64, 8)
+    scores_kernel(const double* __restrict__ q_sk, const double* __restrict__ k_sk, int64_t b, int32_t hq,
+                  int32_t group, int32_t k, double inv_sqrt_k, double* __restrict__ S) {
   grid_dependency_wait();
   allow_dependents();
-  __shared__ __align__(16) double qs[kST][kSC + 4];  // [query block][sketch dim]
-  __shared__ __align__(16) double ks[kSC][kST + 4];  // [sketch dim][key block]
+  __shared__ __align__(16) double qs[kST][kSLd];  // [query block][sketch dim]
+  __shared__ __align__(16) double ks[kST][kSLd];  // [key block][sketch dim]
   const int64_t t = blockIdx.x;
   // tile (ti, tj), tj <= ti, from the linear lower-triangle index
   int64_t ti = static_cast<int64_t>((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
@@ -196,32 +205,28 @@ __global__ void __launch_bounds__(64) scores_kernel(const double* __restrict__ q
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[n8][v] = 0.0;
   for (int c0 = 0; c0 < k; c0 += kSC) {
-    constexpr int kPer = kST * kSC / 64;  // 8 elements of each operand per thread
-    double qv[kPer], kv[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
+    if (c0 > 0) __syncthreads();  // the previous chunk's fragments have been read
+#pragma unroll 4
+    for (int u = 0; u < kST * kSC / 64; ++u) {
       const int e = tid + 64 * u;
-      const int r = e / kSC, c = e % kSC;  // 16 consecutive threads read one row
+      const int r = e / kSC, c = e % kSC;  // a warp copies one row
       const int64_t qi = i0 + r, kj = j0 + r;
-      qv[u] = (qi < b && c0 + c < k) ? qh[qi * k + c0 + c] : 0.0;
-      kv[u] = (kj < b && c0 + c < k) ? kh[kj * k + c0 + c] : 0.0;
+      const bool cok = c0 + c < k;
+      cp_async8(&qs[r][c], (qi < b && cok) ? qh + qi * k + c0 + c : qh, qi < b && cok);
+      cp_async8(&ks[r][c], (kj < b && cok) ? kh + kj * k + c0 + c : kh, kj < b && cok);
     }
-    __syncthreads();  // the previous chunk's fragments have been read
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int e = tid + 64 * u;
-      qs[e / kSC][e % kSC] = qv[u];
-      ks[e % kSC][e / kSC] = kv[u];
-    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < kSC / 4; ++kk) {
       const double a0 = qs[warp * 16 + g][kk * 4 + t4];
       const double a1 = qs[warp * 16 + g + 8][kk * 4 + t4];
 #pragma unroll
-      for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4_s(acc[n8], a0, a1, ks[kk * 4 + t4][n8 * 8 + g]);
+      for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4_s(acc[n8], a0, a1, ks[n8 * 8 + g][kk * 4 + t4]);
     }
   }
+  const bool pairs = (b & 1) == 0;  // 16-byte aligned row starts
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int64_t i = i0 + warp * 16 + g + 8 * hh;
@@ -229,8 +234,14 @@ __global__ void __launch_bounds__(64) scores_kernel(const double* __restrict__ q
 #pragma unroll
     for (int n8 = 0; n8 < 4; ++n8) {
       const int64_t j = j0 + n8 * 8 + 2 * t4;
-      if (j <= i) S[((size_t)h * b + i) * b + j] = acc[n8][2 * hh] * inv_sqrt_k;
-      if (j + 1 <= i) S[((size_t)h * b + i) * b + j + 1] = acc[n8][2 * hh + 1] * inv_sqrt_k;
+      double* dst = S + ((size_t)h * b + i) * b + j;
+      if (pairs && j + 1 <= i) {
+        *reinterpret_cast<double2*>(dst) =
+            make_double2(acc[n8][2 * hh] * inv_sqrt_k, acc[n8][2 * hh + 1] * inv_sqrt_k);
+      } else {
+        if (j <= i) dst[0] = acc[n8][2 * hh] * inv_sqrt_k;
+        if (j + 1 <= i) dst[1] = acc[n8][2 * hh + 1] * inv_sqrt_k;
+      }
     }
   }
 }
