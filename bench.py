@@ -371,6 +371,46 @@ def bench_prefill_variants(args, world, S, W, torch, pf):
         if path.h_dense is not None:
             path.h_dense.close()
         del path
+    out["batch_8x2048"] = bench_prefill_batch(args, world, S, W, torch)
+    return out
+
+
+def bench_prefill_batch(args, world, S, W, torch):
+    """Prefill batching: eight 2048-token sequences of the headline workload's
+    shape (4 layers, 32/8 heads), through PrefillBatch (each sequence's layer
+    on its own stream) and, for comparison, the same paths one after another
+    on one stream."""
+    base = W.PREFILL_16K
+    ws = [base.scaled(name=f"seq{i}", n=2048, seed=base.seed + 100 + i) for i in range(8)]
+    inputs = [[W.prefill_layer_inputs(w, layer, "cuda") for w in ws] for layer in range(base.layers)]
+    h = S.Handle(S.make_config(base.d, base.B, base.k, base.s, 0, base.density, base.seed))
+    batch = S.PrefillBatch(h, [w.n for w in ws], base.hq, base.hkv, torch.bfloat16)
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, 20))
+    out = {"sequences": len(ws), "tokens_per_sequence": 2048, "steps": steps}
+    for mode in ("concurrent_streams", "one_stream"):
+        def step():
+            for layer, ins in enumerate(inputs):
+                if mode == "concurrent_streams":
+                    batch.layer([x[0] for x in ins], [x[1] for x in ins], [x[2] for x in ins], layer == 0)
+                else:
+                    for p, (Q, K, V) in zip(batch.paths, ins):
+                        p.layer(Q, K, V, layer == 0)
+
+        for _ in range(args.warmup):
+            step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        ms = max_over_ranks(a.elapsed_time(b), world) / steps
+        out[mode] = {"tokens_per_s": world * sum(w.n for w in ws) / (ms * 1e-3), "ms_per_step": ms}
+    h.close()
     return out
 
 

@@ -79,6 +79,36 @@ class PrefillPath:
         return self.attention(q, k, v, out, stream, layer)
 
 
+class PrefillBatch:
+    """Prefill of several sequences of different lengths through one handle.
+
+    Each sequence keeps its own PrefillPath (its own walk state and CSR); a
+    layer issues every sequence's sketch, walk and attention on a stream of its
+    own, all ordered after the caller's stream and joined back into it, so the
+    kernels of short sequences overlap on the GPU. Results equal those of the
+    sequences run one by one, bit for bit (tests/test_gpu_prefill.py)."""
+
+    def __init__(self, handle: L.Handle, lengths, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda",
+                 dense_layers: int = 0):
+        self.paths = [PrefillPath(handle, int(n), hq, hkv, dtype, device, dense_layers) for n in lengths]
+        self.streams = [torch.cuda.Stream(device=device) for _ in lengths]
+
+    def layer(self, qs, ks, vs, first_layer: bool, outs=None, layer=None):
+        """qs[i] [hq, n_i, d], ks[i], vs[i] [hkv, n_i, d]: layer inputs of sequence i.
+        Returns the outputs [hq, n_i, d] (the paths' buffers unless ``outs``)."""
+        cur = torch.cuda.current_stream()
+        ready = torch.cuda.Event()
+        ready.record(cur)
+        res = []
+        for i, (p, st) in enumerate(zip(self.paths, self.streams)):
+            st.wait_event(ready)
+            o = None if outs is None else outs[i]
+            res.append(p.layer(qs[i], ks[i], vs[i], first_layer, out=o, stream=st, layer=layer))
+        for st in self.streams:
+            cur.wait_stream(st)
+        return res
+
+
 class DecodePath:
     """Per-layer decode state and the per-step call order:
     sws_decode_step -> sws_sparse_attn_decode for each layer, then

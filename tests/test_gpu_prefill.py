@@ -245,3 +245,27 @@ def test_group_shared_selection(w):
     swaps = run_case(w, shared=True)
     for s in swaps:
         print("tolerated near-tie swap:", s)
+
+
+def test_prefill_batch_matches_single_sequences():
+    """PrefillBatch: three sequences of different lengths (ragged tails), their
+    layers on concurrent streams, give bit for bit what each sequence gives
+    alone through PrefillPath (which the tests above hold to the oracle)."""
+    base = W.PREFILL_16K.scaled(hq=8, hkv=2, layers=2)
+    ws = [base.scaled(name=f"seq{i}", n=n, seed=base.seed + i) for i, n in enumerate((1000, 2065, 640))]
+    cfg = S.make_config(base.d, base.B, base.k, base.s, 0, base.density, base.seed)
+    h = S.Handle(cfg)
+    batch = S.PrefillBatch(h, [w.n for w in ws], base.hq, base.hkv, torch.bfloat16, "cuda")
+    singles = [S.PrefillPath(h, w.n, base.hq, base.hkv, torch.bfloat16, "cuda") for w in ws]
+    for layer in range(base.layers):
+        ins = [W.prefill_layer_inputs(w, layer, "cuda") for w in ws]
+        outs = batch.layer([x[0] for x in ins], [x[1] for x in ins], [x[2] for x in ins], layer == 0)
+        for p, (Q, K, V) in zip(singles, ins):
+            p.layer(Q, K, V, layer == 0)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        for bp, p, o in zip(batch.paths, singles, outs):
+            assert torch.equal(bp.row_ptr, p.row_ptr) and torch.equal(bp.col_idx, p.col_idx)
+            assert torch.equal(bp.walk_state, p.walk_state)
+            assert torch.equal(o.view(torch.int16), p.o.view(torch.int16))
+    h.close()
