@@ -22,67 +22,11 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // keys[0, m): shared memory, written before the call and visible to the warp.
-// Writes the tau chosen indices, ascending, to out[0, tau). If `mark` is not
-// null, also ORs `bit` into mark[j] for every chosen j (shared memory).
-// 1 <= tau <= m <= 65535 * 2 (counts are held in 16-bit fields).
-__device__ __forceinline__ void warp_top_tau(const uint64_t* keys, int m, int tau, int32_t* out, int32_t* err,
-                                             uint32_t* mark = nullptr, uint32_t bit = 0) {
-  const int lane = threadIdx.x & 31;
-  uint64_t prefix = 0, pmask = 0;
-  int need = tau;
-  bool all_cands = false;
-  for (int shift = 62; shift >= 0; shift -= 2) {
-    uint32_t lo = 0, hi = 0;  // 16-bit counters: digits {0,1} in lo, {2,3} in hi
-    for (int j = lane; j < m; j += 32) {
-      const uint64_t key = keys[j];
-      if ((key & pmask) == prefix) {
-        const uint32_t dg = static_cast<uint32_t>(key >> shift) & 3u;
-        const uint32_t inc = 1u << ((dg & 1u) * 16);
-        if (dg < 2) lo += inc; else hi += inc;
-      }
-    }
-    lo = __reduce_add_sync(0xffffffffu, lo);
-    hi = __reduce_add_sync(0xffffffffu, hi);
-    const int cnt[4] = {static_cast<int>(lo & 0xffffu), static_cast<int>(lo >> 16), static_cast<int>(hi & 0xffffu),
-                        static_cast<int>(hi >> 16)};
-    int dsel = 0;
-    for (int dd = 3; dd >= 0; --dd) {
-      if (need <= cnt[dd]) { dsel = dd; break; }
-      need -= cnt[dd];
-    }
-    prefix |= static_cast<uint64_t>(dsel) << shift;
-    pmask |= 3ull << shift;
-    if (cnt[dsel] == need) { all_cands = true; break; }
-  }
-  const unsigned lt = lanemask_lt();
-  int base = 0, ties = 0;
-  for (int j0 = 0; j0 < m; j0 += 32) {
-    const int j = j0 + lane;
-    const bool valid = j < m;
-    const uint64_t km = valid ? (keys[j] & pmask) : 0;
-    const bool above = valid && km > prefix;
-    const bool cand = valid && km == prefix;
-    const unsigned cb = __ballot_sync(0xffffffffu, cand);
-    bool take = cand;
-    if (!all_cands) {
-      take = cand && (ties + __popc(cb & lt)) < need;
-      ties += __popc(cb);
-    }
-    const bool sel = above || take;
-    const unsigned sb = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
-      const int pos = base + __popc(sb & lt);
-      if (pos < tau) out[pos] = j;
-      if (mark) atomicOr(&mark[j], bit);
-    }
-    base += __popc(sb);
-  }
-  if (lane == 0 && base != tau) record_error(err, GUARD_BAD_SELECT);
-}
-
-// The same selection with 8-bit digits: eight passes, each counting the keys
-// that still match the prefix found so far in a 256-bin histogram hist[]
-// (shared memory owned by this warp), then the ordered compaction above.
+// Writes the tau chosen indices, ascending, to out[0, tau) (1 <= tau <= m).
+// An 8-bit radix select: up to eight passes, each counting the keys that still
+// match the prefix found so far in a 256-bin histogram hist[] (shared memory
+// owned by this warp); then an ordered compaction in index order that takes
+// every key above the threshold and the first `need` keys equal to it.
 __device__ __forceinline__ void warp_top_tau8(const uint64_t* keys, int m, int tau, int32_t* out, int* hist,
                                               int32_t* err) {
   const int lane = threadIdx.x & 31;
