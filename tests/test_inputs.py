@@ -64,3 +64,22 @@ def test_head_inputs_match_layer_inputs():
     for h in range(4):
         q, k, v = W.prefill_head_inputs(w, 1, h)
         assert torch.equal(q, Q[h]) and torch.equal(k, K[h // 2]) and torch.equal(v, V[h // 2])
+
+
+def test_decode_sequence_queries():
+    """The exact decode walk's per-position queries: deterministic, one stream
+    per query head (distinct heads differ), the sink on block 0 and the KV
+    group's hubs on the same blocks as the keys."""
+    w = W.DECODE_128K.scaled(batch=2, layers=1, hq=4, hkv=2, n0=640, steps=3, hubs=2)
+    Q = W.decode_sequence_queries(w, 1, 0, "cpu")
+    assert Q.shape == (4, 643, 128) and Q.dtype == torch.bfloat16
+    assert torch.equal(Q, W.decode_sequence_queries(w, 1, 0, "cpu"))
+    assert not torch.equal(Q[0], Q[1])
+    assert not torch.equal(Q, W.decode_sequence_queries(w, 0, 0, "cpu"))
+    q = Q.double()
+    assert abs(q[:, :w.B].mean().item() - 1.0) < 0.15          # sink shift on block 0
+    assert abs(q[:, 2 * w.B:].mean().item()) < 0.15
+    pos, off = W.hub_layout(-(-w.n0 // w.B), w.hubs, w.d, w.seed, 0, 0, "cpu", 1)
+    for j, p in enumerate(pos.tolist()):                       # group 0's hubs move heads 0 and 1 alike
+        blk = q[:2, p * w.B:(p + 1) * w.B].mean(dim=(0, 1))
+        assert torch.corrcoef(torch.stack([blk, off[j]]))[0, 1] > 0.8
