@@ -110,7 +110,8 @@ sws_status sparse_attn_decode(const sws_handle* h, const void* q_tok, const void
   for (const void* p : ptrs)
     if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
   size_t need = 0;
-  sws_workspace_size(&h->cfg, SWS_OP_DECODE_ATTN, kv.max_len, hq, kv.hkv, batch, &need);
+  if (sws_workspace_size(&h->cfg, SWS_OP_DECODE_ATTN, kv.max_len, hq, kv.hkv, batch, &need) != SWS_OK)
+    return SWS_ERR_INVALID_ARG;
   if (ws_bytes < need) return SWS_ERR_WORKSPACE;
   const int32_t splits = decode_num_splits(h->cfg, kv.max_len, group);
   return cuda_status(launch_decode_attn(h, static_cast<const __nv_bfloat16*>(q_tok),
@@ -328,14 +329,14 @@ sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dty
 sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n, int32_t hq, int first_layer,
                            double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
                            void* stream) {
-  if (!h || n < 1 || hq < 1) return SWS_ERR_INVALID_ARG;
+  if (!h || n < 1 || check_heads(hq, 1) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (h->cfg.select_group > 1 && hq % h->cfg.select_group != 0) return SWS_ERR_INVALID_ARG;
   if (!aligned16(scores) || !aligned16(walk_state) || !aligned16(row_ptr) || !aligned16(col_idx) || !aligned16(ws))
     return SWS_ERR_INVALID_ARG;
   const int64_t b = ceil_div64(n, h->cfg.block_size);
   if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
   size_t need = 0;
-  sws_workspace_size(&h->cfg, SWS_OP_WALK_SELECT, n, hq, 1, 1, &need);
+  if (sws_workspace_size(&h->cfg, SWS_OP_WALK_SELECT, n, hq, 1, 1, &need) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (ws_bytes < need) return SWS_ERR_WORKSPACE;
   auto st = static_cast<cudaStream_t>(stream);
   const size_t mat = static_cast<size_t>(hq) * b * b;

@@ -22,6 +22,10 @@
  * Notation: n tokens, B block size, b = ceil(n/B) blocks, d head dim, k sketch dim,
  * s walk power, hq query heads, hkv KV heads (query head h reads KV head h/(hq/hkv)),
  * density num/den, tau_i = ceil((i+1)*num/den) key blocks for query block i.
+ *
+ * Shape limits checked by every call: hkv >= 1, hkv divides hq, hq <= 4096
+ * (SWS_ERR_INVALID_ARG otherwise); the prefill calls take b <= 8192 blocks
+ * (SWS_ERR_UNSUPPORTED beyond).
  */
 #ifndef SWS_H_
 #define SWS_H_
@@ -120,7 +124,7 @@ sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code);
 
 /* ---------------------------------------------------------------- prefill --- */
 
-/* sw_sketch. §3.1 block means (a partial last block divides by its row count),
+/* sws_sketch. §3.1 block means (a partial last block divides by its row count),
  * §3.2 projection q~_i = q_bar_i H_d, k~_j = k_bar_j H_d and the sketched block scores
  * S[h,i,j] = q~_i(h) . k~_j(h/(hq/hkv)) / sqrt(k) for j <= i (causal block mask).
  *   q      (device) [hq, n, d]   dtype
@@ -135,7 +139,7 @@ sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dty
                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, double* scores, void* ws,
                       size_t ws_bytes, void* stream);
 
-/* sw_walk_select. §4: A = row softmax of scores over j <= i (the sketched block
+/* sws_walk_select. §4: A = row softmax of scores over j <= i (the sketched block
  * attention matrix), M = A^s, R = M on the first layer, else R = R_prev * M; then for
  * each query block i the tau_i largest R[i, j], j <= i (ties to the lower j), listed in
  * ascending order as CSR.
@@ -150,7 +154,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
                            double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
                            void* stream);
 
-/* sw_sparse_attn_prefill. §4/§5: exact softmax attention on the original Q, K, V
+/* sws_sparse_attn_prefill. §4/§5: exact softmax attention on the original Q, K, V
  * restricted to the selected key blocks; query token t attends to the tokens u of the
  * blocks listed for its block with u <= t. Online softmax, fp32 accumulation.
  *   q (device) [hq, n, d], k, v (device) [hkv, n, d], o (device) [hq, n, d]: all dtype
@@ -193,7 +197,9 @@ sws_status sws_decode_advance(const sws_handle* h, int32_t* seq_lens, int32_t ba
  *   sel        [batch, hkv, max_blocks] int32: union over the GQA group, ascending
  *   sel_mask   [batch, hkv, max_blocks] uint8: bit r set = query head hkv_index*group + r chose it
  *   sel_cnt    [batch, hkv] int32
- * group = hq/hkv must be <= 8. */
+ * group = hq/hkv must be <= 8, and the selection's shared memory (about
+ * max_blocks * (8 * group + 4) bytes: 5.6K blocks, 364K tokens at B = 64, for a group
+ * of 4) must stay within 200 KB; SWS_ERR_UNSUPPORTED otherwise. */
 sws_status sws_decode_step(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
                            int32_t batch, int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens,
                            void* k_cache, void* v_cache, double* k_psum, double* k_sketch, int first_layer,
@@ -225,11 +231,12 @@ sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const v
                                  double* q_sketch, int first_layer, double* walk_state, int32_t* head_sel,
                                  int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
 
-/* sw_sparse_attn_decode: one query token per (sequence, head) over the tokens
+/* sws_sparse_attn_decode: one query token per (sequence, head) over the tokens
  * (< seq_lens[i]) of the blocks its head selected. Each KV block of the group's union is
  * read once for all the group's heads (split over the union, then combined).
  *   q_tok [batch, hq, d] bf16; o [batch, hq, d] bf16 (device)
- *   ws    sws_workspace_size(SWS_OP_DECODE_ATTN) bytes */
+ *   ws    sws_workspace_size(SWS_OP_DECODE_ATTN) bytes
+ * group = hq/hkv must be 1, 2, 4 or 8 (SWS_ERR_UNSUPPORTED otherwise). */
 sws_status sws_sparse_attn_decode(const sws_handle* h, const void* q_tok, const void* k_cache,
                                   const void* v_cache, int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
                                   const int32_t* seq_lens, const int32_t* sel, const uint8_t* sel_mask,
