@@ -142,6 +142,19 @@ def test_decode_first_token_of_block():
     run_decode(w, [1024, 64], steps=2)
 
 
+@pytest.mark.parametrize("d,B,k", [(64, 64, 16), (128, 128, 32), (64, 128, 16)])
+@pytest.mark.parametrize("paged", [False, True])
+def test_decode_head_dim_and_block_size(d, B, k, paged):
+    """The other instantiations of the decode kernels: head dim 64 and block
+    size 128, contiguous and paged. The first sequence's steps cross a block
+    boundary of either size (766 + 3 > 768); the last holds one full block of
+    64 and a partial one, or a partial second block of 128."""
+    w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=3, d=d, B=B, k=k)
+    swaps = run_decode(w, [766, 1200, 130], steps=3, paged=paged)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
 def test_decode_full_size_sampled():
     """The full decode workload (16 sequences, 131072 cached tokens, 8 layers)
     for a few steps; the oracle recomputes two sampled sequences."""

@@ -133,6 +133,16 @@ def test_decode_exact_group_shared():
         print("tolerated near-tie swap:", s)
 
 
+@pytest.mark.parametrize("d,B,k", [(64, 64, 16), (64, 128, 16), (128, 128, 32)])
+def test_decode_exact_head_dim_and_block_size(d, B, k):
+    """The exact walk's other instantiation (head dim 64) and block size 128,
+    with steps crossing a block boundary of either size."""
+    w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=3, d=d, B=B, k=k)
+    swaps = run_exact(w, [766, 1200, 130], steps=3)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
 def test_decode_exact_16k_sampled():
     """The exact walk at a 16K context (257 blocks, the size its shared-memory
     triangle is built for), batch 4, two layers; one sequence checked."""
