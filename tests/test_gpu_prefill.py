@@ -99,6 +99,10 @@ def test_scaled_workloads_in_full(w):
     (W.PREFILL_16K.scaled(name="odd_blocks_B64", n=1050, hq=2, hkv=1, layers=2), 0),
     (W.PREFILL_16K.scaled(name="bf16_one_block", n=100, hq=2, hkv=1, layers=1, hubs=0), 0),
     (W.PREFILL_64K.scaled(name="bf16_B128_dense", n=700, hq=2, hkv=1, layers=1, density=(1, 1)), 0),
+    (W.PREFILL_16K.scaled(name="bf16_d64_B64", d=64, k=16, n=2500, hq=4, hkv=2, layers=2), 0),
+    (W.PREFILL_16K.scaled(name="fp32_d128_B64", dtype="fp32", n=1100, hq=2, hkv=1, layers=2), 0),
+    (W.PREFILL_64K.scaled(name="fp32_d128_B128", dtype="fp32", n=1500, hq=2, hkv=1, layers=2), 0),
+    (W.TINY.scaled(name="fp32_d64_B128", B=128, n=1000, layers=2), 0),
 ], ids=lambda x: x.name if hasattr(x, "name") else str(x))
 def test_edge_cases(w, mode):
     run_case(w, mode=mode)
@@ -243,6 +247,20 @@ def test_group_shared_selection(w):
     """Group-shared selection: every head of a GQA group gets the top-tau of
     the sum of the group's walk rows; the walk state stays per head."""
     swaps = run_case(w, shared=True)
+    for s in swaps:
+        print("tolerated near-tie swap:", s)
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_beyond_1024_blocks(shared):
+    """b = 1094 key blocks: past the register-resident row kernels, the walk's
+    softmax and the top-tau selection take their general forms (rows staged
+    through global and shared memory). Two heads of one KV head, whole walk
+    chain over two layers, attention on sampled query blocks."""
+    w = W.PREFILL_16K.scaled(name="b1094_B64", n=70000, hq=2, hkv=1, layers=2)
+    b = w.b
+    assert b > 1024
+    swaps = run_case(w, blocks=sorted({0, 1, 511, 1023, 1024, b - 2, b - 1}), shared=shared)
     for s in swaps:
         print("tolerated near-tie swap:", s)
 
