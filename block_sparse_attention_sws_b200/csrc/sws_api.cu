@@ -343,6 +343,9 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
   double* buf[4] = {static_cast<double*>(ws), static_cast<double*>(ws) + mat, static_cast<double*>(ws) + 2 * mat,
                     static_cast<double*>(ws) + 3 * mat};
   bool busy[4] = {false, false, false, false};
+  // At most four products are live at once (base, result, the new product,
+  // and R_prev * M after the loop), so take() always finds a free buffer; a
+  // failure would be a bug in the schedule below and is reported, not used.
   auto take = [&]() -> int {
     for (int q = 0; q < 4; ++q)
       if (!busy[q]) {
@@ -365,6 +368,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
           result = base;
         } else {
           const int dst = take();
+          if (dst < 0) return SWS_ERR_UNSUPPORTED;
           s = cuda_status(launch_tri_gemm(buf[result], buf[base], buf[dst], b, hq, st), "walk power");
           if (s != SWS_OK) return s;
           if (result != base) busy[result] = false;
@@ -374,6 +378,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
       e >>= 1;
       if (!e) break;
       const int dst = take();
+      if (dst < 0) return SWS_ERR_UNSUPPORTED;
       s = cuda_status(launch_tri_gemm(buf[base], buf[base], buf[dst], b, hq, st), "walk square");
       if (s != SWS_OK) return s;
       if (base != result) busy[base] = false;
@@ -385,6 +390,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
   const double* Rnew = buf[m_idx];
   if (!first_layer) {
     const int dst = take();
+    if (dst < 0) return SWS_ERR_UNSUPPORTED;
     s = cuda_status(launch_tri_gemm(walk_state, buf[m_idx], buf[dst], b, hq, st), "walk update");
     if (s != SWS_OK) return s;
     Rnew = buf[dst];
