@@ -51,6 +51,43 @@ def pin_srht_draws():
     assert sorted(perm) == list(range(32))
 
 
+def pin_srht_draws_published_stream():
+    """The draws follow the published splitmix64 stream: a seed equal to the
+    stream tag starts the generator at state 0, whose first three outputs are
+    the golden test vector. d = 2 takes exactly those three: the signs come
+    from the top bits of outputs 0 and 1, the one shuffle step swaps position
+    1 with (output 2 mod 2). H_d is then D H / sqrt(2) in closed form."""
+    with open(os.path.join(GOLDEN, "splitmix64_seed0.txt")) as f:
+        g = [int(x, 16) for x in f.read().split() if x.startswith("0x")]
+    tag = so.SRHT_STREAM_TAG
+    signs = [1 if (x >> 63) == 0 else -1 for x in g[:2]]
+    perm = [0, 1]
+    j = g[2] % 2
+    perm[1], perm[j] = perm[j], perm[1]
+    assert so.srht_draws(2, 2, tag) == (signs, perm)
+    assert so.srht_draws(2, 1, tag) == (signs, perm[:1])
+    H = np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2.0)
+    want = (np.diag(signs) @ H)[:, perm]
+    assert np.allclose(so.srht_matrix(2, 2, tag), want, rtol=0, atol=1e-15)
+
+
+def pin_srht_shuffle_uniform():
+    """Fisher-Yates draws every permutation equally often: over 4800 seeds
+    all 24 orders of d = 4 appear with chi-square well inside its range. A
+    shuffle that swaps with (draw mod r) instead (Sattolo's cyclic variant)
+    never yields the identity and fails."""
+    counts = {}
+    for seed in range(4800):
+        _, perm = so.srht_draws(4, 4, seed)
+        counts[tuple(perm)] = counts.get(tuple(perm), 0) + 1
+    assert len(counts) == 24 and (0, 1, 2, 3) in counts
+    expected = 4800 / 24
+    chi2 = sum((c - expected) ** 2 / expected for c in counts.values())
+    assert chi2 < 60.0  # 23 degrees of freedom: p(chi2 > 60) < 1e-4
+    signs = np.array([so.srht_draws(8, 1, seed)[0] for seed in range(2000)])
+    assert np.all(np.abs(signs.mean(axis=0)) < 0.1)
+
+
 def pin_srht_orthogonal_when_k_equals_d():
     """k = d: H_d is orthogonal, so the sketch keeps every inner product (Parseval)."""
     for d, seed in ((64, 3), (128, 11)):
@@ -170,6 +207,21 @@ def pin_walk_invariants():
         assert np.allclose(R.sum(axis=1), 1.0, atol=1e-12)
         assert np.all(R[np.triu_indices(w.b, 1)] == 0.0)
         assert np.all(R[np.tril_indices(w.b)] > 0.0)
+
+
+def pin_walk_elementwise():
+    """Reading R5's alternative: the entrywise power with rows renormalised is
+    row-stochastic and lower-triangular, keeps each row's order, and raises
+    every ratio of two entries of a row to the power s."""
+    A = so.block_attention(so.sketch_scores(rng.standard_normal((12, 4)), rng.standard_normal((12, 4))))
+    for s in (1, 2, 8):
+        M = so.walk_matrix(A, s, "elementwise")
+        assert np.allclose(M.sum(axis=1), 1.0, atol=1e-14)
+        assert np.all(M[np.triu_indices(12, 1)] == 0.0)
+        for i in range(1, 12):
+            r, a = M[i, :i + 1], A[i, :i + 1]
+            assert np.array_equal(np.argsort(-r, kind="stable"), np.argsort(-a, kind="stable"))
+            assert np.allclose(r[1:] / r[0], (a[1:] / a[0]) ** s, rtol=1e-11)
 
 
 def pin_top_tau_bruteforce():
@@ -437,6 +489,32 @@ PLANTED = {
         pin_attention_dense_limit),
 }
 
+
+PLANTED["signs_from_set_top_bit"] = (
+    "srht_draws", lambda orig: (lambda d, k, seed: ([-x for x in orig(d, k, seed)[0]], orig(d, k, seed)[1])),
+    pin_srht_draws_published_stream)
+
+
+def _sattolo_draws(d, k, seed):
+    signs, _ = _ORIG_DRAWS(d, k, seed)
+    state = (seed ^ so.SRHT_STREAM_TAG) & ((1 << 64) - 1)
+    draws = []
+    for _ in range(2 * d - 1):
+        state, z = so.splitmix64(state)
+        draws.append(z)
+    perm, nxt = list(range(d)), d
+    for r in range(d - 1, 0, -1):
+        j = draws[nxt] % r
+        nxt += 1
+        perm[r], perm[j] = perm[j], perm[r]
+    return signs, perm[:k]
+
+
+_ORIG_DRAWS = so.srht_draws
+PLANTED["shuffle_mod_r"] = ("srht_draws", lambda orig: _sattolo_draws, pin_srht_shuffle_uniform)
+PLANTED["elementwise_not_renormalised"] = (
+    "walk_matrix", lambda orig: (lambda A, s, mode="matrix_power": A ** s if mode == "elementwise" else orig(A, s, mode)),
+    pin_walk_elementwise)
 
 PLANTED["exact_decode_previous_block_row"] = (
     "decode_exact_layer", lambda orig: (lambda Q, K, Hd, B, s, density, state, heads=None, select="per_head": {
