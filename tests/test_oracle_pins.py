@@ -339,6 +339,84 @@ def pin_decode():
     assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
 
 
+def _softmax_plain(z):
+    """exp(z - max) / sum: a probability row, without any logarithm."""
+    e = np.exp(z - z.max())
+    return e / e.sum()
+
+
+def pin_decode_walk_carry():
+    """Decode walk over layers (reading R7): the carried log-domain row, taken
+    back out of the logs, is the entrywise product over the layers of each
+    layer's softmax row raised to s, multiplied out directly (no logarithms):
+    exp(rho^L) = prod_l softmax(z^l)^s. A carry that is dropped, or that adds
+    s * z instead of s * (z - logsumexp z), changes these values. The
+    selection after the last layer is the top-tau of that product."""
+    hq, hkv, d, B, k, s, L = 3, 1, 8, 4, 8, 2, 21
+    Hd = so.srht_matrix(d, k, 11)
+    r = np.random.default_rng(2024)
+    rho, prod, zs = None, None, []
+    for layer in range(3):
+        Kc = r.standard_normal((hkv, 24, d))
+        q = r.standard_normal((hq, d))
+        rho, z, sel = so.decode_layer_select(q, Kc, L, Hd, B, s, (2, 5), rho)
+        zs.append(z)
+        f = np.stack([_softmax_plain(z[h]) ** s for h in range(hq)])
+        prod = f if prod is None else prod * f
+        assert np.allclose(np.exp(rho), prod, rtol=1e-12, atol=0.0)
+        tau = so.tau_of_row(-(-L // B) - 1, 2, 5)
+        for h in range(hq):
+            want = np.sort(np.lexsort((np.arange(prod.shape[1]), -prod[h]))[:tau])
+            assert np.array_equal(sel[h], want)
+    # the three layers' rows differ, so the carry matters for the values
+    assert not np.allclose(zs[0], zs[2])
+
+
+def pin_decode_logits_literal():
+    """With k = d the projection is orthogonal, so the decode row logit of
+    block j is the plain mean over the block's cached tokens of q . K[t] /
+    sqrt(d) (the partial last block by its count), summed here token by token."""
+    d, B, L = 8, 4, 18
+    Kc = rng.standard_normal((1, 20, d))
+    q = rng.standard_normal((1, d))
+    Hd = so.srht_matrix(d, d, 9)
+    _, z, _ = so.decode_layer_select(q, Kc, L, Hd, B, 1, (1, 2), None)
+    nb = -(-L // B)
+    for j in range(nb):
+        toks = range(j * B, min(L, (j + 1) * B))
+        acc = 0.0
+        for t in toks:
+            acc += sum(float(q[0, c]) * float(Kc[0, t, c]) for c in range(d))
+        assert abs(z[0, j] - acc / (len(toks) * math.sqrt(d))) < 1e-12
+
+
+def pin_attention_triple_loop():
+    """Sparse attention against a naive loop: for every query token, every
+    allowed key token (in a selected block, at or before the query), the
+    score, the softmax and the weighted sum of V, one scalar at a time.
+    A random selection (every row holds tau_i blocks) with a ragged tail."""
+    n, d, B = 22, 4, 4
+    Q, K, V = (rng.standard_normal((n, d)) for _ in range(3))
+    b = -(-n // B)
+    rp, ci = so.select_top_tau(rng.random((b, b)), 1, 2)
+    O = so.sparse_attention(Q, K, V, rp, ci, B)
+    for t in range(n):
+        i = t // B
+        allowed = [u for j in ci[rp[i]:rp[i + 1]] for u in range(j * B, min(n, (j + 1) * B)) if u <= t]
+        sc = []
+        for u in allowed:
+            acc = 0.0
+            for c in range(d):
+                acc += Q[t, c] * K[u, c]
+            sc.append(acc / math.sqrt(d))
+        mx = max(sc)
+        w = [math.exp(x - mx) for x in sc]
+        tot = sum(w)
+        for c in range(d):
+            want = sum(w[a] * V[u, c] for a, u in enumerate(allowed)) / tot
+            assert abs(O[t, c] - want) < 1e-12
+
+
 def pin_group_shared_log_rows():
     """The decode group score is log(sum_h exp(rho_h)): scipy's logsumexp on
     rows far below exp's range, and shift invariance."""
@@ -521,6 +599,61 @@ PLANTED["exact_decode_previous_block_row"] = (
         h: dict(r, row=np.append(state.R[h][-2, :-1], 0.0)) for h, r in orig(Q, K, Hd, B, s, density, state, heads,
                                                                              select).items()}),
     pin_exact_decode)
+
+
+
+def _decode_carry_wrapped(wrong_rho):
+    """A decode_layer_select whose returned rho is replaced by wrong_rho(s, z, rho_prev),
+    the selection taken again on it (as the oracle would after that mistake)."""
+    orig = _ORIG_DECODE
+
+    def f(q_tok, Kc, length, Hd, B, s, density, rho_prev, select="per_head"):
+        _, z, _ = orig(q_tok, Kc, length, Hd, B, s, density, rho_prev, select)
+        rho = wrong_rho(s, z, rho_prev)
+        tau = so.tau_of_row(-(-length // B) - 1, *density)
+        return rho, z, [so.top_tau_row(rho[h], tau) for h in range(rho.shape[0])]
+    return f
+
+
+def _lse(z):
+    m = z.max(axis=1, keepdims=True)
+    return m + np.log(np.exp(z - m).sum(axis=1, keepdims=True))
+
+
+_ORIG_DECODE = so.decode_layer_select
+PLANTED["decode_carry_dropped"] = (
+    "decode_layer_select", lambda orig: _decode_carry_wrapped(lambda s, z, rp: s * (z - _lse(z))),
+    pin_decode_walk_carry)
+PLANTED["decode_carry_of_raw_logits"] = (
+    "decode_layer_select", lambda orig: _decode_carry_wrapped(
+        lambda s, z, rp: s * (z - _lse(z)) if rp is None else s * z + rp),
+    pin_decode_walk_carry)
+PLANTED["decode_carry_scaled_twice"] = (
+    "decode_layer_select", lambda orig: _decode_carry_wrapped(
+        lambda s, z, rp: s * (z - _lse(z) + (0.0 if rp is None else rp))),
+    pin_decode_walk_carry)
+PLANTED["decode_logits_scale_sqrt_d"] = (
+    "decode_layer_select", lambda orig: (
+        lambda q_tok, Kc, length, Hd, B, s, density, rho_prev, select="per_head":
+        (lambda r: (r[0], r[1] * 2.0, r[2]))(orig(q_tok, Kc, length, Hd, B, s, density, rho_prev, select))),
+    pin_decode_logits_literal)
+PLANTED["attention_causal_mask_off_by_one"] = (
+    "sparse_attention_block", lambda orig: _attn_mask_lt, pin_attention_triple_loop)
+
+
+def _attn_mask_lt(Q, K, V, i, blocks, B):
+    """sparse_attention_block with the diagonal excluded (u < t instead of u <= t)
+    wherever a token has an earlier allowed key."""
+    n, d = Q.shape
+    t0, t1 = i * B, min(n, (i + 1) * B)
+    u = np.concatenate([np.arange(j * B, min(n, (j + 1) * B)) for j in blocks])
+    s = Q[t0:t1] @ K[u].T / math.sqrt(d)
+    t = np.arange(t0, t1)
+    allow = u[None, :] < t[:, None]
+    allow[~allow.any(axis=1)] = u[None, :] <= t[~allow.any(axis=1), None]
+    s = np.where(allow, s, -np.inf)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    return (p @ V[u]) / p.sum(axis=1, keepdims=True)
 
 
 @pytest.mark.parametrize("name", sorted(PLANTED))
