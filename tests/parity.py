@@ -22,6 +22,27 @@ ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 5e-3
 
 
+# Tolerated near-tie swaps per test, filled by record_ties and summarised at the
+# end of the session (conftest.py prints the counts and writes them as JSON).
+TIE_REPORT: dict = {}
+
+
+def record_ties(swaps, compared: int = 0, name: str = None):
+    """Adds a test's tolerated swaps (each a tuple ending in the oracle's relative
+    gap) and the number of selections it compared to the session's tie report,
+    under the running test's id unless a name is given."""
+    if name is None:
+        import os
+        name = os.environ.get("PYTEST_CURRENT_TEST", "unnamed").rsplit(" (", 1)[0].split("::", 1)[-1]
+    e = TIE_REPORT.setdefault(name, {"swaps": 0, "selections_compared": 0, "largest_gap": 0.0, "examples": []})
+    e["swaps"] += len(swaps)
+    e["selections_compared"] += int(compared)
+    for s in swaps:
+        e["largest_gap"] = max(e["largest_gap"], float(s[-1]))
+        if len(e["examples"]) < 5:
+            e["examples"].append([float(x) if isinstance(x, float) else int(x) for x in s])
+
+
 class LazyHeads:
     """Indexable view of a [H, n, d] tensor that widens one head at a time to fp64 numpy."""
 

@@ -23,7 +23,7 @@ import block_sparse_attention_sws_b200 as S
 import oracle
 import sws_inputs as W
 from oracle import sws_oracle as so
-from parity import compare_attention, compare_selection
+from parity import compare_attention, compare_selection, record_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +105,7 @@ def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None):
                     assert n == len(blocks)
                     assert list(sel[s_, g, :n]) == blocks
                     assert [int(m) for m in msk[s_, g, :n]] == [ug[(g, j)] for j in blocks]
+    record_ties(swaps, compared=steps * w.layers * len(check_seqs) * w.hq)
     h.close()
     return swaps
 
@@ -114,8 +115,6 @@ def test_decode_exact_small_ragged():
     three layers: the walk row, the selection, the union and attention."""
     w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
     swaps = run_exact(w, [1000, 1500, 638], steps=5)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 def test_decode_exact_first_token_of_block():
@@ -129,8 +128,6 @@ def test_decode_exact_group_shared():
     """Exact walk with group-shared selection: the top-tau of the group's summed rows."""
     w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=3)
     swaps = run_exact(w, [900, 1300], steps=3, shared=True)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 @pytest.mark.parametrize("d,B,k", [(64, 64, 16), (64, 128, 16), (128, 128, 32)])
@@ -139,8 +136,6 @@ def test_decode_exact_head_dim_and_block_size(d, B, k):
     with steps crossing a block boundary of either size."""
     w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=3, d=d, B=B, k=k)
     swaps = run_exact(w, [766, 1200, 130], steps=3)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 def test_decode_exact_16k_sampled():

@@ -13,7 +13,8 @@ import block_sparse_attention_sws_b200 as S
 import oracle
 import sws_inputs as W
 from oracle import sws_oracle as so
-from parity import (LazyHeads, check_csr_valid, compare_attention, compare_csr, compare_scores, compare_walk)
+from parity import (LazyHeads, check_csr_valid, compare_attention, compare_csr, compare_scores, compare_walk,
+                    record_ties)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,6 +66,7 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
                 compare_attention(o_gpu[i * w.B:min(w.n, (i + 1) * w.B)], want)
     if report is not None:
         report.extend(swaps)
+    record_ties(swaps, compared=w.layers * len(heads) * w.b)
     h.close()
     return swaps
 
@@ -82,8 +84,6 @@ def test_tiny_workload_in_full():
 ], ids=lambda w: w.name)
 def test_scaled_workloads_in_full(w):
     swaps = run_case(w)
-    for s in swaps:
-        print("tolerated near-tie swap (layer, head, row, gpu-only, oracle-only, gap):", s)
 
 
 @pytest.mark.parametrize("w,mode", [
@@ -148,8 +148,6 @@ def test_full_size_sampled(w):
     b = w.b
     blocks = sorted({0, 1, b // 3, b // 2, b - 2, b - 1})
     swaps = run_case(w, heads=[0, w.hq - 1], blocks=blocks)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 def test_device_guard_reports_bad_csr():
@@ -247,8 +245,6 @@ def test_group_shared_selection(w):
     """Group-shared selection: every head of a GQA group gets the top-tau of
     the sum of the group's walk rows; the walk state stays per head."""
     swaps = run_case(w, shared=True)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 @pytest.mark.parametrize("shared", [False, True])
@@ -261,8 +257,6 @@ def test_beyond_1024_blocks(shared):
     b = w.b
     assert b > 1024
     swaps = run_case(w, blocks=sorted({0, 1, 511, 1023, 1024, b - 2, b - 1}), shared=shared)
-    for s in swaps:
-        print("tolerated near-tie swap:", s)
 
 
 def test_prefill_batch_matches_single_sequences():
