@@ -19,7 +19,6 @@
 //     head, and writes a partial (o, max, sum) per head.
 //   decode_combine_kernel: merges the partials of each (sequence, head).
 #include <algorithm>
-#include <mutex>
 
 #include "select.cuh"
 #include "sws_common.cuh"
@@ -716,30 +715,25 @@ cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, 
 // by the CUDA runtime when the library is loaded on a device and held until
 // the process exits.
 
-namespace {
-
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SWS_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch, looked up once per device. On the host
-// the array's name is only a stand-in for the device symbol; the kernel must
-// receive the address that cudaGetSymbolAddress returns for the current device.
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[256] = {};
+namespace sws {
 
-cudaError_t noalloc_scratch(int device, void** out) {
-  if (device < 0 || device >= 256) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[device]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[device] = p;
-  }
-  *out = g_noalloc_ptr[device];
+// Device address of g_noalloc_scratch on the current device. On the host the
+// array's name is only a stand-in for the device symbol: a kernel must receive
+// the address that cudaGetSymbolAddress returns in the context it runs in.
+// sws_create calls this once per handle, with the handle's device current, and
+// keeps the result in the handle, so a context that is torn down and created
+// again (cudaDeviceReset) gives new handles the new address.
+cudaError_t noalloc_scratch_address(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  *out = p;
   return cudaSuccess;
 }
 
-}  // namespace
+}  // namespace sws
 
 extern "C" sws_status sws_sparse_attn_decode_noalloc(const sws_handle* h, const void* q_tok, const void* k_cache,
                                                      const void* v_cache, int32_t batch, int32_t hq, int32_t hkv,
@@ -757,8 +751,8 @@ extern "C" sws_status sws_sparse_attn_decode_noalloc(const sws_handle* h, const 
   if (need > SWS_NOALLOC_SCRATCH_BYTES) return SWS_ERR_WORKSPACE;  // beyond the built-in scratch
   int device = -1;
   if (cudaGetDevice(&device) != cudaSuccess || device != h->device) return SWS_ERR_INVALID_ARG;
-  void* scratch = nullptr;
-  if (noalloc_scratch(device, &scratch) != cudaSuccess) return SWS_ERR_CUDA;
+  void* scratch = h->noalloc_scratch;
+  if (!scratch) return SWS_ERR_CUDA;
   const cudaError_t e = sws::launch_decode_attn(
       h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_cache),
       static_cast<const __nv_bfloat16*>(v_cache), batch, hq, sws::contiguous_kv(h->cfg, hkv, max_len), seq_lens, sel,

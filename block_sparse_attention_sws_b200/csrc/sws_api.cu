@@ -276,6 +276,7 @@ sws_status sws_create(const sws_config* c, sws_handle** out) {
   if (e == cudaSuccess) e = cudaMemcpy(h->sign, sign.data(), sign_bytes, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(h->col, col.data(), k * sizeof(int32_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int32_t));
+  if (e == cudaSuccess) e = noalloc_scratch_address(&h->noalloc_scratch);
   if (e != cudaSuccess) {
     cudaFree(mem);
     delete h;

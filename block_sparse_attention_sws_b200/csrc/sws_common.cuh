@@ -19,6 +19,7 @@ struct sws_handle {
   int32_t* col;  // [k] the sampled Hadamard columns P of H_d
   double scale;  // 1/sqrt(k): H_d[r][c] = scale * sign[r] * (-1)^popcount(r & col[c])
   int32_t* err;  // device error word (guard code of the first failure, 0 = none)
+  void* noalloc_scratch;  // device address of the built-in decode scratch in this handle's context
 };
 
 namespace sws {
@@ -245,6 +246,7 @@ cudaError_t launch_decode_exact(const sws_handle* h, const __nv_bfloat16* q_tok,
 size_t decode_exact_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
 bool decode_exact_supported(const sws_config& cfg, int64_t max_blocks, int32_t group);
 int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group);
+cudaError_t noalloc_scratch_address(void** out);
 size_t decode_select_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
 cudaError_t launch_decode_attn(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_cache,
                                const __nv_bfloat16* v_cache, int32_t batch, int32_t hq, const KvLayout& kv,

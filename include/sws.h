@@ -285,8 +285,10 @@ sws_status sws_sparse_attn_decode_paged(const sws_handle* h, const void* q_tok, 
  * SWS_NOALLOC_SCRATCH_BYTES built into the library. The CUDA runtime places that array
  * on every device the library is loaded on, and it stays there until the process exits.
  *  - The call allocates nothing (no cudaMalloc, no cudaFree, nothing through a framework).
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *    and keeps it; make that first call on each device before any stream capture.
+ *  - sws_create looks up the array's device address (cudaGetSymbolAddress) with the
+ *    handle's device current and keeps it in the handle, so this call does no set-up of
+ *    its own. The address belongs to the CUDA context the handle was created in: after
+ *    that context is torn down (cudaDeviceReset), create a new handle.
  *  - The handle's device must be the current device.
  *  - Every call shares the one array and finds the previous call's contents in it (each
  *    call overwrites all it reads). Calls whose kernels overlap on the GPU race on it:
