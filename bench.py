@@ -1,14 +1,16 @@
 #!/usr/bin/env python
 """Benchmark of the Sketch&Walk hot path on B200 (one process per GPU).
 
-Default run (N=1): the prefill workload of 4 layers, 32 query / 8 KV heads,
-d=128, n=16384, B=64, k=32, s=8, 20% density (bf16), one step = one pass of
-sws_sketch -> sws_walk_select -> sws_sparse_attn_prefill over all 4 layers.
-The decode workload (16 sequences x 131072 cached tokens, 8 layers, 64 steps)
-is timed in the same run and reported under "decode". Every input is seeded
-synthetic data resident in HBM before the timed region; "e2e" repeats the
-prefill step with the inputs copied from pinned host memory and the outputs
-copied back inside the timed region.
+Default run (N=1): the long-context prefill workload of 4 layers, 32 query /
+8 KV heads, d=128, n=131072, B=128, k=32, s=8, 20% density (bf16); one step =
+one pass of sws_sketch -> sws_walk_select -> sws_sparse_attn_prefill over all
+4 layers. The same workload at 10% density, the 8-layer 65536-token workload
+and the 4-layer 16384-token workload are timed in the same run and reported
+under "prefill_workloads"; the decode workload (16 sequences x 131072 cached
+tokens, 8 layers, 64 steps) under "decode". Every input is seeded synthetic
+data resident in HBM before the timed region; "e2e" repeats the headline step
+with the inputs copied from pinned host memory and the outputs copied back
+inside the timed region.
 
 With --gpus N under torchrun each rank runs an independent replica (the path
 has no data exchange); times are the max over ranks.
@@ -26,7 +28,6 @@ import subprocess
 import sys
 import threading
 import time
-import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -37,7 +38,7 @@ METRIC = "prefill tokens/s + % tensor peak at 20% density; decode step µs + HBM
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
@@ -189,36 +190,41 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------ cpu baseline --
 
-def oracle_head_layers(w):
+ORACLE_SAMPLE_BLOCKS = 64  # query blocks per head-layer whose attention the oracle computes
+
+
+def oracle_head_layers(w, sample_blocks=ORACLE_SAMPLE_BLOCKS):
     """The oracle over the workload one (head, layer) at a time, head by head,
-    each head's walk state carried through its layers; yields the seconds each
-    head-layer took (input generation excluded)."""
+    each head's walk state carried through its layers. Per head-layer it runs
+    the sketch, walk and selection in full and the attention of a seeded
+    sample of query blocks (every block when the workload has no more than
+    sample_blocks), and yields (seconds of the sketch-walk-select part, seconds
+    of the sampled attention, key-block pairs of all query blocks / pairs of
+    the sampled ones). Input generation is not timed."""
+    import numpy as np
     import oracle
     import sws_inputs as W
     from oracle import sws_oracle as so
     Hd = oracle.srht_matrix(w.d, w.k, w.seed)
+    rng = np.random.default_rng(w.seed)
     h = 0
     while True:
         st = so.PrefillState()
         for layer in range(w.layers):
             q, k, v = W.prefill_head_inputs(w, layer, h % w.hq)
-            q64, k64, v64 = (x.double().numpy()[None] for x in (q, k, v))
+            q64, k64, v64 = (x.double().numpy() for x in (q, k, v))
             t0 = time.perf_counter()
-            so.prefill_layer(q64, k64, v64, Hd, w.B, w.s, w.density, st, heads=[0], attention_blocks="all")
-            yield time.perf_counter() - t0
+            out = so.prefill_layer(q64[None], k64[None], v64[None], Hd, w.B, w.s, w.density, st, heads=[0],
+                                   attention_blocks=None)[0]
+            t1 = time.perf_counter()
+            rp, ci = out["row_ptr"], out["col_idx"]
+            blocks = (list(range(w.b)) if w.b <= sample_blocks
+                      else sorted(int(x) for x in rng.choice(w.b, sample_blocks, replace=False)))
+            so.sparse_attention(q64, k64, v64, rp, ci, w.B, blocks)
+            t2 = time.perf_counter()
+            sampled = sum(int(rp[i + 1] - rp[i]) for i in blocks)
+            yield t1 - t0, t2 - t1, int(rp[-1]) / sampled
         h += 1
-
-
-def oracle_prefill_sample(w, budget_s: float):
-    """Times the oracle on whole heads (all layers, every query block) until the
-    budget is spent; returns (seconds, heads done)."""
-    secs, done = 0.0, 0
-    for t in oracle_head_layers(w):
-        secs += t
-        done += 1
-        if done % w.layers == 0 and (secs >= budget_s or done // w.layers >= w.hq):
-            break
-    return secs, done // w.layers
 
 
 def blas_threads() -> int:
@@ -230,40 +236,74 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, budget_s=12.0):
-    secs, heads = oracle_prefill_sample(w, budget_s)
-    full = secs * w.hq / heads
+def head_layer_estimate(t_sws, t_attn, scale) -> float:
+    """Oracle seconds of one whole head-layer: the sketch, walk and selection as
+    run, plus the sampled attention scaled linearly by key-block pairs."""
+    return t_sws + t_attn * scale
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """The oracle on whole heads (every layer of a head, its walk carried) until
+    the budget is spent; one pass = hq x layers head-layers."""
+    measured, est, done = 0.0, 0.0, 0
+    for t_sws, t_attn, scale in oracle_head_layers(w):
+        measured += t_sws + t_attn
+        est += head_layer_estimate(t_sws, t_attn, scale)
+        done += 1
+        if done % w.layers == 0 and (measured >= budget_s or done >= w.hq * w.layers):
+            break
+    full = est / done * w.hq * w.layers
+    sampled = "every query block" if w.b <= ORACLE_SAMPLE_BLOCKS else \
+        f"attention of {ORACLE_SAMPLE_BLOCKS} seeded query blocks of {w.b} per head-layer"
     return {"value": w.n / full, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"oracle (fp64 numpy) on {heads} of {w.hq} query heads x {w.layers} layers, every query block; "
-                      f"{secs:.1f} s measured, scaled by heads to the whole {w.hq}-head pass",
+            "sample": f"oracle (fp64 numpy) on {done // w.layers} of {w.hq} query heads x {w.layers} layers: "
+                      f"sketch, walk and selection in full, {sampled}; {measured:.1f} s measured, extrapolated "
+                      f"linearly (attention by key-block pairs, then by heads) to the whole pass",
+            "extrapolated": w.b > ORACLE_SAMPLE_BLOCKS or done < w.hq * w.layers,
             "host_cpus": os.cpu_count()}
 
 
 # --------------------------------------------------------------- reference --
 
+def workload_config(w, world) -> dict:
+    """The config dict of a prefill workload, the same in both arms."""
+    return {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
+            "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2 ({prefill_input_bytes(w) / 1e6:.0f} MB per step)"}
+
+
+def prefill_input_bytes(w) -> int:
+    elem = 4 if w.dtype == "fp32" else 2
+    return w.layers * (w.hq + 2 * w.hkv) * w.n * w.d * elem
+
+
 def run_reference(args, world, rank):
     import sws_inputs as W
     if rank != 0:
         return 0
-    w = W.PREFILL_16K
+    w = headline_workload(W)
     # one step = one (head, layer) of the pass, heads in turn with their walk
-    # state carried across steps; scaled by the hq x layers head-layers of a pass
+    # state carried across steps: sketch, walk and selection in full, attention
+    # on a seeded sample of query blocks
     it = oracle_head_layers(w)
     for _ in range(args.warmup):
         next(it)
-    times = [next(it) for _ in range(args.steps)]
-    step = statistics.mean(times) * w.hq * w.layers
-    value = w.n / step
+    runs = [next(it) for _ in range(args.steps)]
+    measured = statistics.mean(a + b for a, b, _ in runs)
+    full = statistics.mean(head_layer_estimate(*r) for r in runs) * w.hq * w.layers
+    value = w.n / full
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": measured * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
-                   "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": "replicas"},
+        "config": workload_config(w, world),
+        "extrapolated_ms_per_full_pass": full * 1e3,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
-                         "sample": f"each step: the oracle (fp64 numpy) on one head-layer (1 of {w.hq} query heads, "
-                                   f"1 of {w.layers} layers, every query block), scaled by the {w.hq * w.layers} "
-                                   f"head-layers of one pass"},
+                         "sample": f"each step: the oracle (fp64 numpy) on one head-layer ({w.hq} query heads x "
+                                   f"{w.layers} layers make a pass): sketch, walk and selection in full, attention "
+                                   f"of {min(w.b, ORACLE_SAMPLE_BLOCKS)} seeded query blocks of {w.b}; ms_per_step is "
+                                   f"that measured step; value extrapolates it linearly (attention by key-block "
+                                   f"pairs, then by the {w.hq * w.layers} head-layers) to the whole pass"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -272,8 +312,18 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------- ours ---
 
-def bench_prefill(args, world, S, W, torch):
-    w = W.PREFILL_16K
+def headline_workload(W):
+    """The N=1 workload: the longest prefill (131072 tokens, 4 layers) at 20% density."""
+    return W.PREFILL_128K
+
+
+def extra_workloads(W):
+    """The other prefill workloads, timed after the headline: the same long
+    context at 10% density, 65536 tokens over 8 layers, 16384 tokens over 4."""
+    return [W.PREFILL_128K_D10, W.PREFILL_64K, W.PREFILL_16K]
+
+
+def bench_prefill(args, world, S, W, torch, w, steps):
     cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
     h = S.Handle(cfg)
     path = S.PrefillPath(h, w.n, w.hq, w.hkv, torch.bfloat16)
@@ -300,7 +350,7 @@ def bench_prefill(args, world, S, W, torch):
     torch.cuda.synchronize()
     assert S.sws_sync_check(h) == 0
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(w.layers)]
-           for _ in range(args.steps)]
+           for _ in range(steps)]
     clocks = ClockSampler(gpu_bus_id(torch))
     clocks.start()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -308,7 +358,7 @@ def bench_prefill(args, world, S, W, torch):
     torch.cuda.synchronize()
     launches0 = S.sws_launch_count()
     t_start.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -320,7 +370,7 @@ def bench_prefill(args, world, S, W, torch):
     ms_max = max_over_ranks(ms, world)
     stage = {"sketch": 0.0, "walk_select": 0.0, "attention": 0.0}
     attn_ms = []
-    for i in range(args.steps):
+    for i in range(steps):
         for layer in range(w.layers):
             e = evs[i][layer]
             stage["sketch"] += e[0].elapsed_time(e[1])
@@ -328,18 +378,50 @@ def bench_prefill(args, world, S, W, torch):
             a = e[2].elapsed_time(e[3])
             stage["attention"] += a
             attn_ms.append(a)
-    stage = {k: v / args.steps for k, v in stage.items()}
+    stage = {k: v / steps for k, v in stage.items()}
     flops = w.hq * path.nnz * 4 * w.B * w.B * w.d  # executed block pairs x 4 B^2 d
     sketch_bytes = (w.hq + w.hkv) * w.n * w.d * 2 + 8 * (w.hq + w.hkv) * path.b * w.k + 8 * w.hq * path.b * (path.b + 1) // 2
-    res = dict(w=w, h=h, path=path, inputs=inputs, ms=ms_max, launches=launches, clocks=clk, stage=stage,
-               attn_ms=statistics.mean(attn_ms), flops=flops, sketch_bytes=sketch_bytes, in_bytes=in_bytes)
+    res = dict(w=w, h=h, path=path, inputs=inputs, ms=ms_max, steps=steps, launches=launches, clocks=clk,
+               stage=stage, attn_ms=statistics.mean(attn_ms), flops=flops, sketch_bytes=sketch_bytes,
+               in_bytes=in_bytes)
     return res
 
 
+def prefill_summary(pf, world, peaks, peak_kind) -> dict:
+    """tokens/s, the attention kernel's roofline (its peak chosen by the clocks the
+    timed region saw), the sketch stage's HBM roofline and the stage split."""
+    w = pf["w"]
+    ms_step = pf["ms"] / pf["steps"]
+    attn_tflops = pf["flops"] / (pf["attn_ms"] * 1e-3) / 1e12
+    # The burst GEMM peak was measured at full SM clocks, the sustained one under
+    # the power cap at lower clocks: take the one whose clocks the timed region saw.
+    sm, smx = pf["clocks"].get("sm_mhz"), pf["clocks"].get("sm_max_mhz")
+    burst = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    at_full_clock = sm is None or smx is None or sm >= 0.9 * smx
+    peak_t = burst if at_full_clock else sustained
+    peak_name = "bf16 burst" if at_full_clock else "bf16 sustained"
+    sk = pf["sketch_bytes"] / (pf["stage"]["sketch"] / w.layers * 1e-3) / 1e9
+    return {
+        "tokens_per_s": world * w.n / (ms_step * 1e-3), "ms_per_step": ms_step, "steps": pf["steps"],
+        "config": workload_config(w, world),
+        "stages_ms_per_step": pf["stage"],
+        "roofline": {"kernel": f"attn_tc_kernel<{w.d},{w.B}> (sws_sparse_attn_prefill)", "bound": "tensor",
+                     "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
+                     "traffic": profiled_traffic(f"attn_tc_prefill_n{w.n}_B{w.B}", "k_attn_tc.cu"),
+                     "peak_source": f"{peak_kind} {peak_name}",
+                     "frac_of_burst": attn_tflops / burst, "frac_of_sustained": attn_tflops / sustained,
+                     "flops_per_launch": pf["flops"], "ms_per_launch": pf["attn_ms"]},
+        "sketch_roofline": {"bound": "hbm", "achieved": sk, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": sk / peaks["hbm_gbs"], "bytes_per_layer": pf["sketch_bytes"]},
+        "clocks": pf["clocks"], "gpu_launches": pf["launches"],
+    }
+
+
 def bench_prefill_variants(args, world, S, W, torch, pf):
-    """The pages' own alternatives on the same inputs, timed like the headline
-    step: the entrywise walk power (the other reading of (.)^s) and the
-    dense-first-two-layers policy of §7."""
+    """The pages' own alternatives on the inputs of a prefill measurement (the
+    16384-token workload), timed like its step: the entrywise walk power (the
+    other reading of (.)^s) and the dense-first-two-layers policy of §7."""
     w, inputs = pf["w"], pf["inputs"]
     stream = torch.cuda.current_stream()
     steps = max(3, min(args.steps, 20))
@@ -706,46 +788,31 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return 0
-    pf = bench_prefill(args, world, S, W, torch)
-    w = pf["w"]
-    ms_step = pf["ms"] / args.steps
-    value = world * w.n / (ms_step * 1e-3)
-    attn_tflops = pf["flops"] / (pf["attn_ms"] * 1e-3) / 1e12
-    # The burst GEMM peak was measured at full SM clocks, the sustained one under
-    # the power cap at lower clocks: take the one whose clocks the timed region saw.
-    sm, smx = pf["clocks"].get("sm_mhz"), pf["clocks"].get("sm_max_mhz")
-    burst = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
-    sustained = peaks.get("bf16_tflops_sustained", burst)
-    at_full_clock = sm is None or smx is None or sm >= 0.9 * smx
-    peak_t = burst if at_full_clock else sustained
-    peak_name = "bf16 burst" if at_full_clock else "bf16 sustained"
+    w = headline_workload(W)
+    pf = bench_prefill(args, world, S, W, torch, w, args.steps)
+    head = prefill_summary(pf, world, peaks, peak_kind)
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded AR(1) + sink + hub generator (sws_inputs); no datasets or weights",
-        "config": {"workload": w.name, "layers": w.layers, "hq": w.hq, "hkv": w.hkv, "d": w.d, "n": w.n, "B": w.B,
-                   "k": w.k, "s": w.s, "density": f"{w.density[0]}/{w.density[1]}", "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2 ({pf['in_bytes'] / 1e6:.0f} MB per step)"},
-        "stages_ms_per_step": pf["stage"],
-        "roofline": {"kernel": "sws_sparse_attn_prefill", "bound": "tensor", "achieved": attn_tflops, "peak": peak_t,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
-                     "traffic": profiled_traffic("attn_tc_prefill_n16384_B64", "k_attn_tc.cu"),
-                     "peak_source": f"{peak_kind} {peak_name}",
-                     "frac_of_burst": attn_tflops / burst, "frac_of_sustained": attn_tflops / sustained, "flops_per_launch": pf["flops"],
-                     "ms_per_launch": pf["attn_ms"]},
-        "sketch_roofline": {"bound": "hbm", "achieved": pf["sketch_bytes"] / (pf["stage"]["sketch"] / w.layers * 1e-3) / 1e9,
-                            "peak": peaks["hbm_gbs"], "unit": "GB/s"},
-        "clocks": pf["clocks"], "gpu_launches": pf["launches"],
+        "config": head["config"], "stages_ms_per_step": head["stages_ms_per_step"], "roofline": head["roofline"],
+        "sketch_roofline": head["sketch_roofline"], "clocks": head["clocks"], "gpu_launches": head["gpu_launches"],
     }
-    line["sketch_roofline"]["frac"] = line["sketch_roofline"]["achieved"] / peaks["hbm_gbs"]
     if not args.no_e2e:
         line["e2e"] = bench_prefill_e2e(args, world, S, torch, pf)
-    if not args.no_variants:
-        line["variants"] = bench_prefill_variants(args, world, S, W, torch, pf)
     pf["h"].close()
     del pf
     torch.cuda.empty_cache()
+    line["prefill_workloads"] = {}
+    for wx in extra_workloads(W):
+        px = bench_prefill(args, world, S, W, torch, wx, max(3, min(args.steps, 20)))
+        line["prefill_workloads"][wx.name] = prefill_summary(px, world, peaks, peak_kind)
+        if wx is W.PREFILL_16K and not args.no_variants:
+            line["variants"] = bench_prefill_variants(args, world, S, W, torch, px)
+        px["h"].close()
+        del px
+        torch.cuda.empty_cache()
     if not args.no_decode:
         line["decode"] = bench_decode(args, world, S, W, torch, peaks)
         if not args.no_variants:
@@ -753,7 +820,7 @@ def main():
             line["decode"].setdefault("variants", {})["exact_walk_n16384"] = bench_decode_exact(args, world, S, W,
                                                                                                  torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(W.PREFILL_16K)
+        line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         s = json.dumps(line)
         print(s, flush=True)

@@ -68,6 +68,10 @@ def test_reference_arm_under_torchrun_prints_one_line():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload and config dict as the main arm's line at this world size
+    import sws_inputs as W
+    assert line["config"] == bench.workload_config(bench.headline_workload(W), 2)
+    assert line["ms_per_step"] > 0 and line["extrapolated_ms_per_full_pass"] > line["ms_per_step"]
 
 
 def test_clock_parser_flags_throttle_reasons():
