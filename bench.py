@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--decode-layers", type=int, default=None, help="fewer decode layers (profiling only)")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement (profiling only)")
     ap.add_argument("--no-variants", action="store_true", help="skip the elementwise-walk and dense-first variants")
+    ap.add_argument("--profile-prefill", action="store_true",
+                    help="profiling run: the headline prefill workload alone (scaled by --prefill-n), no bench line")
+    ap.add_argument("--prefill-n", type=int, default=None, help="tokens of the profiled prefill workload")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -383,8 +386,59 @@ def bench_prefill(args, world, S, W, torch, w, steps):
     sketch_bytes = (w.hq + w.hkv) * w.n * w.d * 2 + 8 * (w.hq + w.hkv) * path.b * w.k + 8 * w.hq * path.b * (path.b + 1) // 2
     res = dict(w=w, h=h, path=path, inputs=inputs, ms=ms_max, steps=steps, launches=launches, clocks=clk,
                stage=stage, attn_ms=statistics.mean(attn_ms), flops=flops, sketch_bytes=sketch_bytes,
-               in_bytes=in_bytes)
+               in_bytes=in_bytes, mma_work=mma_work(path, w, torch))
     return res
+
+
+# Whether attn_tc_kernel skips the products of a (query tile, key tile) pair in
+# which no query block of the tile selected a key block of the tile.
+ATTN_SKIPS_UNSELECTED_TILES = False
+
+
+def mma_work(path, w, torch) -> dict:
+    """Tensor-core work that attn_tc_kernel executes for the last layer's CSR
+    against the algorithmic work (4 B^2 d flops per selected block pair). The
+    kernel takes 256 query rows at a time (two 128-row tiles) over the union of
+    their query blocks' key blocks, 128 keys per tile, and runs both tiles' score
+    and PV products on every key tile of the union unless a tile has no selected
+    pair, which it skips."""
+    b, B, QB = path.b, w.B, 256 // w.B
+    rp = path.row_ptr.long()
+    ci = path.col_idx.long()
+    sel = torch.zeros(w.hq, b, b, dtype=torch.bool, device=rp.device)
+    rows = torch.repeat_interleave(torch.arange(b, device=rp.device), rp[0, 1:] - rp[0, :-1])
+    for h in range(w.hq):
+        sel[h, rows, ci[h, :rows.numel()]] = True
+    nslab = -(-b // QB)
+    pad = torch.zeros(w.hq, nslab * QB, b, dtype=torch.bool, device=rp.device)
+    pad[:, :b] = sel
+    slab = pad.reshape(w.hq, nslab, QB, b)
+    union = slab.any(dim=2)                                    # [hq, slab, key block]
+    kb_per_tile = 128 // B
+    # key tiles of the merged stream: union blocks taken kb_per_tile at a time
+    tiles = (union.sum(dim=2) + kb_per_tile - 1) // kb_per_tile  # [hq, slab]
+    qpt = 128 // B  # query blocks per 128-row tile
+    tile_sel = slab.reshape(w.hq, nslab, 2, qpt, b).any(dim=3)  # [hq, slab, query tile, key block]
+    if ATTN_SKIPS_UNSELECTED_TILES:
+        # a query tile runs a key tile only if one of its query blocks selected one of the tile's key blocks
+        ts = tile_sel[..., :b]
+        if kb_per_tile > 1:  # key tiles are consecutive union blocks: count per merged tile
+            executed = 0
+            for h in range(w.hq):
+                for p in range(nslab):
+                    blocks = union[h, p].nonzero().flatten()
+                    for t in range(0, blocks.numel(), kb_per_tile):
+                        blk = blocks[t:t + kb_per_tile]
+                        executed += int(ts[h, p][:, blk].any(dim=1).sum().item())
+        else:
+            executed = int(ts.sum().item())
+    else:
+        executed = 2 * int(tiles.sum().item())  # both query tiles on every key tile of the union
+    algorithmic = int(sel.sum().item())
+    flops_tile = 4 * 128 * 128 * w.d
+    return {"executed_tile_products": executed, "selected_block_pairs": algorithmic,
+            "executed_flops": executed * flops_tile, "algorithmic_flops": algorithmic * 4 * B * B * w.d,
+            "executed_over_algorithmic": executed * flops_tile / (algorithmic * 4 * B * B * w.d)}
 
 
 def prefill_summary(pf, world, peaks, peak_kind) -> dict:
@@ -415,6 +469,7 @@ def prefill_summary(pf, world, peaks, peak_kind) -> dict:
         "sketch_roofline": {"bound": "hbm", "achieved": sk, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": sk / peaks["hbm_gbs"], "bytes_per_layer": pf["sketch_bytes"]},
         "clocks": pf["clocks"], "gpu_launches": pf["launches"],
+        "attention_mma_work": pf["mma_work"],
     }
 
 
@@ -684,6 +739,8 @@ def bench_decode(args, world, S, W, torch, peaks):
             "step_us": sh_ms * 1e3, "kv_bytes_per_step": sh_kv, "union_blocks_per_unit": float(us.mean().item()),
             "hbm_gbs": (sh_kv + sk_bytes + tok_bytes) / (sh_ms * 1e-3) / 1e9}}
         hs.close()
+        out["variants"]["exact_walk_rows"] = bench_decode_exact_rows(args, world, S, W, torch, wd, path, toks_q,
+                                                                     toks_k, toks_v, warm, union_log)
         # the paged cache: the same caches moved to a pool whose pages hold the
         # blocks in a seeded random order, the same steps replayed
         perm = torch.randperm(wd.batch * path.mb, generator=torch.Generator().manual_seed(wd.seed))
@@ -708,6 +765,79 @@ def bench_decode(args, world, S, W, torch, peaks):
             "same_selection_as_contiguous": bool(torch.equal(up, u))}
     h.close()
     return out
+
+
+def bench_decode_exact_rows(args, world, S, W, torch, wd, path, toks_q, toks_k, toks_v, warm, union_log):
+    """The exact decode walk with stored rows (sws_decode_step_exact_rows) on the
+    decode workload's own caches and tokens: the prompt's queries give every
+    block's q~ (one sequence at a time), the rows of every layer are built, and
+    the same steps are replayed with the exact walk selecting."""
+    cfg = path.h.cfg
+    h = S.Handle(S.make_config(wd.d, wd.B, wd.k, wd.s, 0, wd.density, wd.seed))
+    lens = torch.full((wd.batch,), wd.n0, dtype=torch.int32, device="cuda")
+    path.init_cache(lens)
+    f64 = dict(dtype=torch.float64, device="cuda")
+    q_psum = [torch.zeros(wd.batch, wd.hq, wd.d, **f64) for _ in range(wd.layers)]
+    q_sketch = [torch.zeros(wd.batch, wd.hq, path.mb, wd.k, **f64) for _ in range(wd.layers)]
+    e = S.sws_decode_exact_rows_entries(cfg, wd.max_len)
+    rows = [torch.empty(wd.batch, wd.hq, e, dtype=torch.int32, device="cuda") for _ in range(wd.layers)]
+    for layer in range(wd.layers):
+        for s_ in range(wd.batch):
+            Q = W.decode_sequence_queries(wd, s_, layer, "cuda")[None]  # [1, hq, max_len, d]
+            S.sws_decode_init_cache(h, Q, path.seq_lens[s_:s_ + 1], q_psum[layer][s_:s_ + 1],
+                                    q_sketch[layer][s_:s_ + 1])
+            del Q
+        S.sws_decode_exact_rows_init(h, q_sketch[layer], path.k_sketch[layer], path.seq_lens, rows[layer])
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * wd.layers + 1)] for _ in range(wd.steps)]
+
+    def step(t, rec):
+        path.begin_step()
+        if rec:
+            ev[t][0].record(stream)
+        for layer in range(wd.layers):
+            S.sws_decode_step_exact_rows(h, toks_q[t, layer], toks_k[t, layer], toks_v[t, layer], path.seq_lens,
+                                         path.k_cache[layer], path.v_cache[layer], path.k_psum[layer],
+                                         path.k_sketch[layer], q_psum[layer], q_sketch[layer], rows[layer],
+                                         layer == 0, path.walk_state, path.head_sel, path.head_cnt, path.sel,
+                                         path.sel_mask, path.sel_cnt)
+            if rec:
+                ev[t][1 + 2 * layer].record(stream)
+            S.sws_sparse_attn_decode(h, toks_q[t, layer], path.k_cache[layer], path.v_cache[layer], path.seq_lens,
+                                     path.sel, path.sel_mask, path.sel_cnt, path.o, path.ws)
+            if rec:
+                ev[t][2 + 2 * layer].record(stream)
+            union_log[t, layer].copy_(path.sel_cnt, non_blocking=True)
+
+    for t in range(warm):
+        step(t, False)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for t in range(warm, wd.steps):
+        step(t, True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    timed = wd.steps - warm
+    ms = max_over_ranks(a.elapsed_time(b), world) / timed
+    sel_ms = statistics.mean(ev[t][2 * l].elapsed_time(ev[t][1 + 2 * l]) for t in range(warm, wd.steps)
+                             for l in range(wd.layers))
+    attn_ms = statistics.mean(ev[t][1 + 2 * l].elapsed_time(ev[t][2 + 2 * l]) for t in range(warm, wd.steps)
+                              for l in range(wd.layers))
+    u = union_log[warm:].double()
+    rows_bytes = wd.batch * wd.hq * e * 4  # one layer's stored rows, read once by the products (s <= 8)
+    h.close()
+    del rows, q_psum, q_sketch
+    return {"workload": wd.name, "step_us": ms * 1e3, "steps_timed": timed,
+            "union_blocks_per_unit": float(u.mean().item()),
+            "kv_bytes_per_step": float(u.sum().item()) * wd.B * wd.d * 2 * 2 / timed,
+            "stages_us_per_layer": {"exact_select": sel_ms * 1e3, "attention": attn_ms * 1e3},
+            "rows_bytes_per_layer": rows_bytes,
+            "select_stage_gbs_on_rows": rows_bytes / (sel_ms * 1e-3) / 1e9}
 
 
 def bench_decode_exact(args, world, S, W, torch):
@@ -787,6 +917,16 @@ def main():
             import torch.distributed as dist
             dist.barrier()
             dist.destroy_process_group()
+        return 0
+    if args.profile_prefill:
+        # profiling run of one prefill workload (for ncu captures): not a benchmark line
+        wp = headline_workload(W)
+        if args.prefill_n:
+            wp = wp.scaled(name=f"prefill_n{args.prefill_n}_B{wp.B}_k{wp.k}_L{wp.layers}", n=args.prefill_n)
+        px = bench_prefill(args, world, S, W, torch, wp, args.steps)
+        if rank == 0:
+            print(json.dumps({"profiling_only": True, "prefill": prefill_summary(px, world, peaks, peak_kind)}),
+                  flush=True)
         return 0
     w = headline_workload(W)
     pf = bench_prefill(args, world, S, W, torch, w, args.steps)

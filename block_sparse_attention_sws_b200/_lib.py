@@ -25,10 +25,11 @@ SWS_OP_SKETCH, SWS_OP_WALK_SELECT, SWS_OP_PREFILL_ATTN, SWS_OP_DECODE_ATTN = ran
 EXPORTS = [
     "sws_status_string", "sws_config_check", "sws_num_blocks", "sws_csr_nnz", "sws_build_projection_host",
     "sws_workspace_size", "sws_create", "sws_destroy", "sws_projection_device", "sws_launch_count",
-    "sws_sync_check", "sws_sketch",
-    "sws_walk_select", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
+    "sws_sync_check", "sws_layout_check", "sws_sketch",
+    "sws_walk_select", "sws_walk_select_sketch", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
     "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc", "sws_decode_init_cache_paged", "sws_decode_step_paged",
-    "sws_sparse_attn_decode_paged", "sws_decode_step_exact",
+    "sws_sparse_attn_decode_paged", "sws_decode_step_exact", "sws_decode_exact_rows_entries",
+    "sws_decode_exact_rows_init", "sws_decode_step_exact_rows",
 ]
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SWS_NOALLOC_SCRATCH_BYTES
 
@@ -71,9 +72,12 @@ def load() -> ctypes.CDLL:
         "sws_projection_device": (P, [P]),
         "sws_launch_count": (U64, []),
         "sws_sync_check": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
-        "sws_sketch": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, SZ, P]),
+        "sws_sketch": (ctypes.c_int, [P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, P, P, SZ, P]),
+        "sws_layout_check": (ctypes.c_int, [CFG, ctypes.c_int, I64, P]),
         "sws_walk_select": (ctypes.c_int, [P, P, I64, I32, ctypes.c_int, P, P, P, P, SZ, P]),
-        "sws_sparse_attn_prefill": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, SZ, P]),
+        "sws_walk_select_sketch": (ctypes.c_int, [P, P, P, I64, I32, I32, ctypes.c_int, P, P, P, P, SZ, P]),
+        "sws_sparse_attn_prefill": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, P, P, P, P,
+                                                   SZ, P]),
         "sws_decode_init_cache": (ctypes.c_int, [P, P, I32, I32, I64, P, P, P, P]),
         "sws_decode_advance": (ctypes.c_int, [P, P, I32, P]),
         "sws_decode_step": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, ctypes.c_int, P, P, P, P,
@@ -83,6 +87,10 @@ def load() -> ctypes.CDLL:
         "sws_decode_init_cache_paged": (ctypes.c_int, [P, P, I64, P, I64, I32, I32, P, P, P, P]),
         "sws_decode_step_exact": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, P, ctypes.c_int,
                                                  P, P, P, P, P, P, P]),
+        "sws_decode_exact_rows_entries": (I64, [CFG, I64]),
+        "sws_decode_exact_rows_init": (ctypes.c_int, [P, P, P, I32, I32, I32, I64, P, P, P]),
+        "sws_decode_step_exact_rows": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, P, P, P,
+                                                      ctypes.c_int, P, P, P, P, P, P, P]),
         "sws_decode_step_paged": (ctypes.c_int, [P, P, P, P, I32, I32, I32, P, P, I64, P, I64, P, P, P, ctypes.c_int,
                                                  P, P, P, P, P, P, P]),
         "sws_sparse_attn_decode_paged": (ctypes.c_int, [P, P, P, P, I64, P, I64, I32, I32, I32, P, P, P, P, P, P, SZ,
@@ -117,6 +125,17 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return t.data_ptr()
+
+
+def _head_tok(t: torch.Tensor):
+    """(pointer, strides) of a [heads, n, d] operand: strides None when it is
+    dense, else the (head, token) element strides of a view whose rows are
+    contiguous (e.g. x.transpose(0, 1) of a [n, heads, d] activation)."""
+    if t.dim() != 3 or t.stride(-1) != 1:
+        raise ValueError("operands are [heads, n, d] with contiguous rows")
+    if t.is_contiguous():
+        return t.data_ptr(), None
+    return t.data_ptr(), (ctypes.c_int64 * 2)(t.stride(0), t.stride(1))
 
 
 def _stream(stream) -> int:
@@ -210,9 +229,12 @@ def sws_sync_check(h: Handle, stream=None) -> int:
 # --------------------------------------------------------------- prefill ----
 
 def sws_sketch(h: Handle, q, k, q_sk, k_sk, scores, ws, stream=None) -> None:
+    """q [hq, n, d], k [hkv, n, d]: dense or strided views with contiguous rows;
+    scores None skips the score matrix (see sws_walk_select_sketch)."""
     hq, n, _ = q.shape
     hkv = k.shape[0]
-    _check(load().sws_sketch(h.ptr, _ptr(q), _ptr(k), _dtype_code(q), n, hq, hkv, _ptr(q_sk), _ptr(k_sk),
+    (qp, qs), (kp, ks) = _head_tok(q), _head_tok(k)
+    _check(load().sws_sketch(h.ptr, qp, kp, _dtype_code(q), n, hq, hkv, qs, ks, _ptr(q_sk), _ptr(k_sk),
                              _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sws_sketch")
 
 
@@ -224,13 +246,23 @@ def sws_walk_select(h: Handle, scores, n: int, first_layer: bool, walk_state, ro
                                   _stream(stream)), "sws_walk_select")
 
 
+def sws_walk_select_sketch(h: Handle, q_sk, k_sk, n: int, first_layer: bool, walk_state, row_ptr, col_idx, ws,
+                           stream=None) -> None:
+    hq, hkv = q_sk.shape[0], k_sk.shape[0]
+    _check(load().sws_walk_select_sketch(h.ptr, _ptr(q_sk), _ptr(k_sk), n, hq, hkv, int(bool(first_layer)),
+                                         _ptr(walk_state), _ptr(row_ptr), _ptr(col_idx), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)), "sws_walk_select_sketch")
+
+
 def sws_sparse_attn_prefill(h: Handle, q, k, v, row_ptr, col_idx, o, ws=None, stream=None) -> None:
+    """q, o [hq, n, d], k, v [hkv, n, d]: dense or strided views with contiguous rows."""
     hq, n, _ = q.shape
     hkv = k.shape[0]
     wsp = _ptr(ws) if ws is not None else None
     wsb = ws.numel() * ws.element_size() if ws is not None else 0
-    _check(load().sws_sparse_attn_prefill(h.ptr, _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), n, hq, hkv, _ptr(row_ptr),
-                                          _ptr(col_idx), _ptr(o), wsp, wsb, _stream(stream)),
+    (qp, qs), (kp, ks), (vp, vs), (op, os_) = _head_tok(q), _head_tok(k), _head_tok(v), _head_tok(o)
+    _check(load().sws_sparse_attn_prefill(h.ptr, qp, kp, vp, _dtype_code(q), n, hq, hkv, qs, ks, vs, os_,
+                                          _ptr(row_ptr), _ptr(col_idx), op, wsp, wsb, _stream(stream)),
            "sws_sparse_attn_prefill")
 
 
@@ -324,3 +356,33 @@ def sws_decode_step_exact(h: Handle, q_tok, k_tok, v_tok, seq_lens, k_cache, v_c
                                         _ptr(q_psum), _ptr(q_sketch), int(bool(first_layer)), _ptr(walk_state),
                                         _ptr(head_sel), _ptr(head_cnt), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
                                         _stream(stream)), "sws_decode_step_exact")
+
+
+def sws_decode_exact_rows_entries(cfg: SwsConfig, max_len: int) -> int:
+    n = load().sws_decode_exact_rows_entries(ctypes.byref(cfg), max_len)
+    if n < 0:
+        raise SwsError(SWS_ERR_INVALID_ARG, "sws_decode_exact_rows_entries")
+    return n
+
+
+def sws_decode_exact_rows_init(h: Handle, q_sketch, k_sketch, seq_lens, rows, stream=None) -> None:
+    """q_sketch [batch, hq, max_blocks, k], k_sketch [batch, hkv, max_blocks, k] (fp64);
+    rows [batch, hq, E] int32 (uint32 entries), E = sws_decode_exact_rows_entries."""
+    batch, hq, mb, _ = q_sketch.shape
+    hkv = k_sketch.shape[1]
+    max_len = mb * h.cfg.block_size
+    _check(load().sws_decode_exact_rows_init(h.ptr, _ptr(q_sketch), _ptr(k_sketch), batch, hq, hkv, max_len,
+                                             _ptr(seq_lens), _ptr(rows), _stream(stream)), "sws_decode_exact_rows_init")
+
+
+def sws_decode_step_exact_rows(h: Handle, q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch, q_psum,
+                               q_sketch, rows, first_layer: bool, walk_state, head_sel, head_cnt, sel, sel_mask,
+                               sel_cnt, stream=None) -> None:
+    batch, hq, _ = q_tok.shape
+    hkv, max_len = k_cache.shape[1], k_cache.shape[2]
+    _check(load().sws_decode_step_exact_rows(h.ptr, _ptr(q_tok), _ptr(k_tok), _ptr(v_tok), batch, hq, hkv, max_len,
+                                             _ptr(seq_lens), _ptr(k_cache), _ptr(v_cache), _ptr(k_psum),
+                                             _ptr(k_sketch), _ptr(q_psum), _ptr(q_sketch), _ptr(rows),
+                                             int(bool(first_layer)), _ptr(walk_state), _ptr(head_sel),
+                                             _ptr(head_cnt), _ptr(sel), _ptr(sel_mask), _ptr(sel_cnt),
+                                             _stream(stream)), "sws_decode_step_exact_rows")

@@ -18,7 +18,7 @@ namespace {
 template <typename T, int D, int B>
 __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, int64_t n, int32_t group,
-                                                          const int32_t* __restrict__ row_ptr,
+                                                          PrefillLayout lay, const int32_t* __restrict__ row_ptr,
                                                           const int32_t* __restrict__ col_idx, int64_t nnz,
                                                           T* __restrict__ o, float qscale, int32_t* err) {
   grid_dependency_wait();
@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
   const bool qvalid = t < n;
 
   float qv[HD], acc[HD];
-  const T* qrow = q + ((int64_t)h * n + (qvalid ? t : 0)) * D + half * HD;
+  const T* qrow = q + h * lay.q.head + (qvalid ? t : 0) * lay.q.tok + half * HD;
 #pragma unroll
   for (int c = 0; c < HD; ++c) {
     qv[c] = qvalid ? to_f32(qrow[c]) * qscale : 0.f;
@@ -53,8 +53,8 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
     e0 = e1 = 0;
   }
   const int32_t* cols = col_idx + (int64_t)h * nnz;
-  const T* kh = k + (int64_t)g * n * D;
-  const T* vh = v + (int64_t)g * n * D;
+  const T* kh = k + g * lay.k.head;
+  const T* vh = v + g * lay.v.head;
 
   for (int32_t e = e0; e < e1; ++e) {
     const int64_t j = cols[e];
@@ -66,11 +66,11 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
     const int64_t u0 = j * B;
     const int rows = static_cast<int>(std::min<int64_t>(B, n - u0));
     for (int x = threadIdx.x; x < B * D / VE; x += blockDim.x) {
-      const int rr = x / (D / VE);
+      const int rr = x / (D / VE), cv = x % (D / VE);
       uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
       if (rr < rows) {
-        kv = *reinterpret_cast<const uint4*>(kh + u0 * D + (int64_t)x * VE);
-        vv = *reinterpret_cast<const uint4*>(vh + u0 * D + (int64_t)x * VE);
+        kv = *reinterpret_cast<const uint4*>(kh + (u0 + rr) * lay.k.tok + cv * VE);
+        vv = *reinterpret_cast<const uint4*>(vh + (u0 + rr) * lay.v.tok + cv * VE);
       }
       reinterpret_cast<uint4*>(Ks)[x] = kv;
       reinterpret_cast<uint4*>(Vs)[x] = vv;
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
   }
   if (qvalid) {
     const float inv = 1.f / l;
-    T* orow = o + ((int64_t)h * n + t) * D + half * HD;
+    T* orow = o + h * lay.o.head + t * lay.o.tok + half * HD;
 #pragma unroll
     for (int c = 0; c < HD; ++c) orow[c] = from_f32<T>(acc[c] * inv);
   }
@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(2 * B) attn_simt_kernel(const T* __restrict__ 
 
 template <typename T, int D, int B>
 cudaError_t launch_t(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n, int32_t hq,
-                     int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o, cudaStream_t st) {
+                     int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                     cudaStream_t st) {
   const size_t smem = 2 * (size_t)B * D * sizeof(T) + (size_t)B * (B + 1) * sizeof(float);
   auto kern = attn_simt_kernel<T, D, B>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -126,7 +127,7 @@ cudaError_t launch_t(const sws_handle* h, const void* q, const void* k, const vo
   dim3 grid(static_cast<unsigned>(b), hq);
   {
     const cudaError_t le = launch_k(kern, grid, 2 * B, smem, st, static_cast<const T*>(q), static_cast<const T*>(k),
-                                    static_cast<const T*>(v), n, hq / hkv, row_ptr, col_idx, nnz, static_cast<T*>(o),
+                                    static_cast<const T*>(v), n, hq / hkv, lay, row_ptr, col_idx, nnz, static_cast<T*>(o),
                                     qscale, h->err);
     if (le != cudaSuccess) return le;
   }
@@ -136,21 +137,22 @@ cudaError_t launch_t(const sws_handle* h, const void* q, const void* k, const vo
 
 template <typename T>
 cudaError_t launch_d(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n, int32_t hq,
-                     int32_t hkv, const int32_t* rp, const int32_t* ci, void* o, cudaStream_t st) {
+                     int32_t hkv, const PrefillLayout& lay, const int32_t* rp, const int32_t* ci, void* o,
+                     cudaStream_t st) {
   const int d = h->cfg.head_dim, B = h->cfg.block_size;
-  if (d == 128 && B == 128) return launch_t<T, 128, 128>(h, q, k, v, n, hq, hkv, rp, ci, o, st);
-  if (d == 128 && B == 64) return launch_t<T, 128, 64>(h, q, k, v, n, hq, hkv, rp, ci, o, st);
-  if (d == 64 && B == 128) return launch_t<T, 64, 128>(h, q, k, v, n, hq, hkv, rp, ci, o, st);
-  return launch_t<T, 64, 64>(h, q, k, v, n, hq, hkv, rp, ci, o, st);
+  if (d == 128 && B == 128) return launch_t<T, 128, 128>(h, q, k, v, n, hq, hkv, lay, rp, ci, o, st);
+  if (d == 128 && B == 64) return launch_t<T, 128, 64>(h, q, k, v, n, hq, hkv, lay, rp, ci, o, st);
+  if (d == 64 && B == 128) return launch_t<T, 64, 128>(h, q, k, v, n, hq, hkv, lay, rp, ci, o, st);
+  return launch_t<T, 64, 64>(h, q, k, v, n, hq, hkv, lay, rp, ci, o, st);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_prefill_simt(const sws_handle* h, const void* q, const void* k, const void* v, sws_dtype dt,
-                                     int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
-                                     const int32_t* col_idx, void* o, cudaStream_t st) {
-  if (dt == SWS_BF16) return launch_d<__nv_bfloat16>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st);
-  return launch_d<float>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st);
+                                     int64_t n, int32_t hq, int32_t hkv, const PrefillLayout& lay,
+                                     const int32_t* row_ptr, const int32_t* col_idx, void* o, cudaStream_t st) {
+  if (dt == SWS_BF16) return launch_d<__nv_bfloat16>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st);
+  return launch_d<float>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st);
 }
 
 }  // namespace sws

@@ -346,7 +346,8 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
     const __grid_constant__ CUtensorMap tmv, int64_t n, int32_t hq, int32_t group, const int32_t* __restrict__ row_ptr,
-    const int32_t* __restrict__ col_idx, int64_t nnz, __nv_bfloat16* __restrict__ o, float qscale, int32_t* err) {
+    const int32_t* __restrict__ col_idx, int64_t nnz, __nv_bfloat16* __restrict__ o, HeadTok os, float qscale,
+    int32_t* err) {
   grid_dependency_wait();
   allow_dependents();
   using L = Smem<D>;
@@ -658,7 +659,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
       if (!(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = o + (static_cast<int64_t>(h) * n + tok) * D;
+      __nv_bfloat16* orow = o + h * os.head + tok * os.tok;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
@@ -706,13 +707,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [heads][rows][D] bf16 as a 3-D tensor map with a {64, box_rows, 1} box, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, int D, int box_rows) {
+// [heads][rows][D] bf16 (rows and heads at the given element strides) as a 3-D
+// tensor map with a {64, box_rows, 1} box, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, int D, int box_rows, HeadTok st) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(st.tok) * 2, static_cast<cuuint64_t>(st.head) * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -722,10 +724,11 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, i
 
 template <int D, int BLK>
 cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n, int32_t hq,
-                      int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o, cudaStream_t st) {
+                      int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr, const int32_t* col_idx, void* o,
+                      cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, n, hq, D, kTileM) || !make_map(&mk, k, n, hkv, D, BLK == 128 ? 128 : 64) ||
-      !make_map(&mv, v, n, hkv, D, BLK == 128 ? 128 : 64))
+  if (!make_map(&mq, q, n, hq, D, kTileM, lay.q) || !make_map(&mk, k, n, hkv, D, BLK == 128 ? 128 : 64, lay.k) ||
+      !make_map(&mv, v, n, hkv, D, BLK == 128 ? 128 : 64, lay.v))
     return cudaErrorInvalidValue;
   const size_t smem = Smem<D>::total + 1024;
   auto kern = attn_tc_kernel<D, BLK>;
@@ -739,7 +742,7 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
   const float qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
   {
     const cudaError_t le = launch_k(kern, grid, kTcThreads, smem, st, mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx,
-                                    nnz, static_cast<__nv_bfloat16*>(o), qscale, h->err);
+                                    nnz, static_cast<__nv_bfloat16*>(o), lay.o, qscale, h->err);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);
@@ -749,15 +752,15 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
 }  // namespace
 
 cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
-                                   int32_t hq, int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o,
-                                   cudaStream_t st) {
+                                   int32_t hq, int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr,
+                                   const int32_t* col_idx, void* o, cudaStream_t st) {
   const int d = h->cfg.head_dim, B = h->cfg.block_size;
   if (d == 128) {
-    return B == 128 ? launch_tc<128, 128>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st)
-                    : launch_tc<128, 64>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st);
+    return B == 128 ? launch_tc<128, 128>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st)
+                    : launch_tc<128, 64>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st);
   }
-  return B == 128 ? launch_tc<64, 128>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st)
-                  : launch_tc<64, 64>(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st);
+  return B == 128 ? launch_tc<64, 128>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st)
+                  : launch_tc<64, 64>(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st);
 }
 
 }  // namespace sws

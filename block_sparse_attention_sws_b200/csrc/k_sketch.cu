@@ -5,7 +5,7 @@
 // Q~ K~^T / sqrt(k) under the causal block mask).
 //
 // 1. pool_project_kernel: one streaming pass over Q and K (one launch for
-//    both): 16-byte loads of each contiguous B x d block, per-column sums,
+//    both): 16-byte loads of the B rows of each block, per-column sums,
 //    the means, and their projection q~ = q_bar H_d, k~ = k_bar H_d as a
 //    Walsh-Hadamard transform in registers and shuffles. HBM-bound:
 //    Q and K are read exactly once and only the b x k sketches are written.
@@ -32,8 +32,8 @@ constexpr int kPoolBatch = 16;  // 16-byte loads in flight per lane
 
 // Block means of Q (heads [0, hq)) and K (heads [hq, hq + hkv)) and their
 // projection by H_d, in one pass over Q and K. One warp per (head, block)
-// item, items dealt round-robin over all warps of the grid; a block is one
-// contiguous rows x D tile, so lane l always reads the same 16 bytes of
+// item, items dealt round-robin over all warps of the grid; a block is B rows
+// of D contiguous elements (rows at the tensor's token stride), so lane l always reads the same 16 bytes of
 // columns (vector l mod VR of a row) on rows l / VR, l / VR + 32 / VR, ...,
 // kPoolBatch of them in flight at a time. bf16 columns are summed in fp32 over
 // one batch of rows, then in fp64; fp32 inputs are summed in fp64 throughout.
@@ -47,8 +47,9 @@ constexpr int kPoolBatch = 16;  // 16-byte loads in flight per lane
 template <typename T, int D>
 __global__ void __launch_bounds__(kPoolWarps * 32, 2)
     pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
-                        int32_t B, int64_t nblk, const double* __restrict__ sign, const int32_t* __restrict__ col,
-                        double scale, int32_t ksk, double* __restrict__ q_sk, double* __restrict__ k_sk) {
+                        HeadTok qs, HeadTok ks, int32_t B, int64_t nblk, const double* __restrict__ sign,
+                        const int32_t* __restrict__ col, double scale, int32_t ksk, double* __restrict__ q_sk,
+                        double* __restrict__ k_sk) {
   grid_dependency_wait();
   allow_dependents();
   constexpr int VE = 16 / sizeof(T);  // elements per 16-byte vector
@@ -76,7 +77,8 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
     const int64_t head = it / nblk, blk = it % nblk;
     const int64_t r0 = blk * B;
     const int rows = static_cast<int>(n - r0 < B ? n - r0 : (int64_t)B);
-    const T* src = (head < hq ? q + (head * n + r0) * D : k + ((head - hq) * n + r0) * D) + vc * VE;
+    const int64_t rs = head < hq ? qs.tok : ks.tok;  // elements from one row to the next
+    const T* src = (head < hq ? q + head * qs.head : k + (head - hq) * ks.head) + r0 * rs + vc * VE;
 
     double acc[VE];
 #pragma unroll
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
 #pragma unroll
       for (int u = 0; u < kPoolBatch; ++u) {
         const int r = rb + u * LPC;
-        v[u] = r < rows ? ld_stream16(src + (size_t)r * D) : make_uint4(0u, 0u, 0u, 0u);
+        v[u] = r < rows ? ld_stream16(src + r * rs) : make_uint4(0u, 0u, 0u, 0u);
       }
       if constexpr (sizeof(T) == 2) {
         float part[VE];
@@ -248,14 +250,14 @@ __global__ void __launch_bounds__(64, 8)
 
 template <typename T, int D>
 cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int64_t n, int32_t hq, int32_t hkv,
-                                double* q_sk, double* k_sk, cudaStream_t st) {
+                                HeadTok qs, HeadTok ks, double* q_sk, double* k_sk, cudaStream_t st) {
   const int32_t B = h->cfg.block_size;
   const int64_t nblk = ceil_div64(n, B);
   const int64_t total = (int64_t)(hq + hkv) * nblk;
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 2 * (int64_t)h->num_sms));
   {
-    const cudaError_t le = launch_k(pool_project_kernel<T, D>, grid, kPoolWarps * 32, 0, st, q, k, n, hq, hkv, B, nblk,
-                                    h->sign, h->col, h->scale, h->cfg.sketch_dim, q_sk, k_sk);
+    const cudaError_t le = launch_k(pool_project_kernel<T, D>, grid, kPoolWarps * 32, 0, st, q, k, n, hq, hkv, qs, ks,
+                                    B, nblk, h->sign, h->col, h->scale, h->cfg.sketch_dim, q_sk, k_sk);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);
@@ -267,18 +269,19 @@ cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int
 size_t sketch_workspace_bytes(const sws_config&, int64_t, int32_t, int32_t) { return 0; }
 
 cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
-                                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, cudaStream_t st) {
+                                       int32_t hq, int32_t hkv, HeadTok qs, HeadTok ks, double* q_sk, double* k_sk,
+                                       cudaStream_t st) {
   const int d = h->cfg.head_dim;
   if (dt == SWS_BF16) {
     const auto* pq = static_cast<const __nv_bfloat16*>(q);
     const auto* pk = static_cast<const __nv_bfloat16*>(k);
-    return d == 128 ? launch_pool_project<__nv_bfloat16, 128>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st)
-                    : launch_pool_project<__nv_bfloat16, 64>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st);
+    return d == 128 ? launch_pool_project<__nv_bfloat16, 128>(h, pq, pk, n, hq, hkv, qs, ks, q_sk, k_sk, st)
+                    : launch_pool_project<__nv_bfloat16, 64>(h, pq, pk, n, hq, hkv, qs, ks, q_sk, k_sk, st);
   }
   const auto* pq = static_cast<const float*>(q);
   const auto* pk = static_cast<const float*>(k);
-  return d == 128 ? launch_pool_project<float, 128>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st)
-                  : launch_pool_project<float, 64>(h, pq, pk, n, hq, hkv, q_sk, k_sk, st);
+  return d == 128 ? launch_pool_project<float, 128>(h, pq, pk, n, hq, hkv, qs, ks, q_sk, k_sk, st)
+                  : launch_pool_project<float, 64>(h, pq, pk, n, hq, hkv, qs, ks, q_sk, k_sk, st);
 }
 
 cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,

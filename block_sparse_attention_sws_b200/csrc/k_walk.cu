@@ -86,6 +86,137 @@ __global__ void __launch_bounds__(256) block_softmax_wide_kernel(const double* _
   for (int64_t j = lane; j < b; j += 32) a[j] = (j <= i) ? exp(temp * s[j] - mx) * inv : 0.0;
 }
 
+// The same row softmax without the sketched scores in memory: each CTA of two
+// warps takes one 32-row tile of one head and forms its scores
+// S_ij = q~_i . k~_j / sqrt(k), j <= i, itself, 32 key blocks at a time, on the
+// fp64 tensor path (mma.sync m16n8k4 f64), from q~ and k~ staged in shared
+// memory. Two passes over the row tile's key tiles: the first keeps each row's
+// running maximum and sum of exponentials, the second forms the tile's scores
+// again and writes exp(temp S - max) / sum. The scores come out of the same
+// products in the same order as in scores_kernel, so they are bit for bit the
+// ones sws_sketch writes; only the order of the row sum differs from
+// block_softmax_kernel. Row tiles run longest first. Entries above the
+// diagonal are not written (every reader masks them).
+constexpr int kFT = 32;  // rows and key blocks per tile
+
+__device__ __forceinline__ void cp_async8_w(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 8 : 0)
+               : "memory");
+}
+
+// rows r0.. r0 + 31 of a [rows, k] fp64 matrix into a [32][ld] shared tile,
+// zero-filled past `rows` and past k up to kpad
+__device__ __forceinline__ void stage_tile(double* dst, const double* src, int64_t r0, int64_t rows, int32_t k,
+                                           int32_t kpad, int ld, int tid, int nthr) {
+  for (int e = tid; e < kFT * kpad; e += nthr) {
+    const int r = e / kpad, c = e % kpad;
+    const bool ok = r0 + r < rows && c < k;
+    cp_async8_w(dst + r * ld + c, ok ? src + (r0 + r) * k + c : src, ok);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void dmma_16x8x4_f(double (&c)[4], double a0, double a1, double b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a0), "d"(a1), "d"(b0));
+}
+
+__global__ void __launch_bounds__(64) sketch_softmax_kernel(const double* __restrict__ q_sk,
+                                                            const double* __restrict__ k_sk, int64_t b, int32_t hq,
+                                                            int32_t group, int32_t k, int32_t kpad,
+                                                            double inv_sqrt_k, double temp, double* __restrict__ A) {
+  grid_dependency_wait();
+  allow_dependents();
+  extern __shared__ __align__(16) double fsm[];
+  const int ld = kpad + 4;  // kpad % 32 == 0: fragment loads take the minimum two wavefronts
+  double* qs = fsm;                   // [32][ld]
+  double* ks0 = fsm + kFT * ld;       // [2][32][ld]
+  const int64_t nt = ceil_div64(b, kFT);
+  const int64_t ti = nt - 1 - static_cast<int64_t>(blockIdx.x) / hq;  // longest rows first
+  const int h = static_cast<int>(blockIdx.x % hq);
+  const double* qh = q_sk + (size_t)h * b * k;
+  const double* kh = k_sk + (size_t)(h / group) * b * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int64_t i0 = ti * kFT;
+  stage_tile(qs, qh, i0, b, k, kpad, ld, tid, 64);
+  // this lane's two rows: i0 + 16 warp + g + 8 hh
+  double m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0, 0.0};
+  for (int pass = 0; pass < 2; ++pass) {
+    stage_tile(ks0, kh, 0, b, k, kpad, ld, tid, 64);
+    for (int64_t tj = 0; tj <= ti; ++tj) {
+      double* ks = ks0 + (tj & 1) * kFT * ld;
+      if (tj < ti) {
+        stage_tile(ks0 + ((tj + 1) & 1) * kFT * ld, kh, (tj + 1) * kFT, b, k, kpad, ld, tid, 64);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      __syncthreads();
+      double acc[4][4];
+#pragma unroll
+      for (int n8 = 0; n8 < 4; ++n8)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[n8][v] = 0.0;
+      for (int kk = 0; kk < kpad / 4; ++kk) {
+        const double a0 = qs[(warp * 16 + g) * ld + kk * 4 + t4];
+        const double a1 = qs[(warp * 16 + g + 8) * ld + kk * 4 + t4];
+#pragma unroll
+        for (int n8 = 0; n8 < 4; ++n8) dmma_16x8x4_f(acc[n8], a0, a1, ks[(n8 * 8 + g) * ld + kk * 4 + t4]);
+      }
+      const int64_t j0 = tj * kFT;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int64_t i = i0 + warp * 16 + g + 8 * hh;
+        double x[8];
+#pragma unroll
+        for (int n8 = 0; n8 < 4; ++n8)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int64_t j = j0 + n8 * 8 + 2 * t4 + e;
+            x[2 * n8 + e] = (i < b && j <= i) ? temp * (acc[n8][2 * hh + e] * inv_sqrt_k) : -INFINITY;
+          }
+        if (pass == 0) {
+          double tm = x[0];
+#pragma unroll
+          for (int u = 1; u < 8; ++u) tm = fmax(tm, x[u]);
+          tm = fmax(tm, __shfl_xor_sync(0xffffffffu, tm, 1));
+          tm = fmax(tm, __shfl_xor_sync(0xffffffffu, tm, 2));
+          const double mn = fmax(m[hh], tm);
+          double sum = 0.0;
+          if (mn != -INFINITY) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += exp(x[u] - mn);  // exp(-inf) = 0 for masked entries
+          }
+          sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+          sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+          if (mn != -INFINITY) {
+            l[hh] = l[hh] * exp(m[hh] - mn) + sum;  // exp(-inf) = 0 while nothing was seen
+            m[hh] = mn;
+          }
+        } else if (i < b) {
+          const double inv = 1.0 / l[hh];
+          double* arow = A + ((size_t)h * b + i) * b;
+#pragma unroll
+          for (int n8 = 0; n8 < 4; ++n8) {
+            const int64_t j = j0 + n8 * 8 + 2 * t4;
+            const double v0 = exp(x[2 * n8] - m[hh]) * inv, v1 = exp(x[2 * n8 + 1] - m[hh]) * inv;
+            if ((b & 1) == 0 && j + 1 <= i) {
+              *reinterpret_cast<double2*>(arow + j) = make_double2(v0, v1);
+            } else {
+              if (j <= i) arow[j] = v0;
+              if (j + 1 <= i) arow[j + 1] = v1;
+            }
+          }
+        }
+      }
+      __syncthreads();  // every warp is done with this key tile before it is refilled
+    }
+  }
+}
+
 // C = A * Bm for lower-triangular b x b matrices on the fp64 tensor path
 // (mma.sync m16n8k4 f64). On this part each SM sub-partition completes one
 // such product about every 32 cycles, and one warp with one accumulator chain
@@ -415,6 +546,25 @@ cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int6
                                           : block_softmax_wide_kernel;
   {
     const cudaError_t le = launch_k(kern, grid, 256, 0, st, scores, b, rows, temp, A);
+    if (le != cudaSuccess) return le;
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sketch_softmax(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,
+                                  int32_t hkv, double* A, cudaStream_t st) {
+  const int32_t k = h->cfg.sketch_dim;
+  const int32_t kpad = static_cast<int32_t>(ceil_div64(k, 32) * 32);
+  const double temp = h->cfg.walk_mode == SWS_WALK_ELEMENTWISE ? (double)h->cfg.walk_power : 1.0;
+  const int64_t nt = ceil_div64(b, kFT);
+  const size_t smem = 3 * kFT * (kpad + 4) * sizeof(double);
+  const cudaError_t ea =
+      cudaFuncSetAttribute(sketch_softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (ea != cudaSuccess) return ea;
+  {
+    const cudaError_t le = launch_k(sketch_softmax_kernel, static_cast<unsigned>(nt * hq), 64, smem, st, q_sk, k_sk, b,
+                                    hq, hq / hkv, k, kpad, 1.0 / sqrt((double)k), temp, A);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);

@@ -309,37 +309,66 @@ sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code) {
   return v ? SWS_ERR_DEVICE_CHECK : SWS_OK;
 }
 
+extern "C++" {
+namespace {
+
+// The element strides of a [heads, n, d] operand (NULL: dense). Rows keep their
+// d elements contiguous; both strides must move by whole rows (at least d) and by
+// multiples of 16 bytes, so that every row starts 16-byte aligned.
+bool head_tok(const int64_t* strides, int64_t n, int32_t d, size_t elem, HeadTok* out) {
+  if (!strides) {
+    *out = HeadTok{n * d, d};
+    return true;
+  }
+  const int64_t hs = strides[0], ts = strides[1];
+  if (hs < d || ts < d) return false;
+  if ((hs * static_cast<int64_t>(elem)) % 16 != 0 || (ts * static_cast<int64_t>(elem)) % 16 != 0) return false;
+  *out = HeadTok{hs, ts};
+  return true;
+}
+
+}  // namespace
+}  // extern "C++"
+
+sws_status sws_layout_check(const sws_config* cfg, sws_dtype dtype, int64_t n, const int64_t strides[2]) {
+  if (sws_config_check(cfg) != SWS_OK || n < 1 || (dtype != SWS_BF16 && dtype != SWS_FP32))
+    return SWS_ERR_INVALID_ARG;
+  HeadTok ht{};
+  return head_tok(strides, n, cfg->head_dim, dtype == SWS_BF16 ? 2 : 4, &ht) ? SWS_OK : SWS_ERR_INVALID_ARG;
+}
+
 sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n, int32_t hq,
-                      int32_t hkv, double* q_sk, double* k_sk, double* scores, void* ws, size_t ws_bytes,
-                      void* stream) {
+                      int32_t hkv, const int64_t q_strides[2], const int64_t k_strides[2], double* q_sk,
+                      double* k_sk, double* scores, void* ws, size_t ws_bytes, void* stream) {
   if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (dtype != SWS_BF16 && dtype != SWS_FP32) return SWS_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sk) || !aligned16(k_sk) || !aligned16(scores) ||
-      !aligned16(ws))
+  const size_t elem = dtype == SWS_BF16 ? 2 : 4;
+  HeadTok qs{}, ks{};
+  if (!head_tok(q_strides, n, h->cfg.head_dim, elem, &qs) || !head_tok(k_strides, n, h->cfg.head_dim, elem, &ks))
+    return SWS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_sk) || !aligned16(k_sk) || (scores && !aligned16(scores)) ||
+      (ws && !aligned16(ws)))
     return SWS_ERR_INVALID_ARG;
   const int64_t b = ceil_div64(n, h->cfg.block_size);
   if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
   if (ws_bytes < sketch_workspace_bytes(h->cfg, n, hq, hkv)) return SWS_ERR_WORKSPACE;
   auto st = static_cast<cudaStream_t>(stream);
   sws_status s = cuda_status(
-      launch_sketch_pool_project(h, q, k, dtype, n, hq, hkv, q_sk, k_sk, st), "sketch pool+project");
-  if (s != SWS_OK) return s;
+      launch_sketch_pool_project(h, q, k, dtype, n, hq, hkv, qs, ks, q_sk, k_sk, st), "sketch pool+project");
+  if (s != SWS_OK || !scores) return s;
   return cuda_status(launch_sketch_scores(h, q_sk, k_sk, b, hq, hkv, scores, st), "sketch scores");
 }
 
-sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n, int32_t hq, int first_layer,
-                           double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
-                           void* stream) {
-  if (!h || n < 1 || check_heads(hq, 1) != SWS_OK) return SWS_ERR_INVALID_ARG;
-  if (h->cfg.select_group > 1 && hq % h->cfg.select_group != 0) return SWS_ERR_INVALID_ARG;
-  if (!aligned16(scores) || !aligned16(walk_state) || !aligned16(row_ptr) || !aligned16(col_idx) || !aligned16(ws))
-    return SWS_ERR_INVALID_ARG;
-  const int64_t b = ceil_div64(n, h->cfg.block_size);
-  if (b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
-  size_t need = 0;
-  if (sws_workspace_size(&h->cfg, SWS_OP_WALK_SELECT, n, hq, 1, 1, &need) != SWS_OK) return SWS_ERR_INVALID_ARG;
-  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
-  auto st = static_cast<cudaStream_t>(stream);
+extern "C++" {
+namespace {
+
+// The walk and the selection after the block attention matrix: M = A^s by
+// binary powering (matrix power) or M = A (the entrywise power is folded into
+// the softmax's temperature), R = M or R_prev M, then top-tau. `softmax`
+// writes A into the buffer it is given.
+template <typename Softmax>
+sws_status walk_chain(const sws_handle* h, int64_t b, int32_t hq, int first_layer, double* walk_state,
+                      int32_t* row_ptr, int32_t* col_idx, void* ws, cudaStream_t st, Softmax softmax) {
   const size_t mat = static_cast<size_t>(hq) * b * b;
   double* buf[4] = {static_cast<double*>(ws), static_cast<double*>(ws) + mat, static_cast<double*>(ws) + 2 * mat,
                     static_cast<double*>(ws) + 3 * mat};
@@ -356,7 +385,7 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
     return -1;
   };
   const int a = take();
-  sws_status s = cuda_status(launch_block_softmax(h, scores, b, hq, buf[a], st), "block softmax");
+  sws_status s = cuda_status(softmax(buf[a]), "block softmax");
   if (s != SWS_OK) return s;
   int m_idx = a;  // holds M = A^s when done
   if (h->cfg.walk_mode == SWS_WALK_MATRIX_POWER && h->cfg.walk_power > 1) {
@@ -399,21 +428,71 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
   return cuda_status(launch_select(h, Rnew, b, hq, walk_state, row_ptr, col_idx, st), "top-tau select");
 }
 
+// Checks shared by both walk-select entry points; b on success.
+sws_status walk_args(const sws_handle* h, int64_t n, int32_t hq, int32_t hkv, const double* walk_state,
+                     const int32_t* row_ptr, const int32_t* col_idx, const void* ws, size_t ws_bytes, int64_t* b) {
+  if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.select_group > 1 && hq % h->cfg.select_group != 0) return SWS_ERR_INVALID_ARG;
+  if (!aligned16(walk_state) || !aligned16(row_ptr) || !aligned16(col_idx) || !aligned16(ws))
+    return SWS_ERR_INVALID_ARG;
+  *b = ceil_div64(n, h->cfg.block_size);
+  if (*b > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
+  size_t need = 0;
+  if (sws_workspace_size(&h->cfg, SWS_OP_WALK_SELECT, n, hq, hkv, 1, &need) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (ws_bytes < need) return SWS_ERR_WORKSPACE;
+  return SWS_OK;
+}
+
+}  // namespace
+}  // extern "C++"
+
+sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n, int32_t hq, int first_layer,
+                           double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
+                           void* stream) {
+  int64_t b = 0;
+  const sws_status v = walk_args(h, n, hq, 1, walk_state, row_ptr, col_idx, ws, ws_bytes, &b);
+  if (v != SWS_OK) return v;
+  if (!aligned16(scores)) return SWS_ERR_INVALID_ARG;
+  auto st = static_cast<cudaStream_t>(stream);
+  return walk_chain(h, b, hq, first_layer, walk_state, row_ptr, col_idx, ws, st,
+                    [&](double* A) { return launch_block_softmax(h, scores, b, hq, A, st); });
+}
+
+sws_status sws_walk_select_sketch(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t n, int32_t hq,
+                                  int32_t hkv, int first_layer, double* walk_state, int32_t* row_ptr,
+                                  int32_t* col_idx, void* ws, size_t ws_bytes, void* stream) {
+  int64_t b = 0;
+  const sws_status v = walk_args(h, n, hq, hkv, walk_state, row_ptr, col_idx, ws, ws_bytes, &b);
+  if (v != SWS_OK) return v;
+  if (!aligned16(q_sk) || !aligned16(k_sk)) return SWS_ERR_INVALID_ARG;
+  auto st = static_cast<cudaStream_t>(stream);
+  return walk_chain(h, b, hq, first_layer, walk_state, row_ptr, col_idx, ws, st,
+                    [&](double* A) { return launch_sketch_softmax(h, q_sk, k_sk, b, hq, hkv, A, st); });
+}
+
 sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const void* k, const void* v,
-                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
-                                   const int32_t* col_idx, void* o, void* ws, size_t ws_bytes, void* stream) {
+                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int64_t q_strides[2],
+                                   const int64_t k_strides[2], const int64_t v_strides[2],
+                                   const int64_t o_strides[2], const int32_t* row_ptr, const int32_t* col_idx,
+                                   void* o, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;
   (void)ws_bytes;
   if (!h || n < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
   if (dtype != SWS_BF16 && dtype != SWS_FP32) return SWS_ERR_INVALID_ARG;
+  const size_t elem = dtype == SWS_BF16 ? 2 : 4;
+  const int32_t d = h->cfg.head_dim;
+  PrefillLayout lay{};
+  if (!head_tok(q_strides, n, d, elem, &lay.q) || !head_tok(k_strides, n, d, elem, &lay.k) ||
+      !head_tok(v_strides, n, d, elem, &lay.v) || !head_tok(o_strides, n, d, elem, &lay.o))
+    return SWS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(row_ptr) || !aligned16(col_idx))
     return SWS_ERR_INVALID_ARG;
   if (ceil_div64(n, h->cfg.block_size) > kMaxPrefillBlocks) return SWS_ERR_UNSUPPORTED;
   auto st = static_cast<cudaStream_t>(stream);
   if (dtype == SWS_BF16)
-    return cuda_status(launch_attn_prefill_tc(h, q, k, v, n, hq, hkv, row_ptr, col_idx, o, st),
+    return cuda_status(launch_attn_prefill_tc(h, q, k, v, n, hq, hkv, lay, row_ptr, col_idx, o, st),
                        "prefill attention (tensor cores)");
-  return cuda_status(launch_attn_prefill_simt(h, q, k, v, dtype, n, hq, hkv, row_ptr, col_idx, o, st),
+  return cuda_status(launch_attn_prefill_simt(h, q, k, v, dtype, n, hq, hkv, lay, row_ptr, col_idx, o, st),
                      "prefill attention (fp32)");
 }
 
@@ -469,6 +548,47 @@ sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const v
                           q_psum, q_sketch, first_layer, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt,
                           static_cast<cudaStream_t>(stream)),
       "decode step (exact walk)");
+}
+
+int64_t sws_decode_exact_rows_entries(const sws_config* cfg, int64_t max_len) {
+  if (sws_config_check(cfg) != SWS_OK || max_len < 1) return -1;
+  return exact_rows_entries(ceil_div64(max_len, cfg->block_size));
+}
+
+sws_status sws_decode_exact_rows_init(const sws_handle* h, const double* q_sketch, const double* k_sketch,
+                                      int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                      const int32_t* seq_lens, uint32_t* rows, void* stream) {
+  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_sketch, k_sketch, seq_lens, rows};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  if (!exact_wide_supported(h->cfg, ceil_div64(max_len, h->cfg.block_size), hq / hkv)) return SWS_ERR_UNSUPPORTED;
+  return cuda_status(launch_exact_rows_init(h, q_sketch, k_sketch, batch, hq, hkv, max_len, seq_lens, rows,
+                                            static_cast<cudaStream_t>(stream)),
+                     "exact walk rows");
+}
+
+sws_status sws_decode_step_exact_rows(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                      int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                      const int32_t* seq_lens, void* k_cache, void* v_cache, double* k_psum,
+                                      double* k_sketch, double* q_psum, double* q_sketch, uint32_t* rows,
+                                      int first_layer, double* walk_state, int32_t* head_sel, int32_t* head_cnt,
+                                      int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream) {
+  if (!h || batch < 1 || max_len < 1 || check_heads(hq, hkv) != SWS_OK) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.select_group > 1 && h->cfg.select_group != hq / hkv) return SWS_ERR_INVALID_ARG;
+  if (h->cfg.walk_mode != SWS_WALK_MATRIX_POWER) return SWS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_tok, k_tok, v_tok, seq_lens, k_cache, v_cache, k_psum, k_sketch, q_psum, q_sketch,
+                        rows, walk_state, head_sel, head_cnt, sel, sel_mask, sel_cnt};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWS_ERR_INVALID_ARG;
+  if (!exact_wide_supported(h->cfg, ceil_div64(max_len, h->cfg.block_size), hq / hkv)) return SWS_ERR_UNSUPPORTED;
+  return cuda_status(
+      launch_decode_exact_wide(h, static_cast<const __nv_bfloat16*>(q_tok), static_cast<const __nv_bfloat16*>(k_tok),
+                               static_cast<const __nv_bfloat16*>(v_tok), batch, hq, hkv, max_len, seq_lens,
+                               static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), k_psum,
+                               k_sketch, q_psum, q_sketch, rows, first_layer, walk_state, head_sel, head_cnt, sel,
+                               sel_mask, sel_cnt, static_cast<cudaStream_t>(stream)),
+      "decode step (exact walk, stored rows)");
 }
 
 sws_status sws_decode_step_paged(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,

@@ -175,25 +175,38 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
 }
 
+// Element strides of a [heads, tokens, d] operand whose rows of d elements are
+// contiguous: row t of head h starts at base + h * head + t * tok.
+struct HeadTok {
+  int64_t head, tok;
+};
+// The four operands of prefill attention.
+struct PrefillLayout {
+  HeadTok q, k, v, o;
+};
+
 size_t sketch_workspace_bytes(const sws_config& c, int64_t n, int32_t hq, int32_t hkv);
 cudaError_t launch_sketch_pool_project(const sws_handle* h, const void* q, const void* k, sws_dtype dt, int64_t n,
-                                       int32_t hq, int32_t hkv, double* q_sk, double* k_sk, cudaStream_t st);
+                                       int32_t hq, int32_t hkv, HeadTok qs, HeadTok ks, double* q_sk, double* k_sk,
+                                       cudaStream_t st);
 cudaError_t launch_sketch_scores(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,
                                  int32_t hkv, double* scores, cudaStream_t st);
 
 cudaError_t launch_block_softmax(const sws_handle* h, const double* scores, int64_t b, int32_t hq, double* A,
                                  cudaStream_t st);
+cudaError_t launch_sketch_softmax(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t b, int32_t hq,
+                                  int32_t hkv, double* A, cudaStream_t st);
 cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st);
 cudaError_t launch_select(const sws_handle* h, const double* R, int64_t b, int32_t hq, double* walk_state,
                           int32_t* row_ptr, int32_t* col_idx, cudaStream_t st);
 
 cudaError_t launch_attn_prefill_simt(const sws_handle* h, const void* q, const void* k, const void* v, sws_dtype dt,
-                                     int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
-                                     const int32_t* col_idx, void* o, cudaStream_t st);
+                                     int64_t n, int32_t hq, int32_t hkv, const PrefillLayout& lay,
+                                     const int32_t* row_ptr, const int32_t* col_idx, void* o, cudaStream_t st);
 
 cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
-                                   int32_t hq, int32_t hkv, const int32_t* row_ptr, const int32_t* col_idx, void* o,
-                                   cudaStream_t st);
+                                   int32_t hq, int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr,
+                                   const int32_t* col_idx, void* o, cudaStream_t st);
 
 // Where the cached keys (or values) of one (sequence, KV head) live.
 //  contiguous (block_table null): [batch, hkv, max_len, D]; token t of the unit
@@ -243,6 +256,18 @@ cudaError_t launch_decode_exact(const sws_handle* h, const __nv_bfloat16* q_tok,
                                 double* k_psum, double* k_sketch, double* q_psum, double* q_sketch, int first_layer,
                                 double* walk_state, int32_t* head_sel, int32_t* head_cnt, int32_t* sel,
                                 uint8_t* sel_mask, int32_t* sel_cnt, cudaStream_t st);
+int64_t exact_rows_entries(int64_t max_blocks);
+bool exact_wide_supported(const sws_config& c, int64_t max_blocks, int32_t group);
+cudaError_t launch_exact_rows_init(const sws_handle* h, const double* q_sketch, const double* k_sketch, int32_t batch,
+                                   int32_t hq, int32_t hkv, int64_t max_len, const int32_t* seq_lens, uint32_t* rows,
+                                   cudaStream_t st);
+cudaError_t launch_decode_exact_wide(const sws_handle* h, const __nv_bfloat16* q_tok, const __nv_bfloat16* k_tok,
+                                     const __nv_bfloat16* v_tok, int32_t batch, int32_t hq, int32_t hkv,
+                                     int64_t max_len, const int32_t* seq_lens, __nv_bfloat16* k_cache,
+                                     __nv_bfloat16* v_cache, double* k_psum, double* k_sketch, double* q_psum,
+                                     double* q_sketch, uint32_t* rows, int first_layer, double* walk_state,
+                                     int32_t* head_sel, int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask,
+                                     int32_t* sel_cnt, cudaStream_t st);
 size_t decode_exact_smem_bytes(const sws_config& cfg, int64_t max_blocks, int32_t group);
 bool decode_exact_supported(const sws_config& cfg, int64_t max_blocks, int32_t group);
 int32_t decode_num_splits(const sws_config& cfg, int64_t max_len, int32_t group);

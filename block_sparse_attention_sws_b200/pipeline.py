@@ -18,12 +18,18 @@ class PrefillPath:
     ``dense_layers`` is the caller policy of "Scout Before You Attend" §7 (the
     first layers attend densely): layers below it select every causal block,
     through a second handle with density 1/1 and the same projection, while
-    the walk state still runs through them."""
+    the walk state still runs through them.
+
+    ``scores_in_memory`` = False (the default) skips the [hq, b, b] score
+    matrix: sws_sketch writes only the sketches and sws_walk_select_sketch
+    forms the scores on chip. True keeps the score matrix (``self.scores``)
+    and calls sws_walk_select on it."""
 
     def __init__(self, handle: L.Handle, n: int, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda",
-                 dense_layers: int = 0):
+                 dense_layers: int = 0, scores_in_memory: bool = False):
         cfg = handle.cfg
         self.dense_layers = dense_layers
+        self.scores_in_memory = scores_in_memory
         self.h, self.n, self.hq, self.hkv = handle, n, hq, hkv
         self.b = L.sws_num_blocks(cfg, n)
         self.nnz = L.sws_csr_nnz(cfg, n)
@@ -31,7 +37,7 @@ class PrefillPath:
         f64 = dict(dtype=torch.float64, device=device)
         self.q_sk = torch.empty(hq, self.b, k, **f64)
         self.k_sk = torch.empty(hkv, self.b, k, **f64)
-        self.scores = torch.empty(hq, self.b, self.b, **f64)
+        self.scores = torch.empty(hq, self.b, self.b, **f64) if scores_in_memory else None
         self.walk_state = torch.zeros(hq, self.b, self.b, **f64)
         self.row_ptr = torch.empty(hq, self.b + 1, dtype=torch.int32, device=device)
         self.col_idx = torch.empty(hq, self.nnz, dtype=torch.int32, device=device)
@@ -63,7 +69,11 @@ class PrefillPath:
     def walk_select(self, first_layer: bool, stream=None, layer=None):
         h = self.h_dense if self._dense(layer) else self.h
         rp, ci = self.csr(layer)
-        L.sws_walk_select(h, self.scores, self.n, first_layer, self.walk_state, rp, ci, self.ws, stream)
+        if self.scores_in_memory:
+            L.sws_walk_select(h, self.scores, self.n, first_layer, self.walk_state, rp, ci, self.ws, stream)
+        else:
+            L.sws_walk_select_sketch(h, self.q_sk, self.k_sk, self.n, first_layer, self.walk_state, rp, ci, self.ws,
+                                     stream)
 
     def attention(self, q, k, v, out=None, stream=None, layer=None):
         o = self.o if out is None else out
@@ -117,6 +127,10 @@ class DecodePath:
     exact=True selects with the exact decode walk (sws_decode_step_exact): the
     row of the new token's block in the prefill recurrence, which needs the
     prompt's query sketches (init_queries) next to the key sketches.
+    exact="rows" is the same walk for contexts of any length: each layer's
+    block attention rows are kept in device memory (init_rows builds them once
+    the key and query sketches are in place) and the steps call
+    sws_decode_step_exact_rows.
 
     paged=True keeps each layer's keys and values in a pool of pages
     [num_pages, hkv, B, d] addressed through block_table [batch, max_blocks]
@@ -151,6 +165,10 @@ class DecodePath:
             assert not paged, "the exact walk runs on the contiguous cache"
             self.q_psum = [torch.zeros(batch, hq, d, **f64) for _ in range(layers)]
             self.q_sketch = [torch.zeros(batch, hq, self.mb, k, **f64) for _ in range(layers)]
+        self.rows = None
+        if exact == "rows":
+            e = L.sws_decode_exact_rows_entries(cfg, max_len)
+            self.rows = [torch.zeros(batch, hq, e, dtype=torch.int32, device=device) for _ in range(layers)]
         self.seq_lens = torch.zeros(batch, **i32)
         self.walk_state = torch.zeros(batch, hq, self.mb, **f64)
         self.head_sel = torch.zeros(batch, hq, self.mb, **i32)
@@ -219,11 +237,28 @@ class DecodePath:
         assert self.exact and tuple(q_prompt.shape[:3]) == (self.batch, self.hq, self.max_len)
         L.sws_decode_init_cache(self.h, q_prompt, self.seq_lens, self.q_psum[layer], self.q_sketch[layer], stream)
 
+    def init_rows(self, stream=None):
+        """Exact walk with stored rows: every layer's block attention rows from
+        the key sketches (init_cache) and query sketches (init_queries)."""
+        assert self.rows is not None
+        for layer in range(self.layers):
+            L.sws_decode_exact_rows_init(self.h, self.q_sketch[layer], self.k_sketch[layer], self.seq_lens,
+                                         self.rows[layer], stream)
+
     def begin_step(self, stream=None):
         L.sws_decode_advance(self.h, self.seq_lens, stream)
 
     def layer(self, layer: int, q_tok, k_tok, v_tok, out=None, stream=None):
         o = self.o if out is None else out
+        if self.exact == "rows":
+            L.sws_decode_step_exact_rows(self.h, q_tok, k_tok, v_tok, self.seq_lens, self.k_cache[layer],
+                                         self.v_cache[layer], self.k_psum[layer], self.k_sketch[layer],
+                                         self.q_psum[layer], self.q_sketch[layer], self.rows[layer], layer == 0,
+                                         self.walk_state, self.head_sel, self.head_cnt, self.sel, self.sel_mask,
+                                         self.sel_cnt, stream)
+            L.sws_sparse_attn_decode(self.h, q_tok, self.k_cache[layer], self.v_cache[layer], self.seq_lens,
+                                     self.sel, self.sel_mask, self.sel_cnt, o, self.ws, stream)
+            return o
         if self.exact:
             L.sws_decode_step_exact(self.h, q_tok, k_tok, v_tok, self.seq_lens, self.k_cache[layer],
                                     self.v_cache[layer], self.k_psum[layer], self.k_sketch[layer], self.q_psum[layer],

@@ -11,7 +11,8 @@
  *    allocates device memory only in sws_create (the projection matrix) and never in
  *    a compute call.
  *  - Every device pointer must be 16-byte aligned; tensors are dense, row-major,
- *    with the layouts stated per call (no strides).
+ *    with the layouts stated per call, except the per-head activations of the
+ *    prefill calls, which take strides (see "Strided operands" below).
  *  - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and return after the launches were queued. A call that fails its host-side
  *    validation returns a status and queues nothing. Launch failures return SWS_ERR_CUDA.
@@ -123,21 +124,36 @@ uint64_t sws_launch_count(void);
 sws_status sws_sync_check(const sws_handle* h, void* stream, int32_t* code);
 
 /* ---------------------------------------------------------------- prefill --- */
+/* Strided operands. Q, K, V and O of the prefill calls are [heads, n, d] with the
+ * d elements of each row contiguous; `x_strides` (host, two int64) gives the
+ * element distance from one head to the next (x_strides[0]) and from one token to
+ * the next (x_strides[1]), so row t of head h starts at x + h*x_strides[0] +
+ * t*x_strides[1]. NULL means dense: {n*d, d}. A model's [n, heads, d] activations
+ * are read in place with {d, heads*d}. Each stride must be at least d and a
+ * multiple of 16 bytes (SWS_ERR_INVALID_ARG otherwise); every row addressed must
+ * lie in the caller's allocation, and no two rows of O may overlap. */
+
+/* Host only: SWS_OK when `strides` (NULL = dense) is valid for an operand of n
+ * tokens of `dtype` under cfg (the check every prefill call makes), else
+ * SWS_ERR_INVALID_ARG. */
+sws_status sws_layout_check(const sws_config* cfg, sws_dtype dtype, int64_t n, const int64_t strides[2]);
 
 /* sws_sketch. §3.1 block means (a partial last block divides by its row count),
  * §3.2 projection q~_i = q_bar_i H_d, k~_j = k_bar_j H_d and the sketched block scores
  * S[h,i,j] = q~_i(h) . k~_j(h/(hq/hkv)) / sqrt(k) for j <= i (causal block mask).
- *   q      (device) [hq, n, d]   dtype
- *   k      (device) [hkv, n, d]  dtype
+ *   q      (device) [hq, n, d]   dtype, strides q_strides (NULL: dense)
+ *   k      (device) [hkv, n, d]  dtype, strides k_strides (NULL: dense)
  *   q_sk   (device) [hq, b, k]   double, written
  *   k_sk   (device) [hkv, b, k]  double, written
- *   scores (device) [hq, b, b]   double; entries j <= i written, j > i left untouched
+ *   scores (device) [hq, b, b]   double; entries j <= i written, j > i left untouched.
+ *          May be NULL: then the scores are not formed here and the caller goes on
+ *          with sws_walk_select_sketch, which forms them on chip from q_sk and k_sk.
  *   ws     (device) sws_workspace_size(SWS_OP_SKETCH) bytes, currently 0: the block
  *          means stay on chip (may be NULL while the size is 0)
  * Reads Q and K once: one fused pass forms the block means and projects them. */
 sws_status sws_sketch(const sws_handle* h, const void* q, const void* k, sws_dtype dtype, int64_t n,
-                      int32_t hq, int32_t hkv, double* q_sk, double* k_sk, double* scores, void* ws,
-                      size_t ws_bytes, void* stream);
+                      int32_t hq, int32_t hkv, const int64_t q_strides[2], const int64_t k_strides[2],
+                      double* q_sk, double* k_sk, double* scores, void* ws, size_t ws_bytes, void* stream);
 
 /* sws_walk_select. §4: A = row softmax of scores over j <= i (the sketched block
  * attention matrix), M = A^s, R = M on the first layer, else R = R_prev * M; then for
@@ -154,16 +170,34 @@ sws_status sws_walk_select(const sws_handle* h, const double* scores, int64_t n,
                            double* walk_state, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* sws_walk_select_sketch. The same walk and selection as sws_walk_select, from the
+ * sketches instead of the score matrix: the sketched block scores of §3.2,
+ * S[h,i,j] = q~_i(h) . k~_j(h/(hq/hkv)) / sqrt(k), are formed tile by tile on chip
+ * (on the fp64 tensor path, the same products in the same order as sws_sketch
+ * uses, so the same values) and go straight into the row softmax; the [hq, b, b]
+ * score matrix never reaches device memory.
+ *   q_sk (device) [hq, b, k] double, k_sk (device) [hkv, b, k] double: as
+ *        sws_sketch wrote them
+ *   walk_state, row_ptr, col_idx, ws: as sws_walk_select (same workspace size)
+ * The row sums of the softmax are accumulated in another order than in
+ * sws_walk_select, so the two calls agree to rounding (about 1e-15 relative). */
+sws_status sws_walk_select_sketch(const sws_handle* h, const double* q_sk, const double* k_sk, int64_t n,
+                                  int32_t hq, int32_t hkv, int first_layer, double* walk_state, int32_t* row_ptr,
+                                  int32_t* col_idx, void* ws, size_t ws_bytes, void* stream);
+
 /* sws_sparse_attn_prefill. §4/§5: exact softmax attention on the original Q, K, V
  * restricted to the selected key blocks; query token t attends to the tokens u of the
  * blocks listed for its block with u <= t. Online softmax, fp32 accumulation.
- *   q (device) [hq, n, d], k, v (device) [hkv, n, d], o (device) [hq, n, d]: all dtype
+ *   q (device) [hq, n, d], k, v (device) [hkv, n, d], o (device) [hq, n, d]: all dtype,
+ *     each with its strides (NULL: dense)
  *   row_ptr, col_idx: the CSR of sws_walk_select (each row ascending, within [0, i])
  * bf16 runs on the tensor cores (fp32 accumulate, output rounded to nearest);
  * fp32 runs in fp32 FMA. */
 sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const void* k, const void* v,
-                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int32_t* row_ptr,
-                                   const int32_t* col_idx, void* o, void* ws, size_t ws_bytes, void* stream);
+                                   sws_dtype dtype, int64_t n, int32_t hq, int32_t hkv, const int64_t q_strides[2],
+                                   const int64_t k_strides[2], const int64_t v_strides[2],
+                                   const int64_t o_strides[2], const int32_t* row_ptr, const int32_t* col_idx,
+                                   void* o, void* ws, size_t ws_bytes, void* stream);
 
 /* ----------------------------------------------------------------- decode --- */
 /* §5: each decode step scores its single new query token against the cached key
@@ -230,6 +264,38 @@ sws_status sws_decode_step_exact(const sws_handle* h, const void* q_tok, const v
                                  void* k_cache, void* v_cache, double* k_psum, double* k_sketch, double* q_psum,
                                  double* q_sketch, int first_layer, double* walk_state, int32_t* head_sel,
                                  int32_t* head_cnt, int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
+
+/* The exact decode walk above for contexts of any length (up to 2560 blocks: a
+ * 163,840-token context at B = 64), with the rows of each layer's block attention
+ * kept in device memory between steps. Row m of A^l (the causal row softmax of
+ * q~_m . k~_j / sqrt(k), j <= m) no longer changes once block m is complete, so a
+ * step writes only the newest block's row, and the s products read the stored
+ * rows once per eight levels of s (a sweep from the newest block up to block 0).
+ * The selection equals that of sws_decode_step_exact on the same state up to
+ * rounding (the rows are formed by the same operations; the products add in
+ * another order).
+ *   rows (device) per layer: [batch, hq, E] uint32 with E = sws_decode_exact_rows_entries
+ *        entries per (sequence, query head): row m holds columns 0..m, padded with
+ *        zeros to a multiple of 4 entries, at entry offset 4(q+1)(2q+r) with
+ *        q = m div 4, r = m mod 4; each entry is the high 32 bits of the fp64
+ *        value rounded to nearest (sign, exponent, 20 mantissa bits).
+ * Build them once, after sws_decode_init_cache has built the key and query
+ * sketches of the prompt, with sws_decode_exact_rows_init; each call of
+ * sws_decode_step_exact_rows then appends the token (as sws_decode_step_exact)
+ * and rewrites the newest row before the products. Other arguments as
+ * sws_decode_step_exact. Requires sketch_dim <= 32 and max_blocks <= 2560
+ * (SWS_ERR_UNSUPPORTED otherwise). Memory: 4 E bytes per (sequence, query head,
+ * layer), about 2 max_blocks^2 bytes (8.4 MB at 2049 blocks). */
+int64_t sws_decode_exact_rows_entries(const sws_config* cfg, int64_t max_len);
+sws_status sws_decode_exact_rows_init(const sws_handle* h, const double* q_sketch, const double* k_sketch,
+                                      int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                      const int32_t* seq_lens, uint32_t* rows, void* stream);
+sws_status sws_decode_step_exact_rows(const sws_handle* h, const void* q_tok, const void* k_tok, const void* v_tok,
+                                      int32_t batch, int32_t hq, int32_t hkv, int64_t max_len,
+                                      const int32_t* seq_lens, void* k_cache, void* v_cache, double* k_psum,
+                                      double* k_sketch, double* q_psum, double* q_sketch, uint32_t* rows,
+                                      int first_layer, double* walk_state, int32_t* head_sel, int32_t* head_cnt,
+                                      int32_t* sel, uint8_t* sel_mask, int32_t* sel_cnt, void* stream);
 
 /* sws_sparse_attn_decode: one query token per (sequence, head) over the tokens
  * (< seq_lens[i]) of the blocks its head selected. Each KV block of the group's union is

@@ -110,10 +110,13 @@ def test_workspace_sizes(lib):
 def test_null_handle_rejected_without_launch(lib):
     """Host validation fails before any CUDA call, so this runs without a GPU."""
     P = ctypes.c_void_p
-    assert lib.sws_sketch(None, P(16), P(16), 0, 64, 1, 1, P(16), P(16), P(16), P(16), 16, None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_sketch(None, P(16), P(16), 0, 64, 1, 1, None, None, P(16), P(16), P(16), P(16), 16,
+                          None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_walk_select(None, P(16), 64, 1, 1, P(16), P(16), P(16), P(16), 16, None) == S.SWS_ERR_INVALID_ARG
-    assert lib.sws_sparse_attn_prefill(None, P(16), P(16), P(16), 0, 64, 1, 1, P(16), P(16), P(16), None, 0,
-                                       None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_walk_select_sketch(None, P(16), P(16), 64, 1, 1, 1, P(16), P(16), P(16), P(16), 16,
+                                      None) == S.SWS_ERR_INVALID_ARG
+    assert lib.sws_sparse_attn_prefill(None, P(16), P(16), P(16), 0, 64, 1, 1, None, None, None, None, P(16), P(16),
+                                       P(16), None, 0, None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_destroy(None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_projection_device(None) is None
     assert lib.sws_decode_init_cache_paged(None, P(16), 4, P(16), 4, 1, 1, P(16), P(16), P(16),
@@ -122,6 +125,25 @@ def test_null_handle_rejected_without_launch(lib):
                                      P(16), 1, P(16), P(16), P(16), P(16), P(16), P(16), None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_sparse_attn_decode_paged(None, P(16), P(16), P(16), 4, P(16), 4, 1, 4, 1, P(16), P(16), P(16),
                                             P(16), P(16), P(16), 1 << 20, None) == S.SWS_ERR_INVALID_ARG
+
+
+def test_stride_checks(lib):
+    """Strided prefill operands: each stride at least d elements and a multiple of
+    16 bytes; NULL is the dense layout."""
+    cfg = S.make_config(128, 64, 32)
+    ok = lambda dt, st: lib.sws_layout_check(ctypes.byref(cfg), dt, 1000,  # noqa: E731
+                                             None if st is None else (ctypes.c_int64 * 2)(*st))
+    assert ok(S.SWS_BF16, None) == S.SWS_OK
+    assert ok(S.SWS_BF16, (128, 32 * 128)) == S.SWS_OK  # [n, 32 heads, d] read in place
+    assert ok(S.SWS_BF16, (1000 * 128, 128)) == S.SWS_OK  # dense, spelled out
+    assert ok(S.SWS_FP32, (128, 8 * 128)) == S.SWS_OK
+    assert ok(S.SWS_BF16, (128, 32 * 128 + 4)) == S.SWS_ERR_INVALID_ARG  # 8 bytes past a 16-byte multiple
+    assert ok(S.SWS_BF16, (136, 8 * 128)) == S.SWS_OK  # 272 bytes: padded heads
+    assert ok(S.SWS_BF16, (132, 8 * 128)) == S.SWS_ERR_INVALID_ARG  # 264 bytes
+    assert ok(S.SWS_FP32, (128, 8 * 128 + 2)) == S.SWS_ERR_INVALID_ARG  # 8 bytes past
+    assert ok(S.SWS_BF16, (64, 32 * 128)) == S.SWS_ERR_INVALID_ARG  # heads overlap within a row
+    assert ok(S.SWS_BF16, (128, 120)) == S.SWS_ERR_INVALID_ARG  # tokens overlap
+    assert ok(S.SWS_BF16, (0, 128)) == S.SWS_ERR_INVALID_ARG
 
 
 def test_create_reports_error_without_gpu(lib):

@@ -28,15 +28,31 @@ from parity import compare_attention, compare_selection, record_ties
 pytestmark = pytest.mark.gpu
 
 
-def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None):
+class _Heads:
+    """[heads, n, d] device tensor seen by the oracle one head at a time (fp64 numpy)."""
+
+    def __init__(self, t):
+        self.t, self.shape = t, tuple(t.shape)
+
+    def __getitem__(self, h):
+        return self.t[h].double().cpu().numpy()
+
+
+def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None, mode=True, check_heads=None):
+    """mode True: sws_decode_step_exact (shared-memory triangle); "rows": the
+    stored-rows walk (sws_decode_step_exact_rows). check_heads: the query heads
+    compared with the oracle (all by default; a subset for the wide contexts)."""
     dev = "cuda"
     batch = len(n0s)
     group = w.hq // w.hkv
     cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed, select_group=group if shared else 0)
     h = S.Handle(cfg)
     max_len = max(n0s) + steps
-    path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev, exact=True)
+    path = S.DecodePath(h, batch, w.hq, w.hkv, max_len, w.layers, dev, exact=mode)
     check_seqs = list(range(batch)) if check_seqs is None else list(check_seqs)
+    heads = list(range(w.hq)) if check_heads is None else list(check_heads)
+    if shared:  # a shared choice needs every head of a checked head's group
+        heads = sorted({(hh // group) * group + r for hh in heads for r in range(group)})
     KV, Qs = {}, {}
     lens = torch.tensor(n0s, dtype=torch.int32, device=dev)
     for layer in range(w.layers):
@@ -49,23 +65,33 @@ def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None):
             Q = W.decode_sequence_queries(ws_, s_, layer, dev)
             path.write_cache(layer, s_, K, V, n0)
             qp[s_, :, :n0] = Q[:, :n0]
-            KV[(s_, layer)] = (K, V)
-            Qs[(s_, layer)] = Q
+            if s_ in check_seqs:
+                KV[(s_, layer)] = (K, V)
+                Qs[(s_, layer)] = Q
+            else:  # only the tokens the steps append
+                KV[(s_, layer)] = (K[:, n0:].clone(), V[:, n0:].clone())
+                Qs[(s_, layer)] = Q[:, n0:].clone()
+            del K, V, Q
         path.seq_lens.copy_(lens)
         path.init_queries(layer, qp)
         del qp
     path.init_cache(lens)
+    if mode == "rows":
+        path.init_rows()
     Hd = oracle.srht_matrix(w.d, w.k, w.seed)
-    host = {key: (K.double().cpu().numpy(), V.double().cpu().numpy(), Qs[key].double().cpu().numpy())
-            for key, (K, V) in KV.items() if key[0] in check_seqs}
+
+    def tok(s_, layer, kind, t):
+        x = Qs[(s_, layer)] if kind == "q" else KV[(s_, layer)][0 if kind == "k" else 1]
+        return x[:, (n0s[s_] if s_ in check_seqs else 0) + t]
+
     swaps = []
     for t in range(steps):
         path.begin_step()
         states = {s_: so.PrefillState() for s_ in check_seqs}
         for layer in range(w.layers):
-            q_tok = torch.stack([Qs[(s_, layer)][:, n0s[s_] + t] for s_ in range(batch)]).contiguous()
-            k_tok = torch.stack([KV[(s_, layer)][0][:, n0s[s_] + t] for s_ in range(batch)]).contiguous()
-            v_tok = torch.stack([KV[(s_, layer)][1][:, n0s[s_] + t] for s_ in range(batch)]).contiguous()
+            q_tok = torch.stack([tok(s_, layer, "q", t) for s_ in range(batch)]).contiguous()
+            k_tok = torch.stack([tok(s_, layer, "k", t) for s_ in range(batch)]).contiguous()
+            v_tok = torch.stack([tok(s_, layer, "v", t) for s_ in range(batch)]).contiguous()
             o = path.layer(layer, q_tok, k_tok, v_tok)
             torch.cuda.synchronize()
             assert S.sws_sync_check(h) == 0
@@ -79,11 +105,12 @@ def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None):
             for s_ in check_seqs:
                 length = n0s[s_] + t + 1
                 nb = -(-length // w.B)
-                Kh, Vh, Qh = host[(s_, layer)]
-                ref = so.decode_exact_layer(Qh[:, :length], Kh[:, :length], Hd, w.B, w.s, w.density, states[s_],
-                                            select="group_shared" if shared else "per_head")
+                K, V = KV[(s_, layer)]
+                Q = Qs[(s_, layer)]
+                ref = so.decode_exact_layer(_Heads(Q[:, :length]), _Heads(K[:, :length]), Hd, w.B, w.s, w.density,
+                                            states[s_], heads=heads, select="group_shared" if shared else "per_head")
                 ug = {}
-                for hh in range(w.hq):
+                for hh in heads:
                     r = ref[hh]
                     row = u_gpu[s_, hh, :nb]
                     assert np.allclose(row, r["row"], rtol=1e-4, atol=1e-9 * np.abs(r["row"]).max()), (t, layer, hh)
@@ -94,18 +121,23 @@ def run_exact(w: W.DecodeWorkload, n0s, steps, shared=False, check_seqs=None):
                     assert np.all(np.diff(gsel) > 0) and gsel.max() < nb
                     swaps += [(t, layer, s_, hh) + x for x in compare_selection(gsel, r["blocks"], r["score"])]
                     g = hh // group
-                    q = Qh[hh, length - 1]
-                    compare_attention(og[s_, hh], so.decode_attention(q, Kh[g], Vh[g], length, gsel, w.B))
+                    q = Q[hh, length - 1].double().cpu().numpy()
+                    Kg, Vg = K[g, :length].double().cpu().numpy(), V[g, :length].double().cpu().numpy()
+                    compare_attention(og[s_, hh], so.decode_attention(q, Kg, Vg, length, gsel, w.B))
                     for j in gsel:
                         ug.setdefault((g, int(j)), 0)
                         ug[(g, int(j))] |= 1 << (hh % group)
+                full_groups = {g for g in range(w.hkv) if all(g * group + r in heads for r in range(group))}
                 for g in range(w.hkv):
-                    blocks = sorted(j for (gg, j) in ug if gg == g)
                     n = cnt[s_, g]
-                    assert n == len(blocks)
-                    assert list(sel[s_, g, :n]) == blocks
-                    assert [int(m) for m in msk[s_, g, :n]] == [ug[(g, j)] for j in blocks]
-    record_ties(swaps, compared=steps * w.layers * len(check_seqs) * w.hq)
+                    got = {int(j): int(m) for j, m in zip(sel[s_, g, :n], msk[s_, g, :n])}
+                    assert list(sel[s_, g, :n]) == sorted(got)
+                    mine = {j: m for (gg, j), m in ug.items() if gg == g}
+                    if g in full_groups:
+                        assert got == mine
+                    else:  # the checked heads' blocks are in the union with their bits
+                        assert all(got.get(j, 0) & m == m for j, m in mine.items())
+    record_ties(swaps, compared=steps * w.layers * len(check_seqs) * len(heads))
     h.close()
     return swaps
 
@@ -115,6 +147,82 @@ def test_decode_exact_small_ragged():
     three layers: the walk row, the selection, the union and attention."""
     w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
     swaps = run_exact(w, [1000, 1500, 638], steps=5)
+
+
+@pytest.mark.parametrize("shared", [False, True], ids=["per_head", "group_shared"])
+def test_decode_exact_rows_small_ragged(shared):
+    """The stored-rows walk on the same small ragged case: three sequences,
+    steps crossing a block boundary, three layers."""
+    w = W.DECODE_128K.scaled(layers=3, hq=8, hkv=2, hubs=4)
+    run_exact(w, [1000, 1500, 638], steps=5, shared=shared, mode="rows")
+
+
+def test_decode_exact_rows_first_token_of_block():
+    w = W.DECODE_128K.scaled(layers=2, hq=4, hkv=1, hubs=2)
+    run_exact(w, [1024, 64], steps=2, mode="rows")
+
+
+@pytest.mark.parametrize("d,B,k", [(64, 64, 16), (128, 128, 32)])
+def test_decode_exact_rows_head_dim_and_block_size(d, B, k):
+    w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=3, d=d, B=B, k=k)
+    run_exact(w, [766, 1200, 130], steps=3, mode="rows")
+
+
+def test_decode_exact_rows_s_beyond_one_sweep():
+    """s = 11: the products take two sweeps over the stored rows (8 levels, then 3)."""
+    w = W.DECODE_128K.scaled(layers=2, hq=4, hkv=1, hubs=3, s=11)
+    run_exact(w, [2000, 700], steps=2, mode="rows")
+
+
+def test_decode_exact_rows_matches_shared_memory_walk():
+    """Where both fit (a 16K context), the stored-rows walk and the shared-memory
+    walk give the same rows up to rounding and the same selections."""
+    w = W.DECODE_128K.scaled(layers=2, hq=8, hkv=2, hubs=8, batch=2)
+    n0s = [16000, 9000]
+    outs = {}
+    for mode in (True, "rows"):
+        h = S.Handle(S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed))
+        path = S.DecodePath(h, 2, w.hq, w.hkv, max(n0s) + 1, w.layers, exact=mode)
+        lens = torch.tensor(n0s, dtype=torch.int32, device="cuda")
+        toks = []
+        for layer in range(w.layers):
+            qp = torch.zeros(2, w.hq, path.max_len, w.d, dtype=torch.bfloat16, device="cuda")
+            tl = []
+            for s_, n0 in enumerate(n0s):
+                ws_ = w.scaled(n0=n0, steps=1)
+                K, V = W.decode_cache_inputs(ws_, s_, layer, "cuda")
+                Q = W.decode_sequence_queries(ws_, s_, layer, "cuda")
+                path.write_cache(layer, s_, K, V, n0)
+                qp[s_, :, :n0] = Q[:, :n0]
+                tl.append((Q[:, n0], K[:, n0], V[:, n0]))
+            path.seq_lens.copy_(lens)
+            path.init_queries(layer, qp)
+            toks.append(tuple(torch.stack([x[c] for x in tl]).contiguous() for c in range(3)))
+        path.init_cache(lens)
+        if mode == "rows":
+            path.init_rows()
+        path.begin_step()
+        res = []
+        for layer in range(w.layers):
+            path.layer(layer, *toks[layer])
+            res.append((path.walk_state.clone(), path.head_sel.clone(), path.sel.clone(), path.sel_cnt.clone()))
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        outs[mode] = res
+        h.close()
+    for (ua, sa, ua_sel, ca), (ub, sb, ub_sel, cb) in zip(outs[True], outs["rows"]):
+        nz = ua > 1e-300
+        assert ((ua - ub).abs()[nz] / ua[nz]).max().item() < 1e-9
+        assert torch.equal(sa, sb) and torch.equal(ca, cb) and torch.equal(ua_sel, ub_sel)
+
+
+def test_decode_exact_rows_full_context_sampled():
+    """The decode workload's context (131,072 cached tokens, 2049 blocks at
+    B = 64, 32 query / 8 KV heads): the stored-rows walk over two layers, one
+    step, two sequences; the oracle's exact recurrence checked on one sequence
+    for the first and last query head."""
+    w = W.DECODE_128K.scaled(layers=2, batch=2)
+    run_exact(w, [w.n0, w.n0 - 1000], steps=1, check_seqs=[0], mode="rows", check_heads=[0, w.hq - 1])
 
 
 def test_decode_exact_first_token_of_block():

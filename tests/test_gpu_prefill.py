@@ -29,6 +29,9 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
     h = S.Handle(cfg)
     dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
     path = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, dev)
+    # the product path forms the scores on chip (sws_walk_select_sketch); the
+    # score matrix that sws_sketch writes on request is checked on its own
+    scores = torch.empty(w.hq, w.b, w.b, dtype=torch.float64, device=dev)
     Hd = oracle.srht_matrix(w.d, w.k, w.seed)
     st = so.PrefillState()
     heads = list(range(w.hq)) if heads is None else list(heads)
@@ -37,6 +40,7 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
     for layer in range(w.layers):
         Q, K, V = W.prefill_layer_inputs(w, layer, dev)
         path.layer(Q, K, V, layer == 0)
+        S.sws_sketch(h, Q, K, path.q_sk, path.k_sk, scores, path.ws_sketch)
         torch.cuda.synchronize()
         assert S.sws_sync_check(h) == 0
         ref = so.prefill_layer(LazyHeads(Q), LazyHeads(K), LazyHeads(V), Hd, w.B, w.s, w.density, st, heads=heads,
@@ -51,7 +55,7 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
             assert np.allclose(qs, r["q_tilde"], rtol=1e-6, atol=1e-6 * np.abs(r["q_tilde"]).max())
             assert np.allclose(path.k_sk[g].cpu().numpy(), r["k_tilde"], rtol=1e-6,
                                atol=1e-6 * np.abs(r["k_tilde"]).max())
-            compare_scores(path.scores[hh].cpu().numpy(), r["S"])
+            compare_scores(scores[hh].cpu().numpy(), r["S"])
             compare_walk(path.walk_state[hh].cpu().numpy(), r["R"])
             rp, ci = rp_all[hh], ci_all[hh]
             check_csr_valid(rp, ci, w.b, *w.density)
@@ -188,6 +192,85 @@ def test_repeat_runs_bit_identical():
             assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("w,mode", [
+    (W.PREFILL_16K.scaled(name="p16k", n=3000, hq=8, hkv=2, layers=3), 0),
+    (W.PREFILL_64K.scaled(name="p64k", n=9000, hq=4, hkv=1, layers=2), 0),
+    (W.PREFILL_16K.scaled(name="elementwise", n=2000, hq=4, hkv=2, layers=2), 1),
+    (W.PREFILL_16K.scaled(name="k64_d64", d=64, k=64, n=1500, hq=2, hkv=1, layers=2), 0),
+    (W.TINY.scaled(name="tiny_k16", layers=2), 0),
+], ids=lambda x: x.name if hasattr(x, "name") else str(x))
+def test_scores_on_chip_match_scores_in_memory(w, mode):
+    """sws_walk_select_sketch (scores formed on chip) against sws_sketch's score
+    matrix fed to sws_walk_select: the same walk state to rounding, the same
+    selections."""
+    dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
+    cfg = S.make_config(w.d, w.B, w.k, w.s, mode, w.density, w.seed)
+    h = S.Handle(cfg)
+    a = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype)
+    b = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, scores_in_memory=True)
+    for layer in range(w.layers):
+        Q, K, V = W.prefill_layer_inputs(w, layer, "cuda")
+        oa = a.layer(Q, K, V, layer == 0)
+        ob = b.layer(Q, K, V, layer == 0)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        assert torch.equal(a.q_sk, b.q_sk) and torch.equal(a.k_sk, b.k_sk)
+        Ra, Rb = a.walk_state, b.walk_state
+        low = Rb > 1e-280
+        rel = ((Ra - Rb).abs()[low] / Rb[low]).max().item()
+        assert rel < 1e-12, rel
+        assert torch.equal(a.row_ptr, b.row_ptr)
+        same = (a.col_idx == b.col_idx).all().item()
+        if not same:  # only where two walk scores tie to rounding
+            ca, cb = a.col_idx.cpu().numpy(), b.col_idx.cpu().numpy()
+            rp = b.row_ptr.cpu().numpy()
+            Rn = Rb.cpu().numpy()
+            for hh in range(w.hq):
+                for i in range(w.b):
+                    x, y = set(ca[hh, rp[hh, i]:rp[hh, i + 1]]), set(cb[hh, rp[hh, i]:rp[hh, i + 1]])
+                    for u, v in zip(sorted(x - y), sorted(y - x)):
+                        assert abs(Rn[hh, i, u] - Rn[hh, i, v]) <= 1e-12 * Rn[hh, i, v]
+        else:
+            assert torch.equal(oa, ob)
+    h.close()
+
+
+@pytest.mark.parametrize("w", [
+    W.PREFILL_16K.scaled(name="bf16_B64", n=3000, hq=8, hkv=2, layers=2),
+    W.PREFILL_64K.scaled(name="bf16_B128", n=2500, hq=4, hkv=1, layers=2),
+    W.PREFILL_16K.scaled(name="fp32_B64", dtype="fp32", n=1100, hq=2, hkv=1, layers=1),
+], ids=lambda w: w.name)
+def test_strided_operands_read_in_place(w):
+    """Q, K, V held as [n, heads, d] activations (the layout a model produces)
+    and O written into an [n, hq, d] buffer, through strides: the same
+    sketches, selection and output bits as the dense [heads, n, d] layout, and
+    the output within tolerance of the oracle."""
+    dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    dense = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype)
+    strided = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype)
+    for layer in range(w.layers):
+        Q, K, V = W.prefill_layer_inputs(w, layer, "cuda")
+        Qn, Kn, Vn = (x.transpose(0, 1).contiguous() for x in (Q, K, V))  # [n, heads, d]
+        Qv, Kv, Vv = (x.transpose(0, 1) for x in (Qn, Kn, Vn))          # strided [heads, n, d] views
+        assert not Qv.is_contiguous() and Qv.stride() == (w.d, w.hq * w.d, 1)
+        On = torch.full((w.n, w.hq, w.d), float("nan"), dtype=dtype, device="cuda")
+        od = dense.layer(Q, K, V, layer == 0)
+        strided.layer(Qv, Kv, Vv, layer == 0, out=On.transpose(0, 1))
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        assert torch.equal(strided.q_sk, dense.q_sk) and torch.equal(strided.k_sk, dense.k_sk)
+        assert torch.equal(strided.row_ptr, dense.row_ptr) and torch.equal(strided.col_idx, dense.col_idx)
+        assert torch.equal(On.transpose(0, 1), od)
+    # one head of the last layer against the oracle's attention on the same selection
+    rp, ci = dense.row_ptr[0].cpu().numpy(), dense.col_idx[0].cpu().numpy()
+    q64, k64, v64 = (x[0].double().cpu().numpy() for x in (Q, K, V))
+    want = so.sparse_attention(q64, k64, v64, rp, ci, w.B)
+    compare_attention(On[:, 0].float().cpu().numpy(), want)
+    h.close()
+
+
 def test_invalid_arguments_queue_nothing():
     cfg = S.make_config()
     h = S.Handle(cfg)
@@ -203,6 +286,16 @@ def test_invalid_arguments_queue_nothing():
         S.sws_walk_select(h, sc, 256, True, sc, torch.zeros(4, 5, dtype=torch.int32, device="cuda"),
                           torch.zeros(4, 8, dtype=torch.int32, device="cuda"), ws)
     assert e.value.status == S.SWS_ERR_WORKSPACE
+    # a head stride of 132 elements (264 bytes) leaves rows off the 16-byte grid
+    qpad = torch.zeros(256, 4, 132, dtype=torch.bfloat16, device="cuda")[:, :, :128].transpose(0, 1)
+    k1 = torch.zeros(1, 256, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(S.SwsError) as e:
+        S.sws_sketch(h, qpad, k1, out, out, None, ws)
+    assert e.value.status == S.SWS_ERR_INVALID_ARG
+    with pytest.raises(S.SwsError) as e:
+        S.sws_sparse_attn_prefill(h, qpad, k1, k1, torch.zeros(4, 5, dtype=torch.int32, device="cuda"),
+                                  torch.zeros(4, 8, dtype=torch.int32, device="cuda"), torch.zeros_like(q))
+    assert e.value.status == S.SWS_ERR_INVALID_ARG
 
 
 def test_dense_first_layers_policy():
