@@ -781,11 +781,11 @@ def bench_decode_exact_rows(args, world, S, W, torch, wd, path, toks_q, toks_k, 
     q_sketch = [torch.zeros(wd.batch, wd.hq, path.mb, wd.k, **f64) for _ in range(wd.layers)]
     e = S.sws_decode_exact_rows_entries(cfg, wd.max_len)
     rows = [torch.empty(wd.batch, wd.hq, e, dtype=torch.int32, device="cuda") for _ in range(wd.layers)]
+    len1 = torch.full((1,), wd.n0, dtype=torch.int32, device="cuda")  # one sequence's length, 16-byte aligned
     for layer in range(wd.layers):
         for s_ in range(wd.batch):
             Q = W.decode_sequence_queries(wd, s_, layer, "cuda")[None]  # [1, hq, max_len, d]
-            S.sws_decode_init_cache(h, Q, path.seq_lens[s_:s_ + 1], q_psum[layer][s_:s_ + 1],
-                                    q_sketch[layer][s_:s_ + 1])
+            S.sws_decode_init_cache(h, Q, len1, q_psum[layer][s_:s_ + 1], q_sketch[layer][s_:s_ + 1])
             del Q
         S.sws_decode_exact_rows_init(h, q_sketch[layer], path.k_sketch[layer], path.seq_lens, rows[layer])
     torch.cuda.synchronize()
@@ -937,7 +937,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded AR(1) + sink + hub generator (sws_inputs); no datasets or weights",
         "config": head["config"], "stages_ms_per_step": head["stages_ms_per_step"], "roofline": head["roofline"],
-        "sketch_roofline": head["sketch_roofline"], "clocks": head["clocks"], "gpu_launches": head["gpu_launches"],
+        "sketch_roofline": head["sketch_roofline"], "attention_mma_work": head["attention_mma_work"],
+        "clocks": head["clocks"], "gpu_launches": head["gpu_launches"],
     }
     if not args.no_e2e:
         line["e2e"] = bench_prefill_e2e(args, world, S, torch, pf)
