@@ -383,7 +383,10 @@ def bench_prefill(args, world, S, W, torch, w, steps):
             attn_ms.append(a)
     stage = {k: v / steps for k, v in stage.items()}
     flops = w.hq * path.nnz * 4 * w.B * w.B * w.d  # executed block pairs x 4 B^2 d
-    sketch_bytes = (w.hq + w.hkv) * w.n * w.d * 2 + 8 * (w.hq + w.hkv) * path.b * w.k + 8 * w.hq * path.b * (path.b + 1) // 2
+    # Q and K read once, the sketches written; the score matrix only when it is formed in memory
+    sketch_bytes = (w.hq + w.hkv) * w.n * w.d * 2 + 8 * (w.hq + w.hkv) * path.b * w.k
+    if path.scores_in_memory:
+        sketch_bytes += 8 * w.hq * path.b * (path.b + 1) // 2
     res = dict(w=w, h=h, path=path, inputs=inputs, ms=ms_max, steps=steps, launches=launches, clocks=clk,
                stage=stage, attn_ms=statistics.mean(attn_ms), flops=flops, sketch_bytes=sketch_bytes,
                in_bytes=in_bytes, mma_work=mma_work(path, w, torch))
@@ -471,6 +474,47 @@ def prefill_summary(pf, world, peaks, peak_kind) -> dict:
         "clocks": pf["clocks"], "gpu_launches": pf["launches"],
         "attention_mma_work": pf["mma_work"],
     }
+
+
+def bench_scores_on_chip(args, world, S, torch, pf):
+    """The headline step with the sketched scores formed on chip inside the walk
+    (sws_sketch without the score matrix, then sws_walk_select_sketch), on the
+    same inputs: the route that keeps the b x b matrix out of device memory."""
+    w, inputs = pf["w"], pf["inputs"]
+    path = S.PrefillPath(pf["h"], w.n, w.hq, w.hkv, torch.bfloat16, scores_in_memory=False)
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, 20))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(w.layers * steps)]
+
+    def step(rec):
+        for layer, (Q, K, V) in enumerate(inputs):
+            e = ev[rec * w.layers + layer] if rec is not None else None
+            if e:
+                e[0].record(stream)
+            path.sketch(Q, K)
+            path.walk_select(layer == 0)
+            if e:
+                e[1].record(stream)
+            path.attention(Q, K, V)
+            if e:
+                e[2].record(stream)
+
+    for _ in range(args.warmup):
+        step(None)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(pf["h"]) == 0
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    sw = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    del path
+    return {"tokens_per_s": world * w.n / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
+            "sketch_walk_select_ms_per_step": sw}
 
 
 def bench_prefill_variants(args, world, S, W, torch, pf):
@@ -942,6 +986,8 @@ def main():
     }
     if not args.no_e2e:
         line["e2e"] = bench_prefill_e2e(args, world, S, torch, pf)
+    if not args.no_variants:
+        line["headline_variants"] = {"scores_on_chip": bench_scores_on_chip(args, world, S, torch, pf)}
     pf["h"].close()
     del pf
     torch.cuda.empty_cache()

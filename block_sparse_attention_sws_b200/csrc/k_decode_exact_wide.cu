@@ -207,23 +207,43 @@ __global__ void __launch_bounds__(kRowThreads) exact_append_rows_kernel(
              rows + h0 * rows_offset(max_blocks), static_cast<float>(1.0 / sqrt(static_cast<double>(k))), rsm);
 }
 
-// Step part 2: u <- u A^s for one (sequence, query head). NT threads, each
-// owning columns 4t .. 4t + 3; NT * 4 >= max_blocks.
-constexpr int kLevels = 8;  // levels of the product per sweep over the rows
+// Step part 2: u <- u A^s for one (sequence, query head), one sweep over the
+// stored rows per kLevels levels. Rows go in blocks of 32 from the newest
+// block up to block 0. For the columns j left of a block, part[l][j] gathers
+// sum over the rows m of the blocks below of u_l[m] A[m][j] (shared memory,
+// all levels). Per block M, between two barriers:
+//  * warp 0 adds block M's rows to the 32 columns of block M - 32 and then
+//    resolves block M - 32's diagonal triangle level by level: u_{l+1}[m] =
+//    part[l][m] + sum over the block's rows m' >= m of u_l[m'] A[m'][m],
+//    publishing u_0 .. u_{L-1} of its rows for the next block's updates;
+//  * the other warps add block M's rows to every column left of block M - 32,
+//    two adjacent columns a thread at a time (8-byte row reads, the next four
+//    rows loaded while the current four are added), summing over the block's
+//    rows in registers before one update of part.
+// So the chain through the diagonal runs beside the bulk of the row reads,
+// and every stored entry is read once per sweep, in a fixed order.
+constexpr int kLevels = 8;        // levels of the product per sweep over the rows
+constexpr int kWalkThreads = 512;
+constexpr int kWalkWorkers = kWalkThreads - 32;
 
-template <int NT>
-__global__ void __launch_bounds__(NT, 1) exact_walk_kernel(const uint32_t* __restrict__ rows, int64_t max_len,
-                                                           int64_t max_blocks, const int32_t* __restrict__ seq_lens,
-                                                           int32_t B, int32_t hq, int first_layer, int32_t s_pow,
-                                                           double* __restrict__ walk_state, int32_t* err) {
+__device__ __forceinline__ uint2 ld_rows8(const uint32_t* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
+    const uint32_t* __restrict__ rows, int64_t max_len, int64_t max_blocks, const int32_t* __restrict__ seq_lens,
+    int32_t B, int32_t hq, int first_layer, int32_t s_pow, double* __restrict__ walk_state, int32_t* err) {
   grid_dependency_wait();
   allow_dependents();
   extern __shared__ __align__(16) double wsm[];
-  double* u_in = wsm;                                   // [max_blocks]
-  double* u_out = u_in + max_blocks;                    // [max_blocks]
-  double* ub = u_out + max_blocks;                      // [32][kLevels]: u_l of the block's rows
-  double* pd = ub + 32 * kLevels;                       // [kLevels][32]: partial sums of the block's columns
-  uint32_t* ad = reinterpret_cast<uint32_t*>(pd + kLevels * 32);  // [32][33]: the diagonal block
+  const int64_t mbp = (max_blocks + 31) & ~int64_t(31);
+  double* part = wsm;                          // [kLevels][mbp]
+  double* u_in = part + kLevels * mbp;         // [mbp]
+  double* u_out = u_in + mbp;                  // [mbp]
+  double* ub = u_out + mbp;                    // [2][32][kLevels]: u_l of a block's rows (by block parity)
+  uint32_t* ad = reinterpret_cast<uint32_t*>(ub + 2 * 32 * kLevels);  // [32][33]: a diagonal triangle
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t unit = blockIdx.x;
   const int bi = static_cast<int>(unit / hq);
@@ -236,77 +256,112 @@ __global__ void __launch_bounds__(NT, 1) exact_walk_kernel(const uint32_t* __res
   const int i = nb - 1;
   const uint32_t* A = rows + unit * rows_offset(max_blocks);
   double* wrow = walk_state + unit * max_blocks;
-  for (int j = tid; j < nb; j += NT) u_in[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
-  const int c0 = 4 * tid;  // this thread's first column
+  for (int j = tid; j < nb; j += kWalkThreads) u_in[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
+  const int mtop = (i / 32) * 32;
+
+  // warp 0: the diagonal triangle of block M (its columns' part complete)
+  auto diag = [&](int M, int L) {
+    const int m = M + lane;
+    const bool live = m <= i;
+    // the block's triangle, row r of the block in ad[r][.] (zeros above the diagonal and past the newest row)
+    for (int r = 0; r < 32; ++r) ad[r * 33 + lane] = (r >= lane && M + r <= i) ? A[rows_offset(M + r) + m] : 0u;
+    __syncwarp();
+    double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
+    double uprev = live ? u_in[m] : 0.0;
+    for (int l = 0; l < kLevels; ++l) {
+      if (l >= L) {  // levels past this sweep's: zeros, so every product that reads them adds 0
+        ubm[lane * kLevels + l] = 0.0;
+        continue;
+      }
+      ubm[lane * kLevels + l] = uprev;
+      double acc = live ? part[l * mbp + m] : 0.0;
+#pragma unroll 8
+      for (int r = 31; r >= 0; --r) {
+        const double v = __shfl_sync(0xffffffffu, uprev, r);
+        acc = fma(v, from_hi(ad[r * 33 + lane]), acc);
+      }
+      uprev = acc;
+    }
+    if (live) u_out[m] = uprev;
+  };
+
   for (int done = 0; done < s_pow; done += kLevels) {
     const int L = min(kLevels, s_pow - done);
-    double part[4][kLevels];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int l = 0; l < kLevels; ++l) part[c][l] = 0.0;
-    for (int M = (i / 32) * 32; M >= 0; M -= 32) {
-      // the block's columns: their partial sums (all rows below the block are in) and the diagonal block
-      if (c0 >= M && c0 < M + 32) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int l = 0; l < kLevels; ++l) pd[l * 32 + (c0 - M) + c] = part[c][l];
-      }
-      for (int x = tid; x < 32 * 32; x += NT) {
-        const int rr = x >> 5, cc = x & 31;  // row M + rr, column M + cc
-        ad[rr * 33 + cc] = (M + rr <= i && cc <= rr) ? A[rows_offset(M + rr) + M + cc] : 0u;
-      }
-      __syncthreads();
+    for (int x = tid; x < kLevels * mbp; x += kWalkThreads) part[x] = 0.0;
+    __syncthreads();
+    if (warp == 0) diag(mtop, L);
+    __syncthreads();
+    for (int M = mtop; M > 0; M -= 32) {
+      const int nrows = min(32, i - M + 1);
+      const double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
       if (warp == 0) {
-        // u_{l+1}[m] = (rows below the block) + sum over the block's rows m' >= m of u_l[m'] A[m', m]
-        const int m = M + lane;
-        double uprev = m <= i ? u_in[m] : 0.0;
-        for (int l = 0; l < L; ++l) {
-          ub[lane * kLevels + l] = uprev;
-          double acc = pd[l * 32 + lane];
+        // block M's rows into the columns of block M - 32, then that block's diagonal
+        const int c = M - 32 + lane;
+        double acc[kLevels];
 #pragma unroll
-          for (int rr = 31; rr >= 0; --rr) {
-            const double v = __shfl_sync(0xffffffffu, uprev, rr);
-            if (rr >= lane) acc = fma(v, from_hi(ad[rr * 33 + lane]), acc);
-          }
-          uprev = acc;
+        for (int l = 0; l < kLevels; ++l) acc[l] = 0.0;
+        for (int r = 0; r < nrows; ++r) {
+          const double av = from_hi(A[rows_offset(M + r) + c]);
+#pragma unroll
+          for (int l = 0; l < kLevels; ++l) acc[l] = fma(ubm[r * kLevels + l], av, acc[l]);
         }
-        if (m <= i) u_out[m] = uprev;
-      }
-      __syncthreads();
-      // the block's rows into the columns to the left of it
-      if (c0 < M) {
-        const int rend = min(32, i - M + 1);
-        for (int r = 0; r < rend; r += 4) {
-          uint4 a[4];
+        for (int l = 0; l < L; ++l) part[l * mbp + c] += acc[l];
+        __syncwarp();
+        diag(M - 32, L);
+      } else {
+        // block M's rows into the columns left of block M - 32, two at a time
+        const int ng = (M - 32) / 2;
+        for (int grp = tid - 32; grp < ng; grp += kWalkWorkers) {
+          const int c0 = 2 * grp;
+          double acc[2][kLevels];
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int l = 0; l < kLevels; ++l) acc[c][l] = 0.0;
+          uint2 cur[4], nxt[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            a[q] = (r + q < rend) ? __ldg(reinterpret_cast<const uint4*>(A + rows_offset(M + r + q) + c0))
-                                  : make_uint4(0u, 0u, 0u, 0u);
+            cur[q] = q < nrows ? ld_rows8(A + rows_offset(M + q) + c0) : make_uint2(0u, 0u);
+          for (int r = 0; r < nrows; r += 4) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const double av[4] = {from_hi(a[q].x), from_hi(a[q].y), from_hi(a[q].z), from_hi(a[q].w)};
-            const double* uq = ub + (r + q) * kLevels;
+            for (int q = 0; q < 4; ++q)
+              nxt[q] = (r + 4 + q < nrows) ? ld_rows8(A + rows_offset(M + r + 4 + q) + c0) : make_uint2(0u, 0u);
 #pragma unroll
-            for (int l = 0; l < kLevels; ++l) {
-              const double u = uq[l];
+            for (int q = 0; q < 4; ++q) {
+              const double a0 = from_hi(cur[q].x), a1 = from_hi(cur[q].y);
+              const double2* uq = reinterpret_cast<const double2*>(ubm + (r + q) * kLevels);  // rows past the newest carry u = 0
 #pragma unroll
-              for (int c = 0; c < 4; ++c) part[c][l] = fma(u, av[c], part[c][l]);
+              for (int l2 = 0; l2 < kLevels / 2; ++l2) {
+                const double2 u = uq[l2];
+                acc[0][2 * l2] = fma(u.x, a0, acc[0][2 * l2]);
+                acc[1][2 * l2] = fma(u.x, a1, acc[1][2 * l2]);
+                acc[0][2 * l2 + 1] = fma(u.y, a0, acc[0][2 * l2 + 1]);
+                acc[1][2 * l2 + 1] = fma(u.y, a1, acc[1][2 * l2 + 1]);
+              }
             }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+          }
+          for (int l = 0; l < L; ++l) {
+            double2* pp = reinterpret_cast<double2*>(part + l * mbp + c0);
+            double2 p0 = *pp;
+            p0.x += acc[0][l];
+            p0.y += acc[1][l];
+            *pp = p0;
           }
         }
       }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int j = tid; j < nb; j += NT) u_in[j] = u_out[j];
+    for (int j = tid; j < nb; j += kWalkThreads) u_in[j] = u_out[j];
     __syncthreads();
   }
-  for (int j = tid; j < nb; j += NT) wrow[j] = u_in[j];
+  for (int j = tid; j < nb; j += kWalkThreads) wrow[j] = u_in[j];
 }
 
 size_t walk_smem_bytes(int64_t max_blocks) {
-  return (2 * static_cast<size_t>(max_blocks) + 2 * 32 * kLevels) * sizeof(double) + 32 * 33 * sizeof(uint32_t);
+  const size_t mbp = static_cast<size_t>((max_blocks + 31) & ~int64_t(31));
+  return ((kLevels + 2) * mbp + 2 * 32 * kLevels) * sizeof(double) + 32 * 33 * sizeof(uint32_t);
 }
 
 // Step part 3: per head the top-tau of its row (or the group's summed rows for
@@ -401,16 +456,14 @@ size_t select_smem_bytes(int64_t max_blocks, int group) {
          static_cast<size_t>(group) * 256 * 4 + static_cast<size_t>(group) * 4 * 4 + kSelWarps * 4;
 }
 
-template <int NT>
 cudaError_t launch_walk(const uint32_t* rows, int64_t max_len, int64_t mb, int32_t batch, int32_t hq,
                         const int32_t* seq_lens, int32_t B, int first_layer, int32_t s_pow, double* walk_state,
                         int32_t* err, cudaStream_t st) {
   const size_t smem = walk_smem_bytes(mb);
-  auto kern = exact_walk_kernel<NT>;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const cudaError_t e = cudaFuncSetAttribute(exact_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, static_cast<unsigned>((int64_t)batch * hq), NT, smem, st, rows, max_len, mb, seq_lens, B, hq,
-                  first_layer, s_pow, walk_state, err);
+  return launch_k(exact_walk_kernel, static_cast<unsigned>((int64_t)batch * hq), kWalkThreads, smem, st, rows,
+                  max_len, mb, seq_lens, B, hq, first_layer, s_pow, walk_state, err);
 }
 
 }  // namespace
@@ -418,7 +471,8 @@ cudaError_t launch_walk(const uint32_t* rows, int64_t max_len, int64_t mb, int32
 int64_t exact_rows_entries(int64_t max_blocks) { return rows_offset(max_blocks); }
 
 bool exact_wide_supported(const sws_config& c, int64_t max_blocks, int32_t group) {
-  return c.sketch_dim <= kMaxK && group >= 1 && group <= 8 && max_blocks <= 2560 && max_blocks <= 0x7fff &&
+  return c.sketch_dim <= kMaxK && group >= 1 && group <= 8 && max_blocks <= 2560 &&
+         walk_smem_bytes(max_blocks) <= (227u << 10) &&
          select_smem_bytes(max_blocks, group) <= (227u << 10) &&
          rows_smem_bytes(c.sketch_dim, group, 32) <= (200u << 10);
 }
@@ -463,16 +517,8 @@ cudaError_t launch_decode_exact_wide(const sws_handle* h, const __nv_bfloat16* q
   }
   // 2. the walk row of every head
   {
-    cudaError_t e;
-    if (mb <= 4 * 256)
-      e = launch_walk<256>(rows, max_len, mb, batch, hq, seq_lens, c.block_size, first_layer, c.walk_power, walk_state,
-                           h->err, st);
-    else if (mb <= 4 * 544)
-      e = launch_walk<544>(rows, max_len, mb, batch, hq, seq_lens, c.block_size, first_layer, c.walk_power, walk_state,
-                           h->err, st);
-    else
-      e = launch_walk<640>(rows, max_len, mb, batch, hq, seq_lens, c.block_size, first_layer, c.walk_power, walk_state,
-                           h->err, st);
+    const cudaError_t e = launch_walk(rows, max_len, mb, batch, hq, seq_lens, c.block_size, first_layer, c.walk_power,
+                                      walk_state, h->err, st);
     if (e != cudaSuccess) return e;
   }
   // 3. selection and union

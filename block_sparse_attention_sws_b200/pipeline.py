@@ -20,13 +20,14 @@ class PrefillPath:
     through a second handle with density 1/1 and the same projection, while
     the walk state still runs through them.
 
-    ``scores_in_memory`` = False (the default) skips the [hq, b, b] score
-    matrix: sws_sketch writes only the sketches and sws_walk_select_sketch
-    forms the scores on chip. True keeps the score matrix (``self.scores``)
-    and calls sws_walk_select on it."""
+    ``scores_in_memory`` = True (the default) has sws_sketch write the
+    [hq, b, b] score matrix (``self.scores``) and sws_walk_select walk on it:
+    the faster route at every measured size. False skips the matrix (and its
+    memory): sws_sketch writes only the sketches and sws_walk_select_sketch
+    forms the scores on chip."""
 
     def __init__(self, handle: L.Handle, n: int, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda",
-                 dense_layers: int = 0, scores_in_memory: bool = False):
+                 dense_layers: int = 0, scores_in_memory: bool = True):
         cfg = handle.cfg
         self.dense_layers = dense_layers
         self.scores_in_memory = scores_in_memory

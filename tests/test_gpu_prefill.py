@@ -29,9 +29,9 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
     h = S.Handle(cfg)
     dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
     path = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, dev)
-    # the product path forms the scores on chip (sws_walk_select_sketch); the
-    # score matrix that sws_sketch writes on request is checked on its own
-    scores = torch.empty(w.hq, w.b, w.b, dtype=torch.float64, device=dev)
+    # the score matrix of the path, or (when the path forms the scores on chip)
+    # one that sws_sketch writes on request, is checked against the oracle
+    scores = path.scores if path.scores is not None else torch.empty(w.hq, w.b, w.b, dtype=torch.float64, device=dev)
     Hd = oracle.srht_matrix(w.d, w.k, w.seed)
     st = so.PrefillState()
     heads = list(range(w.hq)) if heads is None else list(heads)
@@ -40,7 +40,8 @@ def run_case(w: W.PrefillWorkload, heads=None, blocks=None, mode=S.SWS_WALK_MATR
     for layer in range(w.layers):
         Q, K, V = W.prefill_layer_inputs(w, layer, dev)
         path.layer(Q, K, V, layer == 0)
-        S.sws_sketch(h, Q, K, path.q_sk, path.k_sk, scores, path.ws_sketch)
+        if path.scores is None:
+            S.sws_sketch(h, Q, K, path.q_sk, path.k_sk, scores, path.ws_sketch)
         torch.cuda.synchronize()
         assert S.sws_sync_check(h) == 0
         ref = so.prefill_layer(LazyHeads(Q), LazyHeads(K), LazyHeads(V), Hd, w.B, w.s, w.density, st, heads=heads,
@@ -206,7 +207,7 @@ def test_scores_on_chip_match_scores_in_memory(w, mode):
     dtype = torch.float32 if w.dtype == "fp32" else torch.bfloat16
     cfg = S.make_config(w.d, w.B, w.k, w.s, mode, w.density, w.seed)
     h = S.Handle(cfg)
-    a = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype)
+    a = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, scores_in_memory=False)
     b = S.PrefillPath(h, w.n, w.hq, w.hkv, dtype, scores_in_memory=True)
     for layer in range(w.layers):
         Q, K, V = W.prefill_layer_inputs(w, layer, "cuda")
