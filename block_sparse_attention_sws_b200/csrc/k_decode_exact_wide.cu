@@ -217,8 +217,8 @@ __global__ void __launch_bounds__(kRowThreads) exact_append_rows_kernel(
 //    part[l][m] + sum over the block's rows m' >= m of u_l[m'] A[m'][m],
 //    publishing u_0 .. u_{L-1} of its rows for the next block's updates;
 //  * the other warps add block M's rows to every column left of block M - 32,
-//    two adjacent columns a thread at a time (8-byte row reads, the next four
-//    rows loaded while the current four are added), summing over the block's
+//    two adjacent columns a thread at a time (8-byte row reads, the next eight
+//    rows loaded while the current eight are added), summing over the block's
 //    rows in registers before one update of part.
 // So the chain through the diagonal runs beside the bulk of the row reads,
 // and every stored entry is read once per sweep, in a fixed order.
@@ -300,10 +300,14 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         double acc[kLevels];
 #pragma unroll
         for (int l = 0; l < kLevels; ++l) acc[l] = 0.0;
-        for (int r = 0; r < nrows; ++r) {
-          const double av = from_hi(A[rows_offset(M + r) + c]);
+        uint32_t av[32];  // every row's entry in flight at once
 #pragma unroll
-          for (int l = 0; l < kLevels; ++l) acc[l] = fma(ubm[r * kLevels + l], av, acc[l]);
+        for (int r = 0; r < 32; ++r) av[r] = r < nrows ? A[rows_offset(M + r) + c] : 0u;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          const double a = from_hi(av[r]);
+#pragma unroll
+          for (int l = 0; l < kLevels; ++l) acc[l] = fma(ubm[r * kLevels + l], a, acc[l]);
         }
         for (int l = 0; l < L; ++l) part[l * mbp + c] += acc[l];
         __syncwarp();
@@ -318,16 +322,17 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
           for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int l = 0; l < kLevels; ++l) acc[c][l] = 0.0;
-          uint2 cur[4], nxt[4];
+          constexpr int kRB = 8;  // rows a batch; the next batch's loads fly while this one is added
+          uint2 cur[kRB], nxt[kRB];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < kRB; ++q)
             cur[q] = q < nrows ? ld_rows8(A + rows_offset(M + q) + c0) : make_uint2(0u, 0u);
-          for (int r = 0; r < nrows; r += 4) {
+          for (int r = 0; r < nrows; r += kRB) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              nxt[q] = (r + 4 + q < nrows) ? ld_rows8(A + rows_offset(M + r + 4 + q) + c0) : make_uint2(0u, 0u);
+            for (int q = 0; q < kRB; ++q)
+              nxt[q] = (r + kRB + q < nrows) ? ld_rows8(A + rows_offset(M + r + kRB + q) + c0) : make_uint2(0u, 0u);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < kRB; ++q) {
               const double a0 = from_hi(cur[q].x), a1 = from_hi(cur[q].y);
               const double2* uq = reinterpret_cast<const double2*>(ubm + (r + q) * kLevels);  // rows past the newest carry u = 0
 #pragma unroll
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
               }
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+            for (int q = 0; q < kRB; ++q) cur[q] = nxt[q];
           }
           for (int l = 0; l < L; ++l) {
             double2* pp = reinterpret_cast<double2*>(part + l * mbp + c0);
