@@ -21,11 +21,11 @@
 //     and q~, then write the newest row of A for each query head of the group;
 //  2. exact_walk_kernel, one CTA per (sequence, query head): u <- u A^s in one
 //     sweep over the rows per eight levels of s, from the newest block up to
-//     block 0 in blocks of 32 rows. Each thread keeps the partial sums of four
-//     columns for the eight levels in registers; the 32 x 32 diagonal block of
-//     a row block is resolved level by level by one warp, then every thread
-//     adds the block's rows to its columns to the left of it (16-byte row
-//     reads). Each entry of the rows is read once per sweep, in fixed order;
+//     block 0 in blocks of 32 rows. Shared memory holds the partial sums of
+//     every column for the eight levels. One warp resolves the 32 x 32
+//     diagonal block of a row block level by level, after adding the block
+//     below it; the other warps add the block's rows to the columns left of it
+//     on the fp64 tensor path. Each entry of the rows is read once per sweep;
 //  3. exact_select_kernel, one CTA per (sequence, KV head): the top-tau of
 //     each head's row (or one choice for the group) and the union.
 #include <algorithm>
@@ -217,19 +217,32 @@ __global__ void __launch_bounds__(kRowThreads) exact_append_rows_kernel(
 //    part[l][m] + sum over the block's rows m' >= m of u_l[m'] A[m'][m],
 //    publishing u_0 .. u_{L-1} of its rows for the next block's updates;
 //  * the other warps add block M's rows to every column left of block M - 32,
-//    two adjacent columns a thread at a time (8-byte row reads, the next eight
-//    rows loaded while the current eight are added), summing over the block's
-//    rows in registers before one update of part.
+//    16 columns a warp at a time on the fp64 tensor path (the 8 levels are the
+//    n of an m16n8k4 product, the block's rows its k), the next chunk's rows
+//    loaded while the current chunk's products run, then one update of part.
 // So the chain through the diagonal runs beside the bulk of the row reads,
 // and every stored entry is read once per sweep, in a fixed order.
 constexpr int kLevels = 8;        // levels of the product per sweep over the rows
 constexpr int kWalkThreads = 512;
-constexpr int kWalkWorkers = kWalkThreads - 32;
+constexpr int kWalkWarps = kWalkThreads / 32;
 
-__device__ __forceinline__ uint2 ld_rows8(const uint32_t* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
+__device__ __forceinline__ void dmma_16x8x4(double (&c)[4], double a0, double a1, double b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
+      : "d"(a0), "d"(a1), "d"(b0));
+}
+
+// 4-byte asynchronous copy into shared memory; valid == false writes zero and reads nothing.
+__device__ __forceinline__ void cp_async4(uint32_t* dst, const uint32_t* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Pulls `bytes` (a multiple of 16, from a 16-byte aligned address) into L2; no registers, no completion.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
@@ -244,6 +257,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
   double* u_out = u_in + mbp;                  // [mbp]
   double* ub = u_out + mbp;                    // [2][32][kLevels]: u_l of a block's rows (by block parity)
   uint32_t* ad = reinterpret_cast<uint32_t*>(ub + 2 * 32 * kLevels);  // [32][33]: a diagonal triangle
+  uint32_t* ar = ad + 32 * 33;                 // [32][32]: a row block's entries in the columns of the block below
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t unit = blockIdx.x;
   const int bi = static_cast<int>(unit / hq);
@@ -259,13 +273,32 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
   for (int j = tid; j < nb; j += kWalkThreads) u_in[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
   const int mtop = (i / 32) * 32;
 
-  // warp 0: the diagonal triangle of block M (its columns' part complete)
+  // warp 0 copies into shared memory, asynchronously, the entries its next
+  // step reads: the triangle of block T in ad[r][.] (row T + r; zeros above the
+  // diagonal and past the newest row) and, for T < M, the rows of block M in
+  // the columns of block T in ar[r][.]. Issued as soon as the previous step has
+  // read them, so the copies run while the other warps work.
+  auto stage = [&](int T, int M) {
+    const int c = T + lane;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      const bool ok = r >= lane && T + r <= i;
+      cp_async4(ad + r * 33 + lane, ok ? A + rows_offset(T + r) + c : A, ok);
+    }
+    if (T < M) {
+#pragma unroll 8
+      for (int r = 0; r < 32; ++r) {
+        const bool ok = M + r <= i;
+        cp_async4(ar + r * 32 + lane, ok ? A + rows_offset(M + r) + c : A, ok);
+      }
+    }
+  };
+
+  // warp 0: the diagonal triangle of block M (its columns' part complete, its
+  // triangle staged in ad)
   auto diag = [&](int M, int L) {
     const int m = M + lane;
     const bool live = m <= i;
-    // the block's triangle, row r of the block in ad[r][.] (zeros above the diagonal and past the newest row)
-    for (int r = 0; r < 32; ++r) ad[r * 33 + lane] = (r >= lane && M + r <= i) ? A[rows_offset(M + r) + m] : 0u;
-    __syncwarp();
     double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
     double uprev = live ? u_in[m] : 0.0;
     for (int l = 0; l < kLevels; ++l) {
@@ -274,85 +307,110 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         continue;
       }
       ubm[lane * kLevels + l] = uprev;
-      double acc = live ? part[l * mbp + m] : 0.0;
-#pragma unroll 8
+      // four interleaved partial sums (rows r = 3, 2, 1, 0 mod 4), added in a fixed order
+      double acc[4] = {live ? part[l * mbp + m] : 0.0, 0.0, 0.0, 0.0};
+#pragma unroll
       for (int r = 31; r >= 0; --r) {
         const double v = __shfl_sync(0xffffffffu, uprev, r);
-        acc = fma(v, from_hi(ad[r * 33 + lane]), acc);
+        acc[r & 3] = fma(v, from_hi(ad[r * 33 + lane]), acc[r & 3]);
       }
-      uprev = acc;
+      uprev = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
     if (live) u_out[m] = uprev;
   };
 
+  // The rows of block M (rows M .. M + 31 up to the newest), pulled into L2 two
+  // blocks ahead of their reads by one warp (a bulk prefetch per row), so that
+  // the many small row reads of the other warps find them there.
+  auto prefetch_block = [&](int M) {
+    if (M < 0) return;
+    const int m = M + lane;
+    if (m <= i) prefetch_l2(A + rows_offset(m), static_cast<uint32_t>(((m + 1 + 3) & ~3) * 4));
+  };
   for (int done = 0; done < s_pow; done += kLevels) {
     const int L = min(kLevels, s_pow - done);
+    if (warp == 1) {
+      prefetch_block(mtop);
+      prefetch_block(mtop - 32);
+    }
     for (int x = tid; x < kLevels * mbp; x += kWalkThreads) part[x] = 0.0;
+    if (warp == 0) stage(mtop, mtop);
     __syncthreads();
-    if (warp == 0) diag(mtop, L);
+    if (warp == 0) {
+      cp_async_wait_all();
+      __syncwarp();
+      diag(mtop, L);
+      __syncwarp();
+      if (mtop > 0) stage(mtop - 32, mtop);
+    }
     __syncthreads();
     for (int M = mtop; M > 0; M -= 32) {
       const int nrows = min(32, i - M + 1);
       const double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
+      if (warp == 1) prefetch_block(M - 64);
       if (warp == 0) {
-        // block M's rows into the columns of block M - 32, then that block's diagonal
+        // block M's rows into the columns of block M - 32, then that block's
+        // diagonal; both were staged during the previous step
         const int c = M - 32 + lane;
-        double acc[kLevels];
+        cp_async_wait_all();
+        __syncwarp();
+        double acc[2][kLevels];  // rows of even and odd index, added at the end
 #pragma unroll
-        for (int l = 0; l < kLevels; ++l) acc[l] = 0.0;
-        uint32_t av[32];  // every row's entry in flight at once
-#pragma unroll
-        for (int r = 0; r < 32; ++r) av[r] = r < nrows ? A[rows_offset(M + r) + c] : 0u;
+        for (int l = 0; l < kLevels; ++l) acc[0][l] = acc[1][l] = 0.0;
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
-          const double a = from_hi(av[r]);
+          const double a = from_hi(ar[r * 32 + lane]);
 #pragma unroll
-          for (int l = 0; l < kLevels; ++l) acc[l] = fma(ubm[r * kLevels + l], a, acc[l]);
+          for (int l = 0; l < kLevels; ++l) acc[r & 1][l] = fma(ubm[r * kLevels + l], a, acc[r & 1][l]);
         }
-        for (int l = 0; l < L; ++l) part[l * mbp + c] += acc[l];
+        for (int l = 0; l < L; ++l) part[l * mbp + c] += acc[0][l] + acc[1][l];
         __syncwarp();
         diag(M - 32, L);
+        __syncwarp();
+        if (M - 32 > 0) stage(M - 64, M - 32);
       } else {
-        // block M's rows into the columns left of block M - 32, two at a time
-        const int ng = (M - 32) / 2;
-        for (int grp = tid - 32; grp < ng; grp += kWalkWorkers) {
-          const int c0 = 2 * grp;
-          double acc[2][kLevels];
+        // block M's rows into the columns left of block M - 32 on the fp64 tensor
+        // path: per 16 columns, D[column][level] += sum over the block's rows r of
+        // A[M + r][column] u_level[M + r], i.e. D (16 x 8) += A^T (16 x 4) U (4 x 8)
+        // over the block's 32 rows in 8 products of m16n8k4 (the 8 levels are n).
+        // Lane (g, t4) holds A at rows 4 kk + t4, columns g and g + 8 of the chunk.
+        const int g = lane >> 2, t4 = lane & 3;
+        const int nchunk = (M - 32) / 16;
+        const int wk = warp - 1;
+        uint32_t cur[8][2], nxt[8][2];
+        auto load_chunk = [&](int ch, uint32_t (&dst)[8][2]) {
+          const int c0 = 16 * ch;
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int l = 0; l < kLevels; ++l) acc[c][l] = 0.0;
-          constexpr int kRB = 8;  // rows a batch; the next batch's loads fly while this one is added
-          uint2 cur[kRB], nxt[kRB];
-#pragma unroll
-          for (int q = 0; q < kRB; ++q)
-            cur[q] = q < nrows ? ld_rows8(A + rows_offset(M + q) + c0) : make_uint2(0u, 0u);
-          for (int r = 0; r < nrows; r += kRB) {
-#pragma unroll
-            for (int q = 0; q < kRB; ++q)
-              nxt[q] = (r + kRB + q < nrows) ? ld_rows8(A + rows_offset(M + r + kRB + q) + c0) : make_uint2(0u, 0u);
-#pragma unroll
-            for (int q = 0; q < kRB; ++q) {
-              const double a0 = from_hi(cur[q].x), a1 = from_hi(cur[q].y);
-              const double2* uq = reinterpret_cast<const double2*>(ubm + (r + q) * kLevels);  // rows past the newest carry u = 0
-#pragma unroll
-              for (int l2 = 0; l2 < kLevels / 2; ++l2) {
-                const double2 u = uq[l2];
-                acc[0][2 * l2] = fma(u.x, a0, acc[0][2 * l2]);
-                acc[1][2 * l2] = fma(u.x, a1, acc[1][2 * l2]);
-                acc[0][2 * l2 + 1] = fma(u.y, a0, acc[0][2 * l2 + 1]);
-                acc[1][2 * l2 + 1] = fma(u.y, a1, acc[1][2 * l2 + 1]);
-              }
-            }
-#pragma unroll
-            for (int q = 0; q < kRB; ++q) cur[q] = nxt[q];
+          for (int kk = 0; kk < 8; ++kk) {
+            const int r = 4 * kk + t4;
+            const uint32_t* row = A + rows_offset(M + r);
+            const bool ok = r < nrows;
+            dst[kk][0] = ok ? __ldg(row + c0 + g) : 0u;
+            dst[kk][1] = ok ? __ldg(row + c0 + g + 8) : 0u;
           }
-          for (int l = 0; l < L; ++l) {
-            double2* pp = reinterpret_cast<double2*>(part + l * mbp + c0);
-            double2 p0 = *pp;
-            p0.x += acc[0][l];
-            p0.y += acc[1][l];
-            *pp = p0;
+        };
+        if (wk < nchunk) load_chunk(wk, cur);
+        for (int ch = wk; ch < nchunk; ch += kWalkWarps - 1) {
+          const int nc = ch + kWalkWarps - 1;
+          if (nc < nchunk) load_chunk(nc, nxt);
+          double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            dmma_16x8x4(acc, from_hi(cur[kk][0]), from_hi(cur[kk][1]), ubm[(4 * kk + t4) * kLevels + g]);
+          // acc: D[g][2 t4], D[g][2 t4 + 1], D[g + 8][2 t4], D[g + 8][2 t4 + 1]
+          const int c0 = 16 * ch;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int l = 2 * t4 + e;
+            if (l < L) {
+              part[l * mbp + c0 + g] += acc[e];
+              part[l * mbp + c0 + g + 8] += acc[2 + e];
+            }
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            cur[kk][0] = nxt[kk][0];
+            cur[kk][1] = nxt[kk][1];
           }
         }
       }
@@ -366,7 +424,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
 
 size_t walk_smem_bytes(int64_t max_blocks) {
   const size_t mbp = static_cast<size_t>((max_blocks + 31) & ~int64_t(31));
-  return ((kLevels + 2) * mbp + 2 * 32 * kLevels) * sizeof(double) + 32 * 33 * sizeof(uint32_t);
+  return ((kLevels + 2) * mbp + 2 * 32 * kLevels) * sizeof(double) + (32 * 33 + 32 * 32) * sizeof(uint32_t);
 }
 
 // Step part 3: per head the top-tau of its row (or the group's summed rows for
