@@ -416,6 +416,158 @@ __global__ void __launch_bounds__(kGemmThreads, 3) tri_gemm_kernel(const double*
   }
 }
 
+// The same product with 64 x 64 output tiles, for walks of 1024 blocks and more.
+//
+// One CTA of four warps per tile, four CTAs per SM, operands staged in shared
+// memory: the k range of the tile, key blocks J..I, is streamed in steps of 16
+// through a double-buffered cp.async ring (a 64 x 16 panel of A and a 16 x 64
+// panel of Bm per step). Entries above the diagonals of A and Bm are never
+// read: the copies stop at the diagonal and fill the rest of the panel with
+// zeros, so the products need no masks. Each warp owns a 32 x 32 quarter of
+// the tile for the whole k range (eight independent accumulators, one
+// fragment load per product) and skips the k steps outside its own part of
+// the triangle, so the executed work is 1.10 x the b^3/3 of the product at
+// b = 1024. The panels are padded (A rows 20 doubles, Bm rows 68) so that the
+// fragment reads of each half-warp fall in distinct banks. Staging quarters
+// the L2 traffic of the 32 x 32 tiles; each element is summed in k order.
+constexpr int kW64 = 64, kW64Warps = 4, kW64Threads = 32 * kW64Warps, kW64K = 16, kW64Stages = 2;
+constexpr int kW64LdA = kW64K + 4;   // A panel [m][k]
+constexpr int kW64LdB = kW64 + 4;    // Bm panel [k][n]
+constexpr int kW64StageA = kW64 * kW64LdA, kW64StageB = kW64K * kW64LdB;  // doubles
+constexpr size_t kW64Smem = sizeof(double) * kW64Stages * (kW64StageA + kW64StageB);
+constexpr int64_t kW64MinB = 1024;  // smaller walks keep the 32 x 32 tiles (more CTAs; faster at b = 512)
+
+__device__ __forceinline__ void cp_async16_n(double* dst, const double* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes)
+               : "memory");
+}
+
+template <bool kPairs>
+__global__ void __launch_bounds__(kW64Threads, 4) tri_gemm64_kernel(const double* __restrict__ A,
+                                                                   const double* __restrict__ Bm,
+                                                                   double* __restrict__ C, int64_t b64, int32_t hq) {
+  grid_dependency_wait();
+  allow_dependents();
+  extern __shared__ __align__(16) double w64[];
+  const int b = static_cast<int>(b64);  // b <= 8192: every offset inside a head fits in 32 bits
+  const int nt = (b + kW64 - 1) / kW64;
+  const int64_t head = blockIdx.x % hq;  // tile-major: every head's heaviest tile first
+  int64_t ti64, tj64;
+  tile_of(blockIdx.x / hq, nt, ti64, tj64);
+  const size_t hoff = (size_t)head * b * b;
+  const double* Ah = A + hoff;
+  const double* Bh = Bm + hoff;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int i0 = static_cast<int>(ti64) * kW64, j0 = static_cast<int>(tj64) * kW64;
+  const int kend = min(b, i0 + kW64);
+  const int nsteps = (kend - j0 + kW64K - 1) / kW64K;
+
+  auto load = [&](int st, int slot) {
+    double* sa = w64 + slot * (kW64StageA + kW64StageB);
+    double* sb = sa + kW64StageA;
+    const int k0 = j0 + kW64K * st;
+    if (kPairs) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {  // A: 64 rows x 8 pairs; A[i][k] is read for k <= i < b
+        const int piece = tid + x * kW64Threads;
+        const int m = piece >> 3, pr = piece & 7;
+        const int i = i0 + m, k = k0 + 2 * pr;
+        const int n = i < b ? min(max(i - k + 1, 0), 2) : 0;
+        cp_async16_n(sa + m * kW64LdA + 2 * pr, n ? Ah + i * b + k : Ah, 8 * n);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {  // Bm: 16 rows x 32 pairs; Bm[k][j] is read for j <= k < b
+        const int piece = tid + x * kW64Threads;
+        const int kk = piece >> 5, pr = piece & 31;
+        const int k = k0 + kk, j = j0 + 2 * pr;
+        const int n = k < b ? min(max(k - j + 1, 0), 2) : 0;
+        cp_async16_n(sb + kk * kW64LdB + 2 * pr, n ? Bh + k * b + j : Bh, 8 * n);
+      }
+    } else {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {  // A: 64 rows x 16
+        const int e = tid + x * kW64Threads;
+        const int m = e >> 4, kk = e & 15;
+        const int i = i0 + m, k = k0 + kk;
+        const bool ok = i < b && k <= i;
+        cp_async8_w(sa + m * kW64LdA + kk, ok ? Ah + i * b + k : Ah, ok);
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {  // Bm: 16 rows x 64
+        const int e = tid + x * kW64Threads;
+        const int kk = e >> 6, c = e & 63;
+        const int k = k0 + kk, j = j0 + c;
+        const bool ok = k < b && j <= k;
+        cp_async8_w(sb + kk * kW64LdB + c, ok ? Bh + k * b + j : Bh, ok);
+      }
+    }
+  };
+
+  const int wm = warp >> 1, wn = warp & 1;
+  const int r0 = 32 * wm, c0 = 32 * wn;  // the warp's 32 x 32 part of the tile
+  // the warp's k range: Bm is zero below its first column, A past its last row
+  const int wk_lo = j0 + c0, wk_hi = i0 + r0 + 31;
+  double acc[2][4][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[h][n][v] = 0.0;
+
+  load(0, 0);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int st = 0; st < nsteps; ++st) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (st + 1 < nsteps) load(st + 1, (st + 1) & 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const double* sa = w64 + (st & 1) * (kW64StageA + kW64StageB);
+    const double* sb = sa + kW64StageA;
+    const int k0 = j0 + kW64K * st;
+#pragma unroll
+    for (int q = 0; q < kW64K / 4; ++q) {
+      const int k = k0 + 4 * q;
+      if (k + 3 < wk_lo || k > wk_hi) continue;  // all four k of the step are zero for this warp
+      double fa[2][2], fb[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        fa[h][0] = sa[(r0 + 16 * h + g) * kW64LdA + 4 * q + t4];
+        fa[h][1] = sa[(r0 + 16 * h + g + 8) * kW64LdA + 4 * q + t4];
+      }
+#pragma unroll
+      for (int n = 0; n < 4; ++n) fb[n] = sb[(4 * q + t4) * kW64LdB + c0 + 8 * n + g];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) dmma_16x8x4(acc[h][n], fa[h][0], fa[h][1], fb[n]);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+  // accumulator element v of (h, n): row r0 + 16h + g + 8(v >> 1), column c0 + 8n + 2 t4 + (v & 1)
+  double* Ch = C + hoff;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int hv = 0; hv < 2; ++hv) {
+      const int i = i0 + r0 + 16 * h + g + 8 * hv;
+      if (i >= b) continue;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        const int j = j0 + c0 + 8 * n + 2 * t4;
+        const double x0 = acc[h][n][2 * hv], x1 = acc[h][n][2 * hv + 1];
+        if (kPairs && j + 1 < b) {
+          *reinterpret_cast<double2*>(Ch + (int64_t)i * b + j) = make_double2(x0, x1);
+        } else {
+          if (j < b) Ch[(int64_t)i * b + j] = x0;
+          if (j + 1 < b) Ch[(int64_t)i * b + j + 1] = x1;
+        }
+      }
+    }
+}
+
 // One warp per row: copies R's row to the walk state (zeros above the
 // diagonal), writes row_ptr, and emits the row's top-tau blocks ascending.
 // With G > 1 query heads sharing a selection, a warp takes one row of a
@@ -572,6 +724,18 @@ cudaError_t launch_sketch_softmax(const sws_handle* h, const double* q_sk, const
 }
 
 cudaError_t launch_tri_gemm(const double* A, const double* Bm, double* C, int64_t b, int32_t hq, cudaStream_t st) {
+  if (b >= kW64MinB) {
+    const int64_t nt = ceil_div64(b, kW64);
+    const int64_t ctas = nt * (nt + 1) / 2 * hq;
+    if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+    auto kern = (b & 1) == 0 ? tri_gemm64_kernel<true> : tri_gemm64_kernel<false>;
+    const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kW64Smem);
+    if (ea != cudaSuccess) return ea;
+    const cudaError_t le = launch_k(kern, static_cast<unsigned>(ctas), kW64Threads, kW64Smem, st, A, Bm, C, b, hq);
+    if (le != cudaSuccess) return le;
+    note_launches(1);
+    return cudaGetLastError();
+  }
   const int64_t nt = ceil_div64(b, kTT);
   const int64_t ctas = nt * (nt + 1) / 2 * hq;  // one CTA per tile
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;

@@ -353,6 +353,17 @@ def test_beyond_1024_blocks(shared):
     swaps = run_case(w, blocks=sorted({0, 1, 511, 1023, 1024, b - 2, b - 1}), shared=shared)
 
 
+@pytest.mark.parametrize("b", [1025, 1030])
+def test_walk_products_on_64_tiles(b):
+    """Walks of 1024 blocks and more take the 64 x 64 tiles of the walk product.
+    b = 1025 (odd: rows not 16-byte aligned, 8-byte copies) and b = 1030 (a
+    ragged last tile row): the whole walk chain of two heads over two layers
+    against the oracle, attention on sampled query blocks."""
+    w = W.PREFILL_16K.scaled(name=f"b{b}_B64", n=b * 64 - 21, hq=2, hkv=1, layers=2)
+    assert w.b == b
+    run_case(w, blocks=sorted({0, 1, 63, 64, 511, b - 2, b - 1}))
+
+
 def test_prefill_batch_matches_single_sequences():
     """PrefillBatch: three sequences of different lengths (ragged tails), their
     layers on concurrent streams, give bit for bit what each sequence gives
