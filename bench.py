@@ -558,9 +558,10 @@ def bench_prefill_variants(args, world, S, W, torch, pf):
 
 def bench_prefill_batch(args, world, S, W, torch):
     """Prefill batching: eight 2048-token sequences of the headline workload's
-    shape (4 layers, 32/8 heads), through PrefillBatch (each sequence's layer
-    on its own stream) and, for comparison, the same paths one after another
-    on one stream."""
+    shape (4 layers, 32/8 heads), through PrefillBatch: each sequence's layer
+    on its own stream; the sequences packed end to end with one attention
+    launch for all (the sketches and walks on their streams); and, for
+    comparison, the same paths one after another on one stream."""
     base = W.PREFILL_16K
     ws = [base.scaled(name=f"seq{i}", n=2048, seed=base.seed + 100 + i) for i in range(8)]
     inputs = [[W.prefill_layer_inputs(w, layer, "cuda") for w in ws] for layer in range(base.layers)]
@@ -569,11 +570,14 @@ def bench_prefill_batch(args, world, S, W, torch):
     stream = torch.cuda.current_stream()
     steps = max(3, min(args.steps, 20))
     out = {"sequences": len(ws), "tokens_per_sequence": 2048, "steps": steps}
-    for mode in ("concurrent_streams", "one_stream"):
+    packed = [[torch.cat([x[j] for x in ins], dim=1) for j in range(3)] for ins in inputs]
+    for mode in ("concurrent_streams", "packed_launch", "one_stream"):
         def step():
             for layer, ins in enumerate(inputs):
                 if mode == "concurrent_streams":
                     batch.layer([x[0] for x in ins], [x[1] for x in ins], [x[2] for x in ins], layer == 0)
+                elif mode == "packed_launch":
+                    batch.layer_packed(*packed[layer], layer == 0)
                 else:
                     for p, (Q, K, V) in zip(batch.paths, ins):
                         p.layer(Q, K, V, layer == 0)

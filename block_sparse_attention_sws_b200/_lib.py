@@ -26,7 +26,8 @@ EXPORTS = [
     "sws_status_string", "sws_config_check", "sws_num_blocks", "sws_csr_nnz", "sws_build_projection_host",
     "sws_workspace_size", "sws_create", "sws_destroy", "sws_projection_device", "sws_launch_count",
     "sws_sync_check", "sws_layout_check", "sws_sketch",
-    "sws_walk_select", "sws_walk_select_sketch", "sws_sparse_attn_prefill", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
+    "sws_walk_select", "sws_walk_select_sketch", "sws_sparse_attn_prefill", "sws_sparse_attn_prefill_varlen_ws_bytes",
+    "sws_sparse_attn_prefill_varlen", "sws_decode_init_cache", "sws_decode_advance", "sws_decode_step",
     "sws_sparse_attn_decode", "sws_sparse_attn_decode_noalloc", "sws_decode_init_cache_paged", "sws_decode_step_paged",
     "sws_sparse_attn_decode_paged", "sws_decode_step_exact", "sws_decode_exact_rows_entries",
     "sws_decode_exact_rows_init", "sws_decode_step_exact_rows",
@@ -78,6 +79,9 @@ def load() -> ctypes.CDLL:
         "sws_walk_select_sketch": (ctypes.c_int, [P, P, P, I64, I32, I32, ctypes.c_int, P, P, P, P, SZ, P]),
         "sws_sparse_attn_prefill": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I64, I32, I32, P, P, P, P, P, P, P, P,
                                                    SZ, P]),
+        "sws_sparse_attn_prefill_varlen_ws_bytes": (SZ, [I32, P]),
+        "sws_sparse_attn_prefill_varlen": (ctypes.c_int, [P, P, P, P, ctypes.c_int, I32, P, I32, I32, P, P, P, P, P, P,
+                                                          P, P, SZ, P]),
         "sws_decode_init_cache": (ctypes.c_int, [P, P, I32, I32, I64, P, P, P, P]),
         "sws_decode_advance": (ctypes.c_int, [P, P, I32, P]),
         "sws_decode_step": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I64, P, P, P, P, P, ctypes.c_int, P, P, P, P,
@@ -264,6 +268,34 @@ def sws_sparse_attn_prefill(h: Handle, q, k, v, row_ptr, col_idx, o, ws=None, st
     _check(load().sws_sparse_attn_prefill(h.ptr, qp, kp, vp, _dtype_code(q), n, hq, hkv, qs, ks, vs, os_,
                                           _ptr(row_ptr), _ptr(col_idx), op, wsp, wsb, _stream(stream)),
            "sws_sparse_attn_prefill")
+
+
+def _cu_array(cu_seqlens):
+    return (ctypes.c_int64 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+
+
+def sws_sparse_attn_prefill_varlen_ws_bytes(cu_seqlens) -> int:
+    """Workspace bytes of a packed launch over the sequences cu_seqlens describes
+    (0 for an invalid list)."""
+    return int(load().sws_sparse_attn_prefill_varlen_ws_bytes(len(cu_seqlens) - 1, _cu_array(cu_seqlens)))
+
+
+def sws_sparse_attn_prefill_varlen(h: Handle, q, k, v, cu_seqlens, row_ptrs, col_idxs, o, ws, stream=None) -> None:
+    """q, o [hq, N, d], k, v [hkv, N, d] bf16 (dense or strided views with contiguous
+    rows), the sequences end to end along N; cu_seqlens: nseq + 1 token offsets
+    (host); row_ptrs, col_idxs: each sequence's CSR tensors."""
+    nseq = len(cu_seqlens) - 1
+    hq = q.shape[0]
+    hkv = k.shape[0]
+    if len(row_ptrs) != nseq or len(col_idxs) != nseq:
+        raise ValueError("one CSR per sequence")
+    rp = (ctypes.c_void_p * nseq)(*[_ptr(t) for t in row_ptrs])
+    ci = (ctypes.c_void_p * nseq)(*[_ptr(t) for t in col_idxs])
+    (qp, qs), (kp, ks), (vp, vs), (op, os_) = _head_tok(q), _head_tok(k), _head_tok(v), _head_tok(o)
+    _check(load().sws_sparse_attn_prefill_varlen(h.ptr, qp, kp, vp, _dtype_code(q), nseq, _cu_array(cu_seqlens), hq,
+                                                 hkv, qs, ks, vs, os_, rp, ci, op, _ptr(ws),
+                                                 ws.numel() * ws.element_size(), _stream(stream)),
+           "sws_sparse_attn_prefill_varlen")
 
 
 # ---------------------------------------------------------------- decode ----

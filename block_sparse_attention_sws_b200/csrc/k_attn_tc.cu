@@ -30,9 +30,20 @@
 //             rescaled); P = 2^(s - m) goes to the group's P columns as bf16 once
 //             its previous PV has read them; the group finally writes O / l.
 // Every wait is bounded; a timeout records a guard code and all roles leave.
+//
+// Packed sequences (kVar): one launch over several sequences laid end to end
+// along the token axis of Q, K, V and O. A table of (sequence, slab) entries,
+// longest slabs first across all sequences, replaces the slab index, and each
+// sequence brings its own token offset, length and CSR. Keys past a
+// sequence's end are never unmasked (a selected block before the query's own
+// is complete, and the diagonal block is causal), and rows past its end are
+// not written, so sequences never see each other. The pipeline itself (the
+// barriers, the roles) does not change: the MMA issuers never look at an
+// item's identity.
 #include <cuda.h>
 
 #include <algorithm>
+#include <vector>
 
 #include "sws_common.cuh"
 
@@ -206,6 +217,23 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
 
 // ---- shared state ----------------------------------------------------------------
 
+// One sequence of a packed launch: rows tok0 .. tok0 + n - 1 of the packed
+// tensors; per head its CSR has b + 1 offsets (row_ptr + h (b + 1)) and nnz
+// columns (col_idx + h nnz).
+struct SeqDesc {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  int64_t nnz, n, tok0, b;
+};
+
+// What a role needs of one work item.
+struct ItemCtx {
+  int32_t h, p;  // query head, 256-row slab of the sequence
+  int64_t tok0, n, b, nnz;
+  const int32_t* rp;  // the head's CSR
+  const int32_t* ci;
+};
+
 struct TileMeta {
   int32_t u0, u1;  // key blocks of the two 64-key halves (B = 64), or the key block twice (B = 128)
   int32_t mask;    // bit (key_block_slot * QB + query_block_slot): that query block selected that key block
@@ -342,12 +370,12 @@ struct TileWalker {
   }
 };
 
-template <int D, int BLK>
+template <int D, int BLK, bool kVar>
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
     const __grid_constant__ CUtensorMap tmv, int64_t n, int32_t hq, int32_t group, const int32_t* __restrict__ row_ptr,
     const int32_t* __restrict__ col_idx, int64_t nnz, __nv_bfloat16* __restrict__ o, HeadTok os, float qscale,
-    int32_t* err) {
+    const SeqDesc* __restrict__ seqs, const int2* __restrict__ ents, int32_t nent, int32_t* err) {
   grid_dependency_wait();
   allow_dependents();
   using L = Smem<D>;
@@ -358,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = ceil_div64(n, BLK);
   const int32_t nslab = static_cast<int32_t>(ceil_div64(n, 2 * kTileM));
-  const int64_t items = static_cast<int64_t>(nslab) * hq;
+  const int64_t items = static_cast<int64_t>(kVar ? nent : nslab) * hq;
 
   if (threadIdx.x == 0) {
     mbar_init(&bs->q_full, 1);
@@ -391,9 +419,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
   tc_fence_after();
   const uint32_t tmem = bs->tmem_base;
 
-  auto item_of = [&](int64_t t, int32_t& h, int32_t& p) {
-    p = nslab - 1 - static_cast<int32_t>(t / hq);  // longest rows first
-    h = static_cast<int32_t>(t % hq);
+  auto item_of = [&](int64_t t) {
+    ItemCtx c;
+    c.h = static_cast<int32_t>(t % hq);
+    if constexpr (kVar) {
+      const int2 e = ents[t / hq];  // sorted longest slab first on the host
+      const SeqDesc* sd = seqs + e.x;
+      c.p = e.y;
+      c.tok0 = sd->tok0;
+      c.n = sd->n;
+      c.b = sd->b;
+      c.nnz = sd->nnz;
+      c.rp = sd->row_ptr + static_cast<int64_t>(c.h) * (c.b + 1);
+      c.ci = sd->col_idx + static_cast<int64_t>(c.h) * c.nnz;
+    } else {
+      c.p = nslab - 1 - static_cast<int32_t>(t / hq);  // longest rows first
+      c.tok0 = 0;
+      c.n = n;
+      c.b = b;
+      c.nnz = nnz;
+      c.rp = row_ptr + static_cast<int64_t>(c.h) * (b + 1);
+      c.ci = col_idx + static_cast<int64_t>(c.h) * nnz;
+    }
+    return c;
   };
 
   if (warp == 0) {
@@ -401,8 +449,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     if (lane == 0) {
       uint32_t kv_it = 0, item_cnt = 0;
       for (int64_t t = blockIdx.x; t < items && !bs->abort; t += gridDim.x, ++item_cnt) {
-        int32_t h, p;
-        item_of(t, h, p);
+        const ItemCtx it = item_of(t);
+        const int32_t h = it.h, p = it.p;
+        const int32_t tok0 = static_cast<int32_t>(it.tok0);  // the packed token count fits in 32 bits
         const int32_t g = h / group;
         if (!wait_bar(&bs->q_empty, (item_cnt & 1) ^ 1, bs, err)) break;
         mbar_arrive_expect_tx(&bs->q_full, 2 * L::kQ);
@@ -410,10 +459,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
         for (int w = 0; w < 2; ++w)
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
-            tma_load_3d(smem + L::q + w * L::kQ + a * (kTileM * 128), &tmq, a * 64, p * 2 * kTileM + w * kTileM, h,
-                        &bs->q_full);
+            tma_load_3d(smem + L::q + w * L::kQ + a * (kTileM * 128), &tmq, a * 64,
+                        tok0 + p * 2 * kTileM + w * kTileM, h, &bs->q_full);
         TileWalker<BLK> wk;
-        wk.init(row_ptr + static_cast<int64_t>(h) * (b + 1), col_idx + static_cast<int64_t>(h) * nnz, b, nnz, p, err);
+        wk.init(it.rp, it.ci, it.b, it.nnz, p, err);
         TileMeta cur, nxt;
         bool have = wk.next_tile(cur);
         if (!have) {  // a corrupt CSR: keep the pipeline shape with one fully masked tile
@@ -432,10 +481,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
 #pragma unroll
           for (int a = 0; a < D / 64; ++a) {
             if constexpr (BLK == 128) {
-              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 128, g, &bs->k_full[sk]);
+              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, tok0 + cur.u0 * 128, g, &bs->k_full[sk]);
             } else {
-              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, cur.u0 * 64, g, &bs->k_full[sk]);
-              tma_load_3d(ks + a * (kTileN * 128) + 64 * 128, &tmk, a * 64, cur.u1 * 64, g, &bs->k_full[sk]);
+              tma_load_3d(ks + a * (kTileN * 128), &tmk, a * 64, tok0 + cur.u0 * 64, g, &bs->k_full[sk]);
+              tma_load_3d(ks + a * (kTileN * 128) + 64 * 128, &tmk, a * 64, tok0 + cur.u1 * 64, g, &bs->k_full[sk]);
             }
           }
           if (!wait_bar(&bs->v_empty[sv], ((kv_it / kVStages) & 1) ^ 1, bs, err)) break;
@@ -444,10 +493,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
 #pragma unroll
           for (int a = 0; a < D / 64; ++a) {
             if constexpr (BLK == 128) {
-              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 128, g, &bs->v_full[sv]);
+              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, tok0 + cur.u0 * 128, g, &bs->v_full[sv]);
             } else {
-              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, cur.u0 * 64, g, &bs->v_full[sv]);
-              tma_load_3d(vs + a * (kTileN * 128) + 64 * 128, &tmv, a * 64, cur.u1 * 64, g, &bs->v_full[sv]);
+              tma_load_3d(vs + a * (kTileN * 128), &tmv, a * 64, tok0 + cur.u0 * 64, g, &bs->v_full[sv]);
+              tma_load_3d(vs + a * (kTileN * 128) + 64 * 128, &tmv, a * 64, tok0 + cur.u1 * 64, g, &bs->v_full[sv]);
             }
           }
           ++kv_it;
@@ -541,9 +590,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
     uint32_t kv_it = 0, gt = 0, item_cnt = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok && t < items; t += gridDim.x, ++item_cnt) {
-      int32_t h, p;
-      item_of(t, h, p);
-      const int64_t tok = static_cast<int64_t>(p) * 2 * kTileM + w * kTileM + r;
+      const ItemCtx it = item_of(t);
+      const int32_t h = it.h, p = it.p;
+      const int64_t tok = static_cast<int64_t>(p) * 2 * kTileM + w * kTileM + r;  // row of the sequence
       const int64_t qi = static_cast<int64_t>(p) * QB + qslot;  // query block of this row
       float m_used = -INFINITY, l = 0.f;
       bool first_tile = true;
@@ -659,12 +708,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(
       if (!(ok = warp_wait(&bs->pv_done[w], (gt - 1) & 1, bs, err))) break;
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = o + h * os.head + tok * os.tok;
+      __nv_bfloat16* orow = o + h * os.head + (it.tok0 + tok) * os.tok;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
         tmem_ld32(to + c * 32, v);
-        if (tok < n) {
+        if (tok < it.n) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 u = make_uint4(pack_bf16x2(v[q * 8 + 0] * inv, v[q * 8 + 1] * inv),
@@ -731,7 +780,7 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
       !make_map(&mv, v, n, hkv, D, BLK == 128 ? 128 : 64, lay.v))
     return cudaErrorInvalidValue;
   const size_t smem = Smem<D>::total + 1024;
-  auto kern = attn_tc_kernel<D, BLK>;
+  auto kern = attn_tc_kernel<D, BLK, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t b = ceil_div64(n, BLK);
@@ -741,8 +790,66 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
   const int grid = static_cast<int>(std::min<int64_t>(items, h->num_sms));
   const float qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
   {
-    const cudaError_t le = launch_k(kern, grid, kTcThreads, smem, st, mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx,
-                                    nnz, static_cast<__nv_bfloat16*>(o), lay.o, qscale, h->err);
+    const cudaError_t le =
+        launch_k(kern, grid, kTcThreads, smem, st, mq, mk, mv, n, hq, hq / hkv, row_ptr, col_idx, nnz,
+                 static_cast<__nv_bfloat16*>(o), lay.o, qscale, static_cast<const SeqDesc*>(nullptr),
+                 static_cast<const int2*>(nullptr), 0, h->err);
+    if (le != cudaSuccess) return le;
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// Workspace of a packed launch: the sequence table, then the (sequence, slab)
+// entries, longest slab first.
+size_t varlen_table_bytes(int32_t nseq, const int64_t* cu) {
+  int64_t ent = 0;
+  for (int32_t s = 0; s < nseq; ++s) ent += ceil_div64(cu[s + 1] - cu[s], 2 * kTileM);
+  return ((nseq * sizeof(SeqDesc) + 15) & ~size_t(15)) + static_cast<size_t>(ent) * sizeof(int2);
+}
+
+template <int D, int BLK>
+cudaError_t launch_tc_var(const sws_handle* h, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
+                          const PrefillLayout& lay, int32_t nseq, const int64_t* cu, const int32_t* const* row_ptr,
+                          const int32_t* const* col_idx, void* o, void* ws, cudaStream_t st) {
+  const int64_t ntot = cu[nseq];
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, ntot, hq, D, kTileM, lay.q) || !make_map(&mk, k, ntot, hkv, D, BLK == 128 ? 128 : 64, lay.k) ||
+      !make_map(&mv, v, ntot, hkv, D, BLK == 128 ? 128 : 64, lay.v))
+    return cudaErrorInvalidValue;
+  // the tables, built here and copied into the workspace in stream order (a
+  // pageable source is staged before the call returns; no device wait)
+  const size_t tab = (nseq * sizeof(SeqDesc) + 15) & ~size_t(15);
+  std::vector<uint8_t> host(varlen_table_bytes(nseq, cu));
+  SeqDesc* sd = reinterpret_cast<SeqDesc*>(host.data());
+  int2* ent = reinterpret_cast<int2*>(host.data() + tab);
+  int32_t max_slab = 0;
+  for (int32_t s = 0; s < nseq; ++s) {
+    const int64_t n = cu[s + 1] - cu[s], b = ceil_div64(n, BLK);
+    int64_t nnz = 0;
+    for (int64_t i = 0; i < b; ++i) nnz += tau_of_row(i, h->cfg.density_num, h->cfg.density_den);
+    sd[s] = SeqDesc{row_ptr[s], col_idx[s], nnz, n, cu[s], b};
+    max_slab = std::max(max_slab, static_cast<int32_t>(ceil_div64(n, 2 * kTileM)));
+  }
+  int32_t nent = 0;
+  for (int32_t p = max_slab - 1; p >= 0; --p)  // longest slabs first, sequences in order within a length
+    for (int32_t s = 0; s < nseq; ++s)
+      if (ceil_div64(cu[s + 1] - cu[s], 2 * kTileM) > p) ent[nent++] = make_int2(s, p);
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = Smem<D>::total + 1024;
+  auto kern = attn_tc_kernel<D, BLK, true>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t items = static_cast<int64_t>(nent) * hq;
+  const int grid = static_cast<int>(std::min<int64_t>(items, h->num_sms));
+  const float qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
+  const auto* wsb = static_cast<const uint8_t*>(ws);
+  {
+    const cudaError_t le =
+        launch_k(kern, grid, kTcThreads, smem, st, mq, mk, mv, ntot, hq, hq / hkv, static_cast<const int32_t*>(nullptr),
+                 static_cast<const int32_t*>(nullptr), int64_t(0), static_cast<__nv_bfloat16*>(o), lay.o, qscale,
+                 reinterpret_cast<const SeqDesc*>(wsb), reinterpret_cast<const int2*>(wsb + tab), nent, h->err);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);
@@ -750,6 +857,23 @@ cudaError_t launch_tc(const sws_handle* h, const void* q, const void* k, const v
 }
 
 }  // namespace
+
+size_t attn_prefill_varlen_ws_bytes(int32_t nseq, const int64_t* cu_seqlens) {
+  return varlen_table_bytes(nseq, cu_seqlens);
+}
+
+cudaError_t launch_attn_prefill_tc_varlen(const sws_handle* h, const void* q, const void* k, const void* v,
+                                          int32_t hq, int32_t hkv, const PrefillLayout& lay, int32_t nseq,
+                                          const int64_t* cu_seqlens, const int32_t* const* row_ptr,
+                                          const int32_t* const* col_idx, void* o, void* ws, cudaStream_t st) {
+  const int d = h->cfg.head_dim, B = h->cfg.block_size;
+  if (d == 128) {
+    return B == 128 ? launch_tc_var<128, 128>(h, q, k, v, hq, hkv, lay, nseq, cu_seqlens, row_ptr, col_idx, o, ws, st)
+                    : launch_tc_var<128, 64>(h, q, k, v, hq, hkv, lay, nseq, cu_seqlens, row_ptr, col_idx, o, ws, st);
+  }
+  return B == 128 ? launch_tc_var<64, 128>(h, q, k, v, hq, hkv, lay, nseq, cu_seqlens, row_ptr, col_idx, o, ws, st)
+                  : launch_tc_var<64, 64>(h, q, k, v, hq, hkv, lay, nseq, cu_seqlens, row_ptr, col_idx, o, ws, st);
+}
 
 cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
                                    int32_t hq, int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr,

@@ -496,6 +496,43 @@ sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const voi
                      "prefill attention (fp32)");
 }
 
+size_t sws_sparse_attn_prefill_varlen_ws_bytes(int32_t nseq, const int64_t* cu_seqlens) {
+  if (nseq < 1 || !cu_seqlens) return 0;
+  for (int32_t s = 0; s < nseq; ++s)
+    if (cu_seqlens[s + 1] <= cu_seqlens[s]) return 0;
+  return attn_prefill_varlen_ws_bytes(nseq, cu_seqlens);
+}
+
+sws_status sws_sparse_attn_prefill_varlen(const sws_handle* h, const void* q, const void* k, const void* v,
+                                          sws_dtype dtype, int32_t nseq, const int64_t* cu_seqlens, int32_t hq,
+                                          int32_t hkv, const int64_t q_strides[2], const int64_t k_strides[2],
+                                          const int64_t v_strides[2], const int64_t o_strides[2],
+                                          const int32_t* const* row_ptr, const int32_t* const* col_idx, void* o,
+                                          void* ws, size_t ws_bytes, void* stream) {
+  if (!h || nseq < 1 || !cu_seqlens || !row_ptr || !col_idx || check_heads(hq, hkv) != SWS_OK)
+    return SWS_ERR_INVALID_ARG;
+  if (dtype != SWS_BF16) return dtype == SWS_FP32 ? SWS_ERR_UNSUPPORTED : SWS_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return SWS_ERR_INVALID_ARG;
+  for (int32_t s = 0; s < nseq; ++s) {
+    if (cu_seqlens[s + 1] <= cu_seqlens[s]) return SWS_ERR_INVALID_ARG;
+    if (!aligned16(row_ptr[s]) || !aligned16(col_idx[s])) return SWS_ERR_INVALID_ARG;
+    if (ceil_div64(cu_seqlens[s + 1] - cu_seqlens[s], h->cfg.block_size) > kMaxPrefillBlocks)
+      return SWS_ERR_UNSUPPORTED;
+  }
+  const int64_t ntot = cu_seqlens[nseq];
+  if (ntot > INT32_MAX - 2 * 128) return SWS_ERR_UNSUPPORTED;  // token coordinates of the tensor maps
+  const int32_t d = h->cfg.head_dim;
+  PrefillLayout lay{};
+  if (!head_tok(q_strides, ntot, d, 2, &lay.q) || !head_tok(k_strides, ntot, d, 2, &lay.k) ||
+      !head_tok(v_strides, ntot, d, 2, &lay.v) || !head_tok(o_strides, ntot, d, 2, &lay.o))
+    return SWS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws)) return SWS_ERR_INVALID_ARG;
+  if (ws_bytes < attn_prefill_varlen_ws_bytes(nseq, cu_seqlens)) return SWS_ERR_WORKSPACE;
+  return cuda_status(launch_attn_prefill_tc_varlen(h, q, k, v, hq, hkv, lay, nseq, cu_seqlens, row_ptr, col_idx, o,
+                                                   ws, static_cast<cudaStream_t>(stream)),
+                     "prefill attention (packed sequences)");
+}
+
 sws_status sws_decode_init_cache(const sws_handle* h, const void* k_cache, int32_t batch, int32_t hkv,
                                  int64_t max_len, const int32_t* seq_lens, double* k_psum, double* k_sketch,
                                  void* stream) {

@@ -204,6 +204,11 @@ cudaError_t launch_attn_prefill_simt(const sws_handle* h, const void* q, const v
                                      int64_t n, int32_t hq, int32_t hkv, const PrefillLayout& lay,
                                      const int32_t* row_ptr, const int32_t* col_idx, void* o, cudaStream_t st);
 
+size_t attn_prefill_varlen_ws_bytes(int32_t nseq, const int64_t* cu_seqlens);
+cudaError_t launch_attn_prefill_tc_varlen(const sws_handle* h, const void* q, const void* k, const void* v,
+                                          int32_t hq, int32_t hkv, const PrefillLayout& lay, int32_t nseq,
+                                          const int64_t* cu_seqlens, const int32_t* const* row_ptr,
+                                          const int32_t* const* col_idx, void* o, void* ws, cudaStream_t st);
 cudaError_t launch_attn_prefill_tc(const sws_handle* h, const void* q, const void* k, const void* v, int64_t n,
                                    int32_t hq, int32_t hkv, const PrefillLayout& lay, const int32_t* row_ptr,
                                    const int32_t* col_idx, void* o, cudaStream_t st);

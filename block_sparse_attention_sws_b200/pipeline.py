@@ -93,16 +93,55 @@ class PrefillPath:
 class PrefillBatch:
     """Prefill of several sequences of different lengths through one handle.
 
-    Each sequence keeps its own PrefillPath (its own walk state and CSR); a
-    layer issues every sequence's sketch, walk and attention on a stream of its
-    own, all ordered after the caller's stream and joined back into it, so the
-    kernels of short sequences overlap on the GPU. Results equal those of the
-    sequences run one by one, bit for bit (tests/test_gpu_prefill.py)."""
+    Each sequence keeps its own PrefillPath (its own walk state and CSR).
+    ``layer`` issues every sequence's sketch, walk and attention on a stream of
+    its own, all ordered after the caller's stream and joined back into it, so
+    the kernels of short sequences overlap on the GPU. ``layer_packed`` takes
+    the sequences end to end along the token axis: the sketches and walks run
+    per sequence on those streams, then one attention launch covers them all
+    (sws_sparse_attn_prefill_varlen). Results equal those of the sequences run
+    one by one, bit for bit (tests/test_gpu_prefill.py)."""
 
     def __init__(self, handle: L.Handle, lengths, hq: int, hkv: int, dtype=torch.bfloat16, device="cuda",
                  dense_layers: int = 0):
         self.paths = [PrefillPath(handle, int(n), hq, hkv, dtype, device, dense_layers) for n in lengths]
         self.streams = [torch.cuda.Stream(device=device) for _ in lengths]
+        self.cu_seqlens = [0]
+        for n in lengths:
+            self.cu_seqlens.append(self.cu_seqlens[-1] + int(n))
+        self.hq, self.dtype, self.device = hq, dtype, device
+        self.ws_var = None
+        self.o_packed = None
+
+    def layer_packed(self, q, k, v, first_layer: bool, out=None, layer=None):
+        """q [hq, N, d], k, v [hkv, N, d]: sequence i on tokens cu_seqlens[i] ..
+        cu_seqlens[i + 1] - 1. Returns the packed output [hq, N, d] (a buffer of
+        the batch unless ``out``)."""
+        cu = self.cu_seqlens
+        cur = torch.cuda.current_stream()
+        ready = torch.cuda.Event()
+        ready.record(cur)
+        for i, (p, st) in enumerate(zip(self.paths, self.streams)):
+            st.wait_event(ready)
+            a, z = cu[i], cu[i + 1]
+            p.sketch(q[:, a:z], k[:, a:z], st)
+            p.walk_select(first_layer, st, layer)
+        for st in self.streams:
+            cur.wait_stream(st)
+        if self.ws_var is None:
+            nb = L.sws_sparse_attn_prefill_varlen_ws_bytes(cu)
+            self.ws_var = torch.empty(max(nb, 16), dtype=torch.uint8, device=self.device)
+        o = out
+        if o is None:
+            if self.o_packed is None:
+                self.o_packed = torch.empty(self.hq, cu[-1], q.shape[2], dtype=self.dtype, device=self.device)
+            o = self.o_packed
+        p0 = self.paths[0]
+        h = p0.h_dense if p0._dense(layer) else p0.h
+        csrs = [p.csr(layer) for p in self.paths]
+        L.sws_sparse_attn_prefill_varlen(h, q, k, v, cu, [c[0] for c in csrs], [c[1] for c in csrs], o, self.ws_var,
+                                         cur)
+        return o
 
     def layer(self, qs, ks, vs, first_layer: bool, outs=None, layer=None):
         """qs[i] [hq, n_i, d], ks[i], vs[i] [hkv, n_i, d]: layer inputs of sequence i.

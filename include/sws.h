@@ -199,6 +199,32 @@ sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const voi
                                    const int64_t o_strides[2], const int32_t* row_ptr, const int32_t* col_idx,
                                    void* o, void* ws, size_t ws_bytes, void* stream);
 
+/* sws_sparse_attn_prefill_varlen. The attention of sws_sparse_attn_prefill over
+ * several sequences in one launch (the batching of prompts of different lengths that
+ * §11.4 asks of serving): the sequences lie end to end along the token axis, sequence
+ * s on rows cu_seqlens[s] .. cu_seqlens[s+1] - 1 of every head, and each is attended
+ * with its own selection. The work of all sequences is one list, longest slabs first,
+ * so short sequences fill the GPU together.
+ *   q (device) [hq, N, d], k, v (device) [hkv, N, d], o (device) [hq, N, d]: bf16,
+ *     N = cu_seqlens[nseq], each with its strides (NULL: dense)
+ *   cu_seqlens (host) [nseq + 1] int64: 0 = cu_seqlens[0] < cu_seqlens[1] < ...,
+ *     N < 2^31
+ *   row_ptr, col_idx (host) arrays of nseq device pointers: sequence s's CSR, as
+ *     sws_walk_select writes it for its n_s = cu_seqlens[s+1] - cu_seqlens[s] tokens
+ *   ws (device, 16-byte aligned) sws_sparse_attn_prefill_varlen_ws_bytes bytes: the
+ *     sequence table and the work list, copied there in stream order by this call
+ * For finite inputs each sequence's rows of o equal, bit for bit, what
+ * sws_sparse_attn_prefill writes for that sequence alone (the same tiles and the same
+ * order of operations; keys past a sequence's end are masked in both). Rows of o
+ * outside every sequence are not written. fp32 returns SWS_ERR_UNSUPPORTED. */
+size_t sws_sparse_attn_prefill_varlen_ws_bytes(int32_t nseq, const int64_t* cu_seqlens);
+sws_status sws_sparse_attn_prefill_varlen(const sws_handle* h, const void* q, const void* k, const void* v,
+                                          sws_dtype dtype, int32_t nseq, const int64_t* cu_seqlens, int32_t hq,
+                                          int32_t hkv, const int64_t q_strides[2], const int64_t k_strides[2],
+                                          const int64_t v_strides[2], const int64_t o_strides[2],
+                                          const int32_t* const* row_ptr, const int32_t* const* col_idx, void* o,
+                                          void* ws, size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------------------- decode --- */
 /* §5: each decode step scores its single new query token against the cached key
  * blocks with the same sketch. The query is a block of one row; cached key blocks are

@@ -107,6 +107,18 @@ def test_workspace_sizes(lib):
         S.sws_workspace_size(cfg, S.SWS_OP_WALK_SELECT, 10, 32, 7)  # hq % hkv != 0
 
 
+def test_packed_prefill_workspace(lib):
+    """The packed attention's workspace: a 48-byte entry per sequence (rounded
+    up to 16 bytes), then 8 bytes per 256-row slab of every sequence; 0 for a
+    list that is not strictly increasing."""
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 300, 1000]) == 96 + 8 * (2 + 3)
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 1]) == 48 + 8
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 256, 512, 513]) == 144 + 8 * (1 + 1 + 1)
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 300, 300]) == 0
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 300, 200]) == 0
+    assert S.sws_sparse_attn_prefill_varlen_ws_bytes([0]) == 0
+
+
 def test_null_handle_rejected_without_launch(lib):
     """Host validation fails before any CUDA call, so this runs without a GPU."""
     P = ctypes.c_void_p
@@ -117,6 +129,10 @@ def test_null_handle_rejected_without_launch(lib):
                                       None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_sparse_attn_prefill(None, P(16), P(16), P(16), 0, 64, 1, 1, None, None, None, None, P(16), P(16),
                                        P(16), None, 0, None) == S.SWS_ERR_INVALID_ARG
+    cu = (ctypes.c_int64 * 3)(0, 300, 1000)
+    ptrs = (ctypes.c_void_p * 2)(16, 32)
+    assert lib.sws_sparse_attn_prefill_varlen(None, P(16), P(16), P(16), 0, 2, cu, 1, 1, None, None, None, None,
+                                              ptrs, ptrs, P(16), P(16), 1 << 10, None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_destroy(None) == S.SWS_ERR_INVALID_ARG
     assert lib.sws_projection_device(None) is None
     assert lib.sws_decode_init_cache_paged(None, P(16), 4, P(16), 4, 1, 1, P(16), P(16), P(16),

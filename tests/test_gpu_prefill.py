@@ -386,3 +386,81 @@ def test_prefill_batch_matches_single_sequences():
             assert torch.equal(bp.walk_state, p.walk_state)
             assert torch.equal(o.view(torch.int16), p.o.view(torch.int16))
     h.close()
+
+
+@pytest.mark.parametrize("w0,strided", [
+    (W.PREFILL_16K.scaled(name="packed_B64", hq=8, hkv=2, layers=2), False),
+    (W.PREFILL_16K.scaled(name="packed_B64_strided", hq=8, hkv=2, layers=2), True),
+    (W.PREFILL_64K.scaled(name="packed_B128_d64", d=64, k=16, hq=4, hkv=2, layers=2), False),
+], ids=lambda x: x.name if hasattr(x, "name") else str(x))
+def test_packed_prefill_matches_single_sequences(w0, strided):
+    """sws_sparse_attn_prefill_varlen through PrefillBatch.layer_packed: five
+    sequences end to end (ragged tails, one shorter than a block, one of exactly
+    two slabs) in one attention launch. Each sequence's rows equal, bit for
+    bit, what its own PrefillPath gives (held to the oracle above), its walk and
+    CSR too; sampled query blocks of every sequence are also compared with the
+    oracle on the packed output. strided: Q, K, V and O are [N, heads, d]
+    activations read and written in place."""
+    lengths = (1000, 2065, 40, 512, 1537)
+    ws = [w0.scaled(name=f"seq{i}", n=n, seed=w0.seed + i) for i, n in enumerate(lengths)]
+    cfg = S.make_config(w0.d, w0.B, w0.k, w0.s, 0, w0.density, w0.seed)
+    h = S.Handle(cfg)
+    batch = S.PrefillBatch(h, lengths, w0.hq, w0.hkv, torch.bfloat16, "cuda")
+    singles = [S.PrefillPath(h, n, w0.hq, w0.hkv, torch.bfloat16, "cuda") for n in lengths]
+    cu = batch.cu_seqlens
+    N = cu[-1]
+
+    def packed(parts):
+        x = torch.cat(parts, dim=1)
+        return x.transpose(0, 1).contiguous().transpose(0, 1) if strided else x
+
+    out = torch.full((N, w0.hq, w0.d), float("nan"), dtype=torch.bfloat16, device="cuda").transpose(0, 1) \
+        if strided else None
+    for layer in range(w0.layers):
+        ins = [W.prefill_layer_inputs(w, layer, "cuda") for w in ws]
+        Q, K, V = (packed([x[j] for x in ins]) for j in range(3))
+        o = batch.layer_packed(Q, K, V, layer == 0, out=out)
+        for p, (q, k, v) in zip(singles, ins):
+            p.layer(q, k, v, layer == 0)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        for i, (bp, p) in enumerate(zip(batch.paths, singles)):
+            assert torch.equal(bp.row_ptr, p.row_ptr) and torch.equal(bp.col_idx, p.col_idx)
+            assert torch.equal(bp.walk_state, p.walk_state)
+            assert torch.equal(o[:, cu[i]:cu[i + 1]].contiguous().view(torch.int16), p.o.view(torch.int16))
+    group = w0.hq // w0.hkv
+    for i, (w, (q, k, v)) in enumerate(zip(ws, ins)):
+        rp = batch.paths[i].row_ptr.cpu().numpy()
+        ci = batch.paths[i].col_idx.cpu().numpy()
+        for hh in (0, w0.hq - 1):
+            Qh, Kg, Vg = LazyHeads(q)[hh], LazyHeads(k)[hh // group], LazyHeads(v)[hh // group]
+            o_gpu = o[hh, cu[i]:cu[i + 1]].float().cpu().numpy()
+            for qb in sorted({0, w.b // 2, w.b - 1}):
+                cols = ci[hh][rp[hh][qb]:rp[hh][qb + 1]]
+                compare_attention(o_gpu[qb * w.B:min(w.n, (qb + 1) * w.B)],
+                                  so.sparse_attention_block(Qh, Kg, Vg, qb, cols, w.B))
+    h.close()
+
+
+def test_packed_prefill_invalid_arguments():
+    """Host validation of the packed launch: nothing is queued."""
+    cfg = S.make_config(128, 64, 32)
+    h = S.Handle(cfg)
+    q = torch.zeros(4, 600, 128, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, 600, 128, dtype=torch.bfloat16, device="cuda")
+    rp = [torch.zeros(4, 8, dtype=torch.int32, device="cuda") for _ in range(2)]
+    ci = [torch.zeros(4, 64, dtype=torch.int32, device="cuda") for _ in range(2)]
+    ws = torch.zeros(S.sws_sparse_attn_prefill_varlen_ws_bytes([0, 300, 600]), dtype=torch.uint8, device="cuda")
+    cases = [
+        ([0, 300, 600], q.float(), kv.float(), ws, S.SWS_ERR_UNSUPPORTED),   # fp32
+        ([1, 300, 600], q, kv, ws, S.SWS_ERR_INVALID_ARG),                   # does not start at 0
+        ([0, 300, 300], q, kv, ws, S.SWS_ERR_INVALID_ARG),                   # an empty sequence
+        ([0, 300, 600], q, kv, ws[:16], S.SWS_ERR_WORKSPACE),                # workspace too small
+    ]
+    for cu, qq, kk, w, want in cases:
+        with pytest.raises(S.SwsError) as e:
+            S.sws_sparse_attn_prefill_varlen(h, qq, kk, kk, cu, rp, ci, torch.zeros_like(qq), w)
+        assert e.value.status == want, cu
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    h.close()
