@@ -215,7 +215,9 @@ __global__ void __launch_bounds__(kRowThreads) exact_append_rows_kernel(
 //  * warp 0 adds block M's rows to the 32 columns of block M - 32 and then
 //    resolves block M - 32's diagonal triangle level by level: u_{l+1}[m] =
 //    part[l][m] + sum over the block's rows m' >= m of u_l[m'] A[m'][m],
-//    publishing u_0 .. u_{L-1} of its rows for the next block's updates;
+//    publishing u_0 .. u_{L-1} of its rows for the next block's updates. The
+//    entries it reads (a row block's 32 x 32 piece and a triangle) are copied
+//    into shared memory two blocks ahead, into buffers of alternating parity;
 //  * the other warps add block M's rows to every column left of block M - 32,
 //    16 columns a warp at a time on the fp64 tensor path (the 8 levels are the
 //    n of an m16n8k4 product, the block's rows its k), the next chunk's rows
@@ -256,8 +258,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
   double* u_in = part + kLevels * mbp;         // [mbp]
   double* u_out = u_in + mbp;                  // [mbp]
   double* ub = u_out + mbp;                    // [2][32][kLevels]: u_l of a block's rows (by block parity)
-  uint32_t* ad = reinterpret_cast<uint32_t*>(ub + 2 * 32 * kLevels);  // [32][33]: a diagonal triangle
-  uint32_t* ar = ad + 32 * 33;                 // [32][32]: a row block's entries in the columns of the block below
+  uint32_t* ad2 = reinterpret_cast<uint32_t*>(ub + 2 * 32 * kLevels);  // [2][32][33]: diagonal triangles
+  uint32_t* ar2 = ad2 + 2 * 32 * 33;           // [2][32][32]: a row block's entries in the columns of the block below
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t unit = blockIdx.x;
   const int bi = static_cast<int>(unit / hq);
@@ -273,13 +275,16 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
   for (int j = tid; j < nb; j += kWalkThreads) u_in[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
   const int mtop = (i / 32) * 32;
 
-  // warp 0 copies into shared memory, asynchronously, the entries its next
+  // warp 0 copies into shared memory, asynchronously, the entries a later
   // step reads: the triangle of block T in ad[r][.] (row T + r; zeros above the
   // diagonal and past the newest row) and, for T < M, the rows of block M in
-  // the columns of block T in ar[r][.]. Issued as soon as the previous step has
-  // read them, so the copies run while the other warps work.
+  // the columns of block T in ar[r][.], into the buffers of T's parity. Issued
+  // two steps ahead of their use (one commit group each), so the copies run
+  // while the chain and the other warps work on the step before.
   auto stage = [&](int T, int M) {
     const int c = T + lane;
+    uint32_t* ad = ad2 + ((T >> 5) & 1) * 32 * 33;
+    uint32_t* ar = ar2 + ((T >> 5) & 1) * 32 * 32;
 #pragma unroll 8
     for (int r = 0; r < 32; ++r) {
       const bool ok = r >= lane && T + r <= i;
@@ -292,6 +297,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         cp_async4(ar + r * 32 + lane, ok ? A + rows_offset(M + r) + c : A, ok);
       }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
   // warp 0: the diagonal triangle of block M (its columns' part complete, its
@@ -300,6 +306,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
     const int m = M + lane;
     const bool live = m <= i;
     double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
+    const uint32_t* ad = ad2 + ((M >> 5) & 1) * 32 * 33;
     double uprev = live ? u_in[m] : 0.0;
     for (int l = 0; l < kLevels; ++l) {
       if (l >= L) {  // levels past this sweep's: zeros, so every product that reads them adds 0
@@ -334,14 +341,19 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
       prefetch_block(mtop - 32);
     }
     for (int x = tid; x < kLevels * mbp; x += kWalkThreads) part[x] = 0.0;
-    if (warp == 0) stage(mtop, mtop);
+    if (warp == 0) {
+      stage(mtop, mtop);
+      if (mtop > 0) stage(mtop - 32, mtop);
+    }
     __syncthreads();
     if (warp == 0) {
-      cp_async_wait_all();
+      if (mtop > 0)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else
+        cp_async_wait_all();
       __syncwarp();
       diag(mtop, L);
       __syncwarp();
-      if (mtop > 0) stage(mtop - 32, mtop);
     }
     __syncthreads();
     for (int M = mtop; M > 0; M -= 32) {
@@ -352,8 +364,15 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         // block M's rows into the columns of block M - 32, then that block's
         // diagonal; both were staged during the previous step
         const int c = M - 32 + lane;
-        cp_async_wait_all();
+        // the next step's entries go out now; this step's, issued a step ago, are waited for
+        if (M - 32 > 0) {
+          stage(M - 64, M - 32);
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+          cp_async_wait_all();
+        }
         __syncwarp();
+        const uint32_t* ar = ar2 + (((M - 32) >> 5) & 1) * 32 * 32;
         double acc[2][kLevels];  // rows of even and odd index, added at the end
 #pragma unroll
         for (int l = 0; l < kLevels; ++l) acc[0][l] = acc[1][l] = 0.0;
@@ -366,8 +385,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         for (int l = 0; l < L; ++l) part[l * mbp + c] += acc[0][l] + acc[1][l];
         __syncwarp();
         diag(M - 32, L);
-        __syncwarp();
-        if (M - 32 > 0) stage(M - 64, M - 32);
       } else {
         // block M's rows into the columns left of block M - 32 on the fp64 tensor
         // path: per 16 columns, D[column][level] += sum over the block's rows r of
@@ -424,7 +441,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
 
 size_t walk_smem_bytes(int64_t max_blocks) {
   const size_t mbp = static_cast<size_t>((max_blocks + 31) & ~int64_t(31));
-  return ((kLevels + 2) * mbp + 2 * 32 * kLevels) * sizeof(double) + (32 * 33 + 32 * 32) * sizeof(uint32_t);
+  return ((kLevels + 2) * mbp + 2 * 32 * kLevels) * sizeof(double) + 2 * (32 * 33 + 32 * 32) * sizeof(uint32_t);
 }
 
 // Step part 3: per head the top-tau of its row (or the group's summed rows for
