@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--profile-prefill", action="store_true",
                     help="profiling run: the headline prefill workload alone (scaled by --prefill-n), no bench line")
     ap.add_argument("--prefill-n", type=int, default=None, help="tokens of the profiled prefill workload")
+    ap.add_argument("--profile-workload", default="headline", choices=sorted(PROFILE_WORKLOADS),
+                    help="the prefill workload --profile-prefill runs")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -314,6 +316,11 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------------- ours ---
+
+# --profile-prefill's choice of workload (attribute names in sws_inputs)
+PROFILE_WORKLOADS = {"headline": "PREFILL_128K", "prefill_128k_d10": "PREFILL_128K_D10", "prefill_64k": "PREFILL_64K",
+                     "prefill_16k": "PREFILL_16K"}
+
 
 def headline_workload(W):
     """The N=1 workload: the longest prefill (131072 tokens, 4 layers) at 20% density."""
@@ -968,7 +975,7 @@ def main():
         return 0
     if args.profile_prefill:
         # profiling run of one prefill workload (for ncu captures): not a benchmark line
-        wp = headline_workload(W)
+        wp = getattr(W, PROFILE_WORKLOADS[args.profile_workload])
         if args.prefill_n:
             wp = wp.scaled(name=f"prefill_n{args.prefill_n}_B{wp.B}_k{wp.k}_L{wp.layers}", n=args.prefill_n)
         px = bench_prefill(args, world, S, W, torch, wp, args.steps)
