@@ -225,6 +225,17 @@ def test_decode_exact_rows_full_context_sampled():
     run_exact(w, [w.n0, w.n0 - 1000], steps=1, check_seqs=[0], mode="rows", check_heads=[0, w.hq - 1])
 
 
+def test_decode_exact_rows_at_the_largest_context():
+    """The largest context the stored-rows walk takes: 2560 blocks of 64
+    (163,840 tokens; the walk's shared memory at its limit), one sequence, four
+    query heads of one KV head, two layers; the step's token is the last of
+    the 2560th block. The first and last head against the oracle's exact
+    recurrence, the union with their bits."""
+    w = W.DECODE_128K.scaled(layers=2, batch=1, hq=4, hkv=1, hubs=4)
+    n0 = 2560 * 64 - 1
+    run_exact(w, [n0], steps=1, mode="rows", check_heads=[0, 3])
+
+
 def test_decode_exact_first_token_of_block():
     """n0 a multiple of B: the first decoded token opens a block of its own,
     whose query sketch is that token's projection."""

@@ -464,3 +464,62 @@ def test_packed_prefill_invalid_arguments():
     torch.cuda.synchronize()
     assert S.sws_sync_check(h) == 0
     h.close()
+
+
+def test_prefill_at_the_largest_walk():
+    """The largest walk the library takes: 8192 key blocks (524,288 tokens at
+    B = 64), two query heads of one KV head, one layer, in the 64 x 64-tile walk
+    products and the general selection kernel.
+    - Sketches and sampled score rows against the oracle.
+    - The walk: A and R are lower-triangular, so the leading m x m block of
+      R = A^s is the s-th power of A's leading m x m block; the oracle's walk on
+      the first 512 blocks is compared with the GPU's, and so is the selection
+      of those rows. The whole of R is lower-triangular and row-stochastic.
+    - Sampled rows past 512: the selection is the top-tau (ties to the lower
+      index) of the GPU's own row of R, and the CSR is valid throughout.
+    - Attention on sampled query blocks against the oracle fed the GPU's CSR."""
+    w = W.PREFILL_16K.scaled(name="b8192_B64", n=8192 * 64, hq=2, hkv=1, layers=1)
+    b, m = w.b, 512
+    assert b == 8192
+    num, den = w.density
+    cfg = S.make_config(w.d, w.B, w.k, w.s, 0, w.density, w.seed)
+    h = S.Handle(cfg)
+    path = S.PrefillPath(h, w.n, w.hq, w.hkv, torch.bfloat16, "cuda")
+    Q, K, V = W.prefill_layer_inputs(w, 0, "cuda")
+    path.layer(Q, K, V, True)
+    torch.cuda.synchronize()
+    assert S.sws_sync_check(h) == 0
+    Hd = oracle.srht_matrix(w.d, w.k, w.seed)
+    Kt = so.sketch_project(so.block_means(LazyHeads(K)[0], w.B), Hd)
+    assert np.allclose(path.k_sk[0].cpu().numpy(), Kt, rtol=1e-6, atol=1e-6 * np.abs(Kt).max())
+    rows = sorted({0, 1, 511, 512, 1023, 1024, 4095, b - 2, b - 1})
+    rp_all, ci_all = path.row_ptr.cpu().numpy(), path.col_idx.cpu().numpy()
+    swaps = []
+    for hh in range(w.hq):
+        Qt = so.sketch_project(so.block_means(LazyHeads(Q)[hh], w.B), Hd)
+        assert np.allclose(path.q_sk[hh].cpu().numpy(), Qt, rtol=1e-6, atol=1e-6 * np.abs(Qt).max())
+        S_or = so.sketch_scores(Qt, Kt)
+        S_gpu = path.scores[hh].cpu().numpy()
+        for i in rows:
+            want, got = S_or[i, :i + 1], S_gpu[i, :i + 1]
+            bound = 1e-3 * np.maximum(np.abs(want), np.sqrt((want ** 2).mean()))
+            assert np.all(np.abs(got - want) <= bound), i
+        R = path.walk_state[hh].cpu().numpy()
+        assert not np.triu(R, 1).any()
+        assert np.allclose(R.sum(axis=1), 1.0, rtol=0, atol=1e-9)
+        R_lead = so.walk_matrix(so.block_attention(S_or[:m, :m]), w.s)
+        compare_walk(R[:m, :m], R_lead)
+        rp, ci = rp_all[hh], ci_all[hh]
+        check_csr_valid(rp, ci, b, num, den)
+        orp, oci = so.select_top_tau(R_lead, num, den)
+        swaps += compare_csr(rp[:m + 1], ci, orp, oci, R_lead)
+        for i in rows:
+            assert np.array_equal(ci[rp[i]:rp[i + 1]], so.top_tau_row(R[i, :i + 1], so.tau_of_row(i, num, den))), i
+        del S_or, S_gpu, R
+        Qh, Kg, Vg = LazyHeads(Q)[hh], LazyHeads(K)[0], LazyHeads(V)[0]
+        o_gpu = path.o[hh].float().cpu().numpy()
+        for i in (0, 4095, b - 1):
+            cols = ci[rp[i]:rp[i + 1]]
+            compare_attention(o_gpu[i * w.B:(i + 1) * w.B], so.sparse_attention_block(Qh, Kg, Vg, i, cols, w.B))
+    record_ties(swaps, compared=w.hq * m)
+    h.close()
