@@ -215,10 +215,12 @@ __global__ void __launch_bounds__(kRowThreads) exact_append_rows_kernel(
 //  * warp 0 adds block M's rows to the 32 columns of block M - 32 and then
 //    resolves block M - 32's diagonal triangle level by level: u_{l+1}[m] =
 //    part[l][m] + sum over the block's rows m' >= m of u_l[m'] A[m'][m],
-//    publishing u_0 .. u_{L-1} of its rows for the next block's updates. The
-//    entries it reads (a row block's 32 x 32 piece and a triangle) are copied
-//    into shared memory two blocks ahead, into buffers of alternating parity;
-//  * the other warps add block M's rows to every column left of block M - 32,
+//    publishing u_0 .. u_{L-1} of its rows for the next block's updates;
+//  * warp 1 loads what the chain reads at the next block (a row block's 32 x 32
+//    piece and the next triangle) into shared memory, into buffers of
+//    alternating parity, sixteen rows at a time, and pulls the rows of
+//    the blocks two ahead into L2;
+//  * warps 2-15 add block M's rows to every column left of block M - 32,
 //    16 columns a warp at a time on the fp64 tensor path (the 8 levels are the
 //    n of an m16n8k4 product, the block's rows its k), the next chunk's rows
 //    loaded while the current chunk's products run, then one update of part.
@@ -234,13 +236,6 @@ __device__ __forceinline__ void dmma_16x8x4(double (&c)[4], double a0, double a1
       : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3])
       : "d"(a0), "d"(a1), "d"(b0));
 }
-
-// 4-byte asynchronous copy into shared memory; valid == false writes zero and reads nothing.
-__device__ __forceinline__ void cp_async4(uint32_t* dst, const uint32_t* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Pulls `bytes` (a multiple of 16, from a 16-byte aligned address) into L2; no registers, no completion.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -275,29 +270,33 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
   for (int j = tid; j < nb; j += kWalkThreads) u_in[j] = first_layer ? (j == i ? 1.0 : 0.0) : wrow[j];
   const int mtop = (i / 32) * 32;
 
-  // warp 0 copies into shared memory, asynchronously, the entries a later
-  // step reads: the triangle of block T in ad[r][.] (row T + r; zeros above the
-  // diagonal and past the newest row) and, for T < M, the rows of block M in
-  // the columns of block T in ar[r][.], into the buffers of T's parity. Issued
-  // two steps ahead of their use (one commit group each), so the copies run
-  // while the chain and the other warps work on the step before.
+  // warp 1 loads into shared memory the entries the chain's next step reads:
+  // the triangle of block T in ad[r][.] (row T + r; zeros above the diagonal
+  // and past the newest row) and, for T < M, the rows of block M in the
+  // columns of block T in ar[r][.], into the buffers of T's parity, which the
+  // chain last read a step earlier.
   auto stage = [&](int T, int M) {
     const int c = T + lane;
     uint32_t* ad = ad2 + ((T >> 5) & 1) * 32 * 33;
     uint32_t* ar = ar2 + ((T >> 5) & 1) * 32 * 32;
-#pragma unroll 8
-    for (int r = 0; r < 32; ++r) {
-      const bool ok = r >= lane && T + r <= i;
-      cp_async4(ad + r * 33 + lane, ok ? A + rows_offset(T + r) + c : A, ok);
+    uint32_t v[16];  // sixteen rows' entries in flight at once
+#pragma unroll
+    for (int h = 0; h < 32; h += 16) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        v[r] = (h + r >= lane && T + h + r <= i) ? __ldg(A + rows_offset(T + h + r) + c) : 0u;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) ad[(h + r) * 33 + lane] = v[r];
     }
     if (T < M) {
-#pragma unroll 8
-      for (int r = 0; r < 32; ++r) {
-        const bool ok = M + r <= i;
-        cp_async4(ar + r * 32 + lane, ok ? A + rows_offset(M + r) + c : A, ok);
+#pragma unroll
+      for (int h = 0; h < 32; h += 16) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) v[r] = M + h + r <= i ? __ldg(A + rows_offset(M + h + r) + c) : 0u;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) ar[(h + r) * 32 + lane] = v[r];
       }
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
   // warp 0: the diagonal triangle of block M (its columns' part complete, its
@@ -314,14 +313,14 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         continue;
       }
       ubm[lane * kLevels + l] = uprev;
-      // four interleaved partial sums (rows r = 3, 2, 1, 0 mod 4), added in a fixed order
-      double acc[4] = {live ? part[l * mbp + m] : 0.0, 0.0, 0.0, 0.0};
+      // eight interleaved partial sums (rows r mod 8), added in a fixed order
+      double acc[8] = {live ? part[l * mbp + m] : 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
       for (int r = 31; r >= 0; --r) {
         const double v = __shfl_sync(0xffffffffu, uprev, r);
-        acc[r & 3] = fma(v, from_hi(ad[r * 33 + lane]), acc[r & 3]);
+        acc[r & 7] = fma(v, from_hi(ad[r * 33 + lane]), acc[r & 7]);
       }
-      uprev = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      uprev = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     }
     if (live) u_out[m] = uprev;
   };
@@ -341,37 +340,24 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
       prefetch_block(mtop - 32);
     }
     for (int x = tid; x < kLevels * mbp; x += kWalkThreads) part[x] = 0.0;
-    if (warp == 0) {
+    if (warp == 1) {
       stage(mtop, mtop);
       if (mtop > 0) stage(mtop - 32, mtop);
     }
     __syncthreads();
-    if (warp == 0) {
-      if (mtop > 0)
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      else
-        cp_async_wait_all();
-      __syncwarp();
-      diag(mtop, L);
-      __syncwarp();
-    }
+    if (warp == 0) diag(mtop, L);
     __syncthreads();
     for (int M = mtop; M > 0; M -= 32) {
       const int nrows = min(32, i - M + 1);
       const double* ubm = ub + ((M >> 5) & 1) * 32 * kLevels;
-      if (warp == 1) prefetch_block(M - 64);
-      if (warp == 0) {
+      if (warp == 1) {
+        // the entries the chain reads at the next block, staged while it works on this one
+        prefetch_block(M - 64);
+        if (M - 32 > 0) stage(M - 64, M - 32);
+      } else if (warp == 0) {
         // block M's rows into the columns of block M - 32, then that block's
         // diagonal; both were staged during the previous step
         const int c = M - 32 + lane;
-        // the next step's entries go out now; this step's, issued a step ago, are waited for
-        if (M - 32 > 0) {
-          stage(M - 64, M - 32);
-          asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-          cp_async_wait_all();
-        }
-        __syncwarp();
         const uint32_t* ar = ar2 + (((M - 32) >> 5) & 1) * 32 * 32;
         double acc[2][kLevels];  // rows of even and odd index, added at the end
 #pragma unroll
@@ -393,7 +379,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
         // Lane (g, t4) holds A at rows 4 kk + t4, columns g and g + 8 of the chunk.
         const int g = lane >> 2, t4 = lane & 3;
         const int nchunk = (M - 32) / 16;
-        const int wk = warp - 1;
+        const int wk = warp - 2;
         uint32_t cur[8][2], nxt[8][2];
         auto load_chunk = [&](int ch, uint32_t (&dst)[8][2]) {
           const int c0 = 16 * ch;
@@ -407,8 +393,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) exact_walk_kernel(
           }
         };
         if (wk < nchunk) load_chunk(wk, cur);
-        for (int ch = wk; ch < nchunk; ch += kWalkWarps - 1) {
-          const int nc = ch + kWalkWarps - 1;
+        for (int ch = wk; ch < nchunk; ch += kWalkWarps - 2) {
+          const int nc = ch + kWalkWarps - 2;
           if (nc < nchunk) load_chunk(nc, nxt);
           double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
