@@ -560,23 +560,31 @@ def bench_prefill_variants(args, world, S, W, torch, pf):
             path.h_dense.close()
         del path
     out["batch_8x2048"] = bench_prefill_batch(args, world, S, W, torch)
+    out["batch_mixed_lengths"] = bench_prefill_batch(args, world, S, W, torch, MIXED_LENGTHS)
     return out
 
 
-def bench_prefill_batch(args, world, S, W, torch):
-    """Prefill batching: eight 2048-token sequences of the headline workload's
-    shape (4 layers, 32/8 heads), through PrefillBatch: each sequence's layer
-    on its own stream; the sequences packed end to end with one attention
-    launch for all (the sketches and walks on their streams); and, for
-    comparison, the same paths one after another on one stream."""
+# sequence lengths of the mixed prefill batch (tokens; 33,276 in all)
+MIXED_LENGTHS = (8192, 6144, 4096, 3000, 2048, 2048, 1536, 1024, 1024, 2900, 700, 564)
+
+
+def bench_prefill_batch(args, world, S, W, torch, lengths=None):
+    """Prefill batching: eight 2048-token sequences (or the given lengths) of the
+    headline workload's shape (4 layers, 32/8 heads), through PrefillBatch:
+    each sequence's layer on its own stream; the sequences packed end to end
+    with one attention launch for all (the sketches and walks on their
+    streams); and, for comparison, the same paths one after another on one
+    stream."""
     base = W.PREFILL_16K
-    ws = [base.scaled(name=f"seq{i}", n=2048, seed=base.seed + 100 + i) for i in range(8)]
+    lengths = (2048,) * 8 if lengths is None else tuple(lengths)
+    ws = [base.scaled(name=f"seq{i}", n=n, seed=base.seed + 100 + i) for i, n in enumerate(lengths)]
     inputs = [[W.prefill_layer_inputs(w, layer, "cuda") for w in ws] for layer in range(base.layers)]
     h = S.Handle(S.make_config(base.d, base.B, base.k, base.s, 0, base.density, base.seed))
     batch = S.PrefillBatch(h, [w.n for w in ws], base.hq, base.hkv, torch.bfloat16)
     stream = torch.cuda.current_stream()
     steps = max(3, min(args.steps, 20))
-    out = {"sequences": len(ws), "tokens_per_sequence": 2048, "steps": steps}
+    out = {"sequences": len(ws), "tokens_per_sequence": list(lengths) if len(set(lengths)) > 1 else lengths[0],
+           "steps": steps}
     packed = [[torch.cat([x[j] for x in ins], dim=1) for j in range(3)] for ins in inputs]
     for mode in ("concurrent_streams", "packed_launch", "one_stream"):
         def step():
