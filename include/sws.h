@@ -216,7 +216,9 @@ sws_status sws_sparse_attn_prefill(const sws_handle* h, const void* q, const voi
  * For finite inputs each sequence's rows of o equal, bit for bit, what
  * sws_sparse_attn_prefill writes for that sequence alone (the same tiles and the same
  * order of operations; keys past a sequence's end are masked in both). Rows of o
- * outside every sequence are not written. fp32 returns SWS_ERR_UNSUPPORTED. */
+ * outside every sequence are not written. fp32 returns SWS_ERR_UNSUPPORTED.
+ * The tables are copied from pageable host memory, so a stream that is being
+ * captured into a CUDA graph rejects the call (SWS_ERR_CUDA). */
 size_t sws_sparse_attn_prefill_varlen_ws_bytes(int32_t nseq, const int64_t* cu_seqlens);
 sws_status sws_sparse_attn_prefill_varlen(const sws_handle* h, const void* q, const void* k, const void* v,
                                           sws_dtype dtype, int32_t nseq, const int64_t* cu_seqlens, int32_t hq,
