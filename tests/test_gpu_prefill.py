@@ -523,3 +523,32 @@ def test_prefill_at_the_largest_walk():
             compare_attention(o_gpu[i * w.B:(i + 1) * w.B], so.sparse_attention_block(Qh, Kg, Vg, i, cols, w.B))
     record_ties(swaps, compared=w.hq * m)
     h.close()
+
+
+def test_packed_prefill_with_dense_layers_and_shared_selection():
+    """The packed launch under the dense-first-layers policy (layer 0 through a
+    density-1/1 handle) and group-shared selection: each sequence's rows equal
+    its own PrefillPath's, bit for bit, over three layers."""
+    w0 = W.PREFILL_16K.scaled(name="packed_policy", hq=8, hkv=2, layers=3)
+    lengths = (1500, 333, 2100)
+    ws = [w0.scaled(name=f"seq{i}", n=n, seed=w0.seed + 10 + i) for i, n in enumerate(lengths)]
+    cfg = S.make_config(w0.d, w0.B, w0.k, w0.s, 0, w0.density, w0.seed, select_group=w0.hq // w0.hkv)
+    h = S.Handle(cfg)
+    batch = S.PrefillBatch(h, lengths, w0.hq, w0.hkv, torch.bfloat16, "cuda", dense_layers=1)
+    singles = [S.PrefillPath(h, n, w0.hq, w0.hkv, torch.bfloat16, "cuda", dense_layers=1) for n in lengths]
+    cu = batch.cu_seqlens
+    for layer in range(w0.layers):
+        ins = [W.prefill_layer_inputs(w, layer, "cuda") for w in ws]
+        Q, K, V = (torch.cat([x[j] for x in ins], dim=1) for j in range(3))
+        o = batch.layer_packed(Q, K, V, layer == 0, layer=layer)
+        for p, (q, k, v) in zip(singles, ins):
+            p.layer(q, k, v, layer == 0, layer=layer)
+        torch.cuda.synchronize()
+        assert S.sws_sync_check(h) == 0
+        for i, (bp, p) in enumerate(zip(batch.paths, singles)):
+            rp_b, ci_b = bp.csr(layer)
+            rp_s, ci_s = p.csr(layer)
+            assert torch.equal(rp_b, rp_s) and torch.equal(ci_b, ci_s)
+            assert torch.equal(bp.walk_state, p.walk_state)
+            assert torch.equal(o[:, cu[i]:cu[i + 1]].contiguous().view(torch.int16), p.o.view(torch.int16))
+    h.close()
