@@ -44,7 +44,9 @@ constexpr int kPoolBatch = 16;  // 16-byte loads in flight per lane
 // registers, then over the lane bits with xor shuffles; lane j fetches
 // transform entry col_j and scales it by scale / rows (the mean divides the
 // sums by the rows the block holds).
-template <typename T, int D>
+// kDense: Q and K are dense [heads, n, D] (the strides are then compile-time
+// constants and the row addressing a shift).
+template <typename T, int D, bool kDense>
 __global__ void __launch_bounds__(kPoolWarps * 32, 2)
     pool_project_kernel(const T* __restrict__ q, const T* __restrict__ k, int64_t n, int32_t hq, int32_t hkv,
                         HeadTok qs, HeadTok ks, int32_t B, int64_t nblk, const double* __restrict__ sign,
@@ -77,8 +79,9 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 2)
     const int64_t head = it / nblk, blk = it % nblk;
     const int64_t r0 = blk * B;
     const int rows = static_cast<int>(n - r0 < B ? n - r0 : (int64_t)B);
-    const int64_t rs = head < hq ? qs.tok : ks.tok;  // elements from one row to the next
-    const T* src = (head < hq ? q + head * qs.head : k + (head - hq) * ks.head) + r0 * rs + vc * VE;
+    const int64_t rs = kDense ? D : (head < hq ? qs.tok : ks.tok);  // elements from one row to the next
+    const int64_t hs = kDense ? n * D : (head < hq ? qs.head : ks.head);
+    const T* src = (head < hq ? q + head * hs : k + (head - hq) * hs) + r0 * rs + vc * VE;
 
     double acc[VE];
 #pragma unroll
@@ -255,9 +258,11 @@ cudaError_t launch_pool_project(const sws_handle* h, const T* q, const T* k, int
   const int64_t nblk = ceil_div64(n, B);
   const int64_t total = (int64_t)(hq + hkv) * nblk;
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div64(total, kPoolWarps), 2 * (int64_t)h->num_sms));
+  const bool dense = qs.tok == D && ks.tok == D && qs.head == n * D && ks.head == n * D;
   {
-    const cudaError_t le = launch_k(pool_project_kernel<T, D>, grid, kPoolWarps * 32, 0, st, q, k, n, hq, hkv, qs, ks,
-                                    B, nblk, h->sign, h->col, h->scale, h->cfg.sketch_dim, q_sk, k_sk);
+    const cudaError_t le =
+        launch_k(dense ? pool_project_kernel<T, D, true> : pool_project_kernel<T, D, false>, grid, kPoolWarps * 32, 0,
+                 st, q, k, n, hq, hkv, qs, ks, B, nblk, h->sign, h->col, h->scale, h->cfg.sketch_dim, q_sk, k_sk);
     if (le != cudaSuccess) return le;
   }
   note_launches(1);
